@@ -1,0 +1,223 @@
+"""fp4q oracle: the plain CPU restatement of block-scaled 4-bit quantization.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
+and its Python binding never import, link or call it, and it imports nothing
+from them.
+
+The arithmetic lives in ``fp4q_oracle.c`` (scalar loops, IEEE binary32 /
+binary64, no fast-math); this module is a numpy/ctypes wrapper around it.  The
+header comment of the C file lists the page passages it follows and the
+readings it takes where the pages are silent.  Functions whose result is not
+pinned by an independent check are marked "parity unpinned" in their
+docstring; at present every function is pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+NVFP4, NVFP4_RAZER, MXFP4 = 0, 1, 2
+FORMAT_NAMES = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4q_oracle.c")
+_LIB = os.path.join(_HERE, "libfp4q_oracle.so")
+CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-shared", "-fPIC", "-pthread"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library in place (gcc) and return its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        i64, i32, f32, f64 = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double
+        vp = ctypes.c_void_p
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]; L.orc_bf16_to_f32.restype = f32
+        L.orc_f32_to_bf16.argtypes = [f32]; L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_e2m1_value.argtypes = [i32]; L.orc_e2m1_value.restype = f64
+        L.orc_e2m1_encode.argtypes = [f32]; L.orc_e2m1_encode.restype = i32
+        L.orc_e4m3_value.argtypes = [i32]; L.orc_e4m3_value.restype = f64
+        L.orc_e4m3_encode.argtypes = [f32]; L.orc_e4m3_encode.restype = i32
+        L.orc_e8m0_value.argtypes = [i32]; L.orc_e8m0_value.restype = f64
+        L.orc_mx_exponent.argtypes = [f32]; L.orc_mx_exponent.restype = i32
+        L.orc_hadamard_entry.argtypes = [i32, i32]; L.orc_hadamard_entry.restype = i32
+        L.orc_wht_constant.argtypes = []; L.orc_wht_constant.restype = f32
+        L.orc_wht32.argtypes = [vp, vp]; L.orc_wht32.restype = None
+        L.orc_tensor_amax.argtypes = [vp, i64, i64, i64, i32, i32]; L.orc_tensor_amax.restype = f32
+        L.orc_tensor_scale_from_amax.argtypes = [f32]; L.orc_tensor_scale_from_amax.restype = f32
+        L.orc_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, i32]
+        L.orc_quantize.restype = i32
+        L.orc_dequantize.argtypes = [vp, vp, f32, i64, i64, i32, i32, vp, vp, i64, i32]
+        L.orc_dequantize.restype = i32
+        L.orc_error.argtypes = [vp, i64, vp, vp, f32, i64, i64, i32, i32, vp, i32]
+        L.orc_error.restype = i32
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _fmt(fmt) -> int:
+    return FORMAT_NAMES[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def block_size(fmt) -> int:
+    return 32 if _fmt(fmt) == MXFP4 else 16
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+# ---- scalar format helpers (each pinned by enumeration in the tests) --------
+
+def e2m1_value(code: int) -> float:
+    return lib().orc_e2m1_value(int(code))
+
+
+def e2m1_encode(v: float) -> int:
+    return lib().orc_e2m1_encode(float(v))
+
+
+def e4m3_value(byte: int) -> float:
+    return lib().orc_e4m3_value(int(byte))
+
+
+def e4m3_encode(t: float) -> int:
+    return lib().orc_e4m3_encode(float(t))
+
+
+def e8m0_value(byte: int) -> float:
+    return lib().orc_e8m0_value(int(byte))
+
+
+def mx_exponent(a: float) -> int:
+    return lib().orc_mx_exponent(float(a))
+
+
+def hadamard_entry(i: int, j: int) -> int:
+    return lib().orc_hadamard_entry(int(i), int(j))
+
+
+def wht_constant() -> float:
+    return lib().orc_wht_constant()
+
+
+def wht32(x) -> np.ndarray:
+    """Rotated 32-group, RN_f32(RN_f32(H x) * c)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32).reshape(32))
+    out = np.empty(32, dtype=np.float32)
+    lib().orc_wht32(_ptr(a), _ptr(out))
+    return out
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float32).ravel()
+    L = lib()
+    return np.array([L.orc_f32_to_bf16(float(v)) for v in a], dtype=np.uint16).reshape(np.shape(x))
+
+
+# ---- tensor entry points ------------------------------------------------------
+
+def _as_bf16_bits(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (uint16)")
+    if x.ndim != 2:
+        raise ValueError("expected a 2-D matrix")
+    if x.strides[1] != 2:
+        raise ValueError("rows must be contiguous")
+    return x
+
+
+def tensor_amax(x: np.ndarray, rotate: bool = False, nthreads: int | None = None) -> float:
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    return lib().orc_tensor_amax(_ptr(x), rows, cols, x.strides[0] // 2, int(rotate),
+                                 nthreads or default_threads())
+
+
+def tensor_scale_from_amax(amax: float) -> float:
+    return lib().orc_tensor_scale_from_amax(float(amax))
+
+
+def quantize(x: np.ndarray, fmt, rotate: bool = False, tensor_scale: float | None = None,
+             want_sse: bool = True, nthreads: int | None = None):
+    """Quantize a bf16 matrix (uint16 bit patterns, rows contiguous).
+
+    Returns ``(codes[rows, cols/2] u8, scales[rows, cols/B] u8, tensor_scale
+    f32, sse f64 or None)``.  ``tensor_scale`` given means the NVFP4 tensor
+    scale is an input (no absmax pass); it is ignored for MXFP4.
+    """
+    x = _as_bf16_bits(x)
+    f = _fmt(fmt)
+    rows, cols = x.shape
+    B = block_size(f)
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // B), dtype=np.uint8)
+    ts = np.array([tensor_scale if tensor_scale is not None else 0.0], dtype=np.float32)
+    sse = np.zeros(1, dtype=np.float64)
+    rc = lib().orc_quantize(_ptr(x), rows, cols, x.strides[0] // 2, f, int(rotate),
+                            int(tensor_scale is not None), _ptr(ts), _ptr(codes), _ptr(scales),
+                            _ptr(sse) if want_sse else None, nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle rejected shape {x.shape} for format {fmt} rotate={rotate}")
+    return codes, scales, np.float32(ts[0]), (float(sse[0]) if want_sse else None)
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, tensor_scale: float, fmt,
+               rotate: bool = False, nthreads: int | None = None):
+    """Return ``(y_f32, y_bf16_bits)``, the reconstruction before and after bf16 rounding."""
+    f = _fmt(fmt)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    y32 = np.empty((rows, cols), dtype=np.float32)
+    y16 = np.empty((rows, cols), dtype=np.uint16)
+    rc = lib().orc_dequantize(_ptr(codes), _ptr(scales), float(tensor_scale), rows, cols, f,
+                              int(rotate), _ptr(y32), _ptr(y16), cols,
+                              nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected shape")
+    return y32, y16
+
+
+def error(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, tensor_scale: float, fmt,
+          rotate: bool = False, nthreads: int | None = None) -> float:
+    """Sum of squared errors of the reconstruction against ``x`` (original domain)."""
+    x = _as_bf16_bits(x)
+    f = _fmt(fmt)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = x.shape
+    sse = np.zeros(1, dtype=np.float64)
+    rc = lib().orc_error(_ptr(x), x.strides[0] // 2, _ptr(codes), _ptr(scales),
+                         float(tensor_scale), rows, cols, f, int(rotate), _ptr(sse),
+                         nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected shape")
+    return float(sse[0])

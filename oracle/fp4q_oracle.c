@@ -1,0 +1,556 @@
+/*
+ * fp4q oracle -- plain, slow, scalar CPU implementation of block-scaled 4-bit
+ * quantize / dequantize / error (NVFP4, NVFP4 with RaZeR redundant-zero
+ * remapping, MXFP4, each optionally after a 32-point Walsh-Hadamard rotation).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
+ * this file; only the test suite, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or constant with the
+ * CUDA library: every number below is restated here from the pages' text.
+ *
+ * Sources (title, section):
+ *  [RaZeR]  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant
+ *           Zero Remapping", technical summary sect. 1 (E2M1 value set, E4M3
+ *           block scale with an unused sign bit) and sect. 2.2 (the redundant
+ *           -0 code remapped to a special value, chosen per block by minimum
+ *           squared error; one free bit for activations = one pair; +-5).
+ *  [TORQ]   "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization",
+ *           technical summary sect. 1 (32-element blocks sharing one exponent
+ *           scale, e2m1 codebook) and sect. 2 (orthogonal intra-block rotation,
+ *           "S-step" scale from the block maximum, rotations absorbed into the
+ *           neighbouring weights).
+ *
+ * Readings where the pages are silent (each one restated where it is used):
+ *  R1 element rounding: nearest E2M1 value, ties to the even code, |v| > 6
+ *     saturates to 6, a zero result is always +0 (code 0b0000).
+ *  R2 NVFP4 is two-level: a per-tensor fp32 scale s_t = RN(A / (6*448)) with A
+ *     the tensor absmax, then per 16-block an E4M3 scale (round to nearest
+ *     even, saturating at 448).  Elements are encoded as RN(y * r) with
+ *     r = RN(1 / RN(dec(sb) * s_t)).
+ *  R3 MXFP4 scale: e = floor(log2(block absmax)) - 2, clamped to [-127, 127],
+ *     stored as the E8M0 byte e + 127.
+ *  R4 RaZeR (activation mode): the pair {+5, -5}; the scale sign bit selects
+ *     -5; choose -5 only if it lowers the block's squared error strictly more
+ *     than +5 does; the regular code wins ties between an element's regular
+ *     value and the special value.
+ *  R5 rotation: y = RN_f32(RN_f32(H32 x) * RN_f32(1/sqrt(32))) with H32 the
+ *     Sylvester-ordered +-1 Hadamard matrix; the sum is taken in double.
+ *  R6 layout: codes row-major, element 2k in the low nibble of byte k; scales
+ *     dense row-major [rows][cols / block].
+ *
+ * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC
+ * -pthread.  Floating point is IEEE binary32/binary64 with round-to-nearest
+ * and no flush-to-zero, as on any x86-64 / aarch64 host without fast-math.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_NVFP4 0
+#define ORC_NVFP4_RAZER 1
+#define ORC_MXFP4 2
+
+/* ------------------------------------------------------------------------ */
+/* bf16 and fp32 bit helpers                                                 */
+/* ------------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 is the upper half of a binary32; widening is exact. */
+float orc_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* binary32 -> bf16, round to nearest, ties to even (inputs are finite). */
+uint16_t orc_f32_to_bf16(float f)
+{
+    uint32_t u = bits_from_f32(f);
+    uint32_t lower = u & 0xFFFFu;
+    uint32_t upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 element format  [RaZeR sect. 1: {+-0,+-0.5,+-1,+-1.5,+-2,+-3,+-4,+-6}] */
+/* code bit 3 = sign, bits 0..2 = index into the magnitude list below.       */
+/* ------------------------------------------------------------------------ */
+
+static const double E2M1_MAGNITUDE[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double orc_e2m1_value(int code)
+{
+    double m = E2M1_MAGNITUDE[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* R1: nearest magnitude, ties to the even index, saturating at 6.  The
+ * thresholds are the midpoints of neighbouring magnitudes; at a midpoint the
+ * comparison sends the value to whichever neighbour has the even index
+ * (0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4). */
+int orc_e2m1_encode(float v)
+{
+    double a = fabs((double)v);
+    int m;
+    if (a <= 0.25) m = 0;
+    else if (a < 0.75) m = 1;
+    else if (a <= 1.25) m = 2;
+    else if (a < 1.75) m = 3;
+    else if (a <= 2.5) m = 4;
+    else if (a < 3.5) m = 5;
+    else if (a <= 5.0) m = 6;
+    else m = 7;
+    if (m == 0) return 0;              /* zero is always +0 */
+    return (v < 0.0f) ? (8 | m) : m;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 E4M3 block scale  [RaZeR sect. 1: the block scale is an FP8-E4M3       */
+/* value; it is always positive, so its sign bit is free]                    */
+/* bias 7; exponent field 0 = subnormal (m * 2^-9); 0x7F / 0xFF are NaN.     */
+/* ------------------------------------------------------------------------ */
+
+double orc_e4m3_value(int byte)
+{
+    int s = (byte >> 7) & 1, e = (byte >> 3) & 15, m = byte & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* R2: round a non-negative fp32 to E4M3, nearest, ties to even mantissa,
+ * saturating at 448 (byte 0x7E); never produces NaN.  Direct arithmetic:
+ * split t = f * 2^k with f in [1, 2), round (f - 1) * 8 to an integer. */
+int orc_e4m3_encode(float t)
+{
+    double x = (double)t;
+    if (!(x > 0.0)) return 0;
+    if (x >= 448.0) return 0x7E;
+    int k;
+    double f = frexp(x, &k);       /* x = f * 2^k, f in [0.5, 1) */
+    k -= 1;                        /* x = (2f) * 2^k, 2f in [1, 2) */
+    if (k < -6) {                  /* subnormal range: quantum 2^-9 */
+        double q = x / ldexp(1.0, -9);
+        double r = floor(q);
+        double frac = q - r;
+        if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+        /* r == 8 is the smallest normal, exponent field 1, mantissa 0 */
+        return (int)r;             /* r in [0, 8]; 8 encodes as 0x08 */
+    }
+    double q = (2.0 * f - 1.0) * 8.0;  /* mantissa in units of 1/8 */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    int mant = (int)r, ex = k + 7;
+    if (mant == 8) { mant = 0; ex += 1; }
+    if (ex > 15 || (ex == 15 && mant > 6)) return 0x7E;
+    return (ex << 3) | mant;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E8M0 shared exponent  [TORQ sect. 1: MXFP4 = 32-element blocks sharing an   */
+/* exponent scale].  byte b stands for 2^(b - 127); 0xFF is NaN.             */
+/* ------------------------------------------------------------------------ */
+
+double orc_e8m0_value(int byte)
+{
+    if ((byte & 255) == 255) return NAN;
+    return ldexp(1.0, (byte & 255) - 127);
+}
+
+/* R3: e = floor(log2 a) - 2 for a > 0 (2 = exponent of the largest E2M1
+ * magnitude, 6 = 1.5 * 2^2), clamped to [-127, 127].  frexp is exact. */
+int orc_mx_exponent(float a)
+{
+    int k;
+    (void)frexp((double)a, &k);    /* a = f * 2^k, f in [0.5, 1) => floor(log2 a) = k - 1 */
+    int e = (k - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 32-point Walsh-Hadamard rotation  [TORQ sect. 2: an orthogonal rotation     */
+/* inside each block; R5 fixes it to the Sylvester Hadamard matrix / sqrt 32]  */
+/* ------------------------------------------------------------------------ */
+
+static int popcount5(int v) { int c = 0; for (int b = 0; b < 5; ++b) c += (v >> b) & 1; return c; }
+
+/* entry (i, j) of the Sylvester-ordered 32x32 Hadamard matrix */
+int orc_hadamard_entry(int i, int j) { return (popcount5(i & j) & 1) ? -1 : 1; }
+
+float orc_wht_constant(void) { return (float)(1.0 / sqrt(32.0)); }
+
+/* out_i = RN_f32( RN_f32( sum_j H_ij in_j ) * c ), the sum in double.
+ * H / sqrt(32) is symmetric and orthogonal, so the same call inverts it. */
+void orc_wht32(const float* in, float* out)
+{
+    const float c = orc_wht_constant();
+    float tmp[32];
+    for (int i = 0; i < 32; ++i) {
+        double s = 0.0;
+        for (int j = 0; j < 32; ++j)
+            s += orc_hadamard_entry(i, j) * (double)in[j];
+        tmp[i] = (float)s;
+    }
+    for (int i = 0; i < 32; ++i) out[i] = tmp[i] * c;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Row helpers                                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Load one row as fp32, rotated in 32-groups when asked. */
+static void load_row(const uint16_t* x, int64_t cols, int rotate, float* y)
+{
+    for (int64_t j = 0; j < cols; ++j) y[j] = orc_bf16_to_f32(x[j]);
+    if (rotate)
+        for (int64_t g = 0; g < cols; g += 32) {
+            float t[32];
+            orc_wht32(y + g, t);
+            memcpy(y + g, t, sizeof t);
+        }
+}
+
+static int block_size(int fmt) { return fmt == ORC_MXFP4 ? 32 : 16; }
+
+/* ------------------------------------------------------------------------ */
+/* Tensor absmax (NVFP4 first level, R2)                                      */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t* x; int64_t r0, r1, cols, ldx; int rotate; float amax;
+} amax_job;
+
+static void* amax_worker(void* p)
+{
+    amax_job* j = (amax_job*)p;
+    float* y = (float*)malloc(sizeof(float) * (size_t)j->cols);
+    float m = 0.0f;
+    for (int64_t r = j->r0; r < j->r1; ++r) {
+        load_row(j->x + r * j->ldx, j->cols, j->rotate, y);
+        for (int64_t c = 0; c < j->cols; ++c) {
+            float a = fabsf(y[c]);
+            if (a > m) m = a;
+        }
+    }
+    free(y);
+    j->amax = m;
+    return NULL;
+}
+
+float orc_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
+                      int rotate, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = (int)rows;
+    amax_job* jobs = (amax_job*)calloc((size_t)nthreads, sizeof(amax_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = (amax_job){x, rows * t / nthreads, rows * (t + 1) / nthreads, cols, ldx, rotate, 0.0f};
+        pthread_create(&th[t], NULL, amax_worker, &jobs[t]);
+    }
+    float m = 0.0f;
+    for (int t = 0; t < nthreads; ++t) {
+        pthread_join(th[t], NULL);
+        if (jobs[t].amax > m) m = jobs[t].amax;
+    }
+    free(jobs); free(th);
+    return m;
+}
+
+/* R2: s_t maps the tensor maximum onto the largest E2M1 value (6) times the
+ * largest E4M3 value (448). */
+float orc_tensor_scale_from_amax(float amax) { return amax / 2688.0f; }
+
+/* ------------------------------------------------------------------------ */
+/* Block decode: the fp32 reconstruction of one element                      */
+/* ------------------------------------------------------------------------ */
+
+/* NVFP4 / RaZeR: den = RN(dec(sb) * s_t); x^ = RN(value(code) * den).  Under
+ * RaZeR the magnitude of the scale is the low 7 bits and code 0b1000 stands
+ * for +5 (scale bit 7 clear) or -5 (bit 7 set)  [RaZeR sect. 2.2]. */
+static float nv_den(int fmt, int sbyte, float s_t)
+{
+    double sv = orc_e4m3_value(fmt == ORC_NVFP4_RAZER ? (sbyte & 0x7F) : sbyte);
+    return (float)sv * s_t;
+}
+
+static float nv_decode(int fmt, int code, int sbyte, float den)
+{
+    double q;
+    if (fmt == ORC_NVFP4_RAZER && code == 8) q = (sbyte & 0x80) ? -5.0 : 5.0;
+    else q = orc_e2m1_value(code);
+    return (float)q * den;
+}
+
+static float mx_decode(int code, int sbyte)
+{
+    return (float)(orc_e2m1_value(code) * orc_e8m0_value(sbyte));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize one row                                                           */
+/* ------------------------------------------------------------------------ */
+
+static void set_code(uint8_t* row_codes, int64_t j, int code)
+{
+    uint8_t* b = row_codes + (j >> 1);
+    if (j & 1) *b = (uint8_t)((*b & 0x0F) | (code << 4));
+    else       *b = (uint8_t)((*b & 0xF0) | code);
+}
+
+static int get_code(const uint8_t* row_codes, int64_t j)
+{
+    uint8_t b = row_codes[j >> 1];
+    return (j & 1) ? (b >> 4) : (b & 0x0F);
+}
+
+/* RaZeR selection for one 16-block given the scaled values v[] and the
+ * regular codes q[] (R4).  Squared errors are formed in double; every
+ * difference involved is exact in binary32 and every square and sum of the
+ * candidates is exact in binary64, so the comparison is exact.  Returns
+ * 0 (use +5) or 1 (use -5) and rewrites the winning elements to 0b1000. */
+static int razer_select(const float* v, int* q, int n)
+{
+    double gain[2] = {0.0, 0.0};
+    const double special[2] = {5.0, -5.0};
+    for (int s = 0; s < 2; ++s)
+        for (int i = 0; i < n; ++i) {
+            double e_reg = (double)v[i] - orc_e2m1_value(q[i]);
+            double e_sp = (double)v[i] - special[s];
+            if (fabs(e_sp) < fabs(e_reg))           /* strictly closer: remap */
+                gain[s] += e_reg * e_reg - e_sp * e_sp;
+        }
+    int pick = gain[1] > gain[0] ? 1 : 0;           /* ties keep +5 */
+    for (int i = 0; i < n; ++i) {
+        double e_reg = (double)v[i] - orc_e2m1_value(q[i]);
+        double e_sp = (double)v[i] - special[pick];
+        if (fabs(e_sp) < fabs(e_reg)) q[i] = 8;
+    }
+    return pick;
+}
+
+/* Quantize the row y[0..cols) (already rotated when asked).  Writes codes and
+ * scales for the row and returns nothing; s_t is used for NVFP4 formats. */
+static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
+                         uint8_t* row_codes, uint8_t* row_scales)
+{
+    const int B = block_size(fmt);
+    for (int64_t b0 = 0; b0 < cols; b0 += B) {
+        float a = 0.0f;
+        for (int i = 0; i < B; ++i) { float t = fabsf(y[b0 + i]); if (t > a) a = t; }
+        float v[32];
+        int q[32];
+        int sbyte;
+        if (fmt == ORC_MXFP4) {
+            /* TORQ sect. 1 / R3 */
+            if (a == 0.0f) {
+                sbyte = 0;
+                for (int i = 0; i < B; ++i) q[i] = 0;
+            } else {
+                int e = orc_mx_exponent(a);
+                sbyte = e + 127;
+                float r = (float)ldexp(1.0, -e);    /* exact power of two */
+                for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
+            }
+        } else {
+            /* RaZeR sect. 1 / R2: block scale from the block absmax */
+            float six_st = 6.0f * s_t;
+            float t = (six_st > 0.0f) ? a / six_st : 0.0f;
+            sbyte = orc_e4m3_encode(t);
+            float den = (float)orc_e4m3_value(sbyte) * s_t;
+            if (sbyte == 0 || den == 0.0f) {
+                /* a zero (or underflowed) scale decodes every element to 0 */
+                for (int i = 0; i < B; ++i) q[i] = 0;
+            } else {
+                float r = 1.0f / den;
+                for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
+                if (fmt == ORC_NVFP4_RAZER && razer_select(v, q, B)) sbyte |= 0x80;
+            }
+        }
+        row_scales[b0 / B] = (uint8_t)sbyte;
+        for (int i = 0; i < B; ++i) set_code(row_codes, b0 + i, q[i]);
+    }
+}
+
+/* Reconstruct the row in the original domain (inverse rotation when asked). */
+static void dequant_row(const uint8_t* row_codes, const uint8_t* row_scales, int64_t cols,
+                        int fmt, int rotate, float s_t, float* out)
+{
+    const int B = block_size(fmt);
+    for (int64_t b0 = 0; b0 < cols; b0 += B) {
+        int sbyte = row_scales[b0 / B];
+        float den = (fmt == ORC_MXFP4) ? 0.0f : nv_den(fmt, sbyte, s_t);
+        for (int i = 0; i < B; ++i) {
+            int code = get_code(row_codes, b0 + i);
+            out[b0 + i] = (fmt == ORC_MXFP4) ? mx_decode(code, sbyte)
+                                             : nv_decode(fmt, code, sbyte, den);
+        }
+    }
+    if (rotate)
+        for (int64_t g = 0; g < cols; g += 32) {
+            float t[32];
+            orc_wht32(out + g, t);
+            memcpy(out + g, t, sizeof t);
+        }
+}
+
+static double row_sse(const uint16_t* x, const float* xhat, int64_t cols)
+{
+    double s = 0.0;
+    for (int64_t j = 0; j < cols; ++j) {
+        double d = (double)orc_bf16_to_f32(x[j]) - (double)xhat[j];
+        s += d * d;
+    }
+    return s;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Whole-tensor entry points (rows split over pthreads; SSE summed in order) */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t* x; int64_t r0, r1, cols, ldx; int fmt, rotate; float s_t;
+    uint8_t* codes; uint8_t* scales; const uint8_t* ccodes; const uint8_t* cscales;
+    float* y_f32; uint16_t* y_bf16; int64_t ldy; int want_sse; double sse;
+} row_job;
+
+static void* quant_worker(void* p)
+{
+    row_job* j = (row_job*)p;
+    const int B = block_size(j->fmt);
+    float* y = (float*)malloc(sizeof(float) * (size_t)j->cols);
+    float* xh = (float*)malloc(sizeof(float) * (size_t)j->cols);
+    double sse = 0.0;
+    for (int64_t r = j->r0; r < j->r1; ++r) {
+        uint8_t* rc = j->codes + r * (j->cols / 2);
+        uint8_t* rs = j->scales + r * (j->cols / B);
+        load_row(j->x + r * j->ldx, j->cols, j->rotate, y);
+        quantize_row(y, j->cols, j->fmt, j->s_t, rc, rs);
+        if (j->want_sse) {
+            dequant_row(rc, rs, j->cols, j->fmt, j->rotate, j->s_t, xh);
+            sse += row_sse(j->x + r * j->ldx, xh, j->cols);
+        }
+    }
+    free(y); free(xh);
+    j->sse = sse;
+    return NULL;
+}
+
+static double run_rows(void* (*fn)(void*), row_job proto, int64_t rows, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = (int)rows;
+    row_job* jobs = (row_job*)calloc((size_t)nthreads, sizeof(row_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = proto;
+        jobs[t].r0 = rows * t / nthreads;
+        jobs[t].r1 = rows * (t + 1) / nthreads;
+        pthread_create(&th[t], NULL, fn, &jobs[t]);
+    }
+    double sse = 0.0;
+    for (int t = 0; t < nthreads; ++t) { pthread_join(th[t], NULL); sse += jobs[t].sse; }
+    free(jobs); free(th);
+    return sse;
+}
+
+/* Quantize a rows x cols bf16 matrix (row stride ldx elements).
+ *  scale_given != 0: *tensor_scale is read (NVFP4 formats), else computed
+ *  and written.  sse (nullable) receives the sum of squared errors against
+ *  the fp32 reconstruction in the original domain.  Returns 0, or -1 on a
+ *  shape the formats do not allow. */
+int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
+                 int fmt, int rotate, int scale_given, float* tensor_scale,
+                 uint8_t* codes, uint8_t* scales, double* sse, int nthreads)
+{
+    const int B = block_size(fmt);
+    if (rows < 0 || cols % B || (rotate && cols % 32) || ldx < cols) return -1;
+    float s_t = 0.0f;
+    if (fmt != ORC_MXFP4) {
+        if (scale_given) s_t = *tensor_scale;
+        else {
+            s_t = orc_tensor_scale_from_amax(orc_tensor_amax(x, rows, cols, ldx, rotate, nthreads));
+            *tensor_scale = s_t;
+        }
+    }
+    if (rows == 0 || cols == 0) { if (sse) *sse = 0.0; return 0; }
+    row_job proto = {0};
+    proto.x = x; proto.cols = cols; proto.ldx = ldx; proto.fmt = fmt; proto.rotate = rotate;
+    proto.s_t = s_t; proto.codes = codes; proto.scales = scales; proto.want_sse = sse != NULL;
+    double s = run_rows(quant_worker, proto, rows, nthreads);
+    if (sse) *sse = s;
+    return 0;
+}
+
+static void* dequant_worker(void* p)
+{
+    row_job* j = (row_job*)p;
+    const int B = block_size(j->fmt);
+    float* xh = (float*)malloc(sizeof(float) * (size_t)j->cols);
+    for (int64_t r = j->r0; r < j->r1; ++r) {
+        dequant_row(j->ccodes + r * (j->cols / 2), j->cscales + r * (j->cols / B), j->cols,
+                    j->fmt, j->rotate, j->s_t, xh);
+        for (int64_t c = 0; c < j->cols; ++c) {
+            if (j->y_f32) j->y_f32[r * j->ldy + c] = xh[c];
+            if (j->y_bf16) j->y_bf16[r * j->ldy + c] = orc_f32_to_bf16(xh[c]);
+        }
+    }
+    free(xh);
+    j->sse = 0.0;
+    return NULL;
+}
+
+/* Dequantize to fp32 (y_f32, nullable) and/or bf16 (y_bf16, nullable), both
+ * with row stride ldy. */
+int orc_dequantize(const uint8_t* codes, const uint8_t* scales, float tensor_scale,
+                   int64_t rows, int64_t cols, int fmt, int rotate,
+                   float* y_f32, uint16_t* y_bf16, int64_t ldy, int nthreads)
+{
+    const int B = block_size(fmt);
+    if (rows < 0 || cols % B || (rotate && cols % 32) || ldy < cols) return -1;
+    if (rows == 0 || cols == 0) return 0;
+    row_job proto = {0};
+    proto.cols = cols; proto.fmt = fmt; proto.rotate = rotate; proto.s_t = tensor_scale;
+    proto.ccodes = codes; proto.cscales = scales; proto.y_f32 = y_f32; proto.y_bf16 = y_bf16;
+    proto.ldy = ldy;
+    run_rows(dequant_worker, proto, rows, nthreads);
+    return 0;
+}
+
+static void* error_worker(void* p)
+{
+    row_job* j = (row_job*)p;
+    const int B = block_size(j->fmt);
+    float* xh = (float*)malloc(sizeof(float) * (size_t)j->cols);
+    double sse = 0.0;
+    for (int64_t r = j->r0; r < j->r1; ++r) {
+        dequant_row(j->ccodes + r * (j->cols / 2), j->cscales + r * (j->cols / B), j->cols,
+                    j->fmt, j->rotate, j->s_t, xh);
+        sse += row_sse(j->x + r * j->ldx, xh, j->cols);
+    }
+    free(xh);
+    j->sse = sse;
+    return NULL;
+}
+
+/* Sum of squared errors between x and the reconstruction of (codes, scales). */
+int orc_error(const uint16_t* x, int64_t ldx, const uint8_t* codes, const uint8_t* scales,
+              float tensor_scale, int64_t rows, int64_t cols, int fmt, int rotate,
+              double* sse, int nthreads)
+{
+    const int B = block_size(fmt);
+    if (rows < 0 || cols % B || (rotate && cols % 32) || ldx < cols) return -1;
+    if (rows == 0 || cols == 0) { *sse = 0.0; return 0; }
+    row_job proto = {0};
+    proto.x = x; proto.ldx = ldx; proto.cols = cols; proto.fmt = fmt; proto.rotate = rotate;
+    proto.s_t = tensor_scale; proto.ccodes = codes; proto.cscales = scales;
+    *sse = run_rows(error_worker, proto, rows, nthreads);
+    return 0;
+}

@@ -1,0 +1,411 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself.  Each pin comes from the pages'
+printed values (``tests/golden``), an exhaustive enumeration, exact rational
+arithmetic, a library cast (``ml_dtypes``, ``scipy``), a closed form or an
+invariant -- chosen so that a dropped term, a wrong sign, a wrong tie rule, a
+swapped nibble or a mis-indexed scale fails at least one of them.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import scipy.linalg
+
+from tests import bruteforce as bf
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+# ---------------------------------------------------------------- E2M1 elements
+
+def test_e2m1_value_set_is_the_pages_set(orc):
+    page = sorted(float(r[0]) for r in bf.read_golden("e2m1_value_set.txt"))
+    mine = sorted(orc.e2m1_value(c) for c in range(16))
+    assert mine == page
+    # sign-magnitude: code | 8 is the negation, -0 included
+    for c in range(8):
+        assert orc.e2m1_value(c | 8) == -orc.e2m1_value(c)
+        assert math.copysign(1.0, orc.e2m1_value(c | 8)) == -1.0
+
+
+def test_e2m1_decode_matches_bit_fields_and_ml_dtypes(orc):
+    lib = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    for c in range(16):
+        assert orc.e2m1_value(c) == bf.e2m1_from_bits(c) == float(lib[c])
+
+
+def _e2m1_sweep():
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    pts = set(grid)
+    for a, b in zip(grid, grid[1:]):
+        m = np.float32((a + b) / 2)
+        pts.update([float(m), float(np.nextafter(m, np.float32(0))), float(np.nextafter(m, np.float32(9)))])
+    for g in grid:
+        g32 = np.float32(g)
+        pts.update([float(np.nextafter(g32, np.float32(-1))), float(np.nextafter(g32, np.float32(9)))])
+    pts.update([7.0, 100.0, 3.0e38, 1e-40, 2 ** -149, 0.2499999, 5.5, 4.5])
+    rng = np.random.default_rng(11)
+    pts.update(float(v) for v in rng.uniform(0, 8, 3000).astype(np.float32))
+    vals = sorted(pts)
+    return [v for v in vals] + [-v for v in vals]
+
+
+def test_e2m1_encode_equals_exhaustive_argmin(orc):
+    for v in _e2m1_sweep():
+        assert orc.e2m1_encode(v) == bf.e2m1_nearest(v), v
+
+
+def test_e2m1_encode_ties_follow_even_code():
+    # the tie rule fixed for the oracle, checked against ml_dtypes' RNE cast
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    expect = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    got = ties.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    assert list(got) == expect
+
+
+def test_e2m1_encode_agrees_with_ml_dtypes_cast(orc):
+    sweep = np.array(_e2m1_sweep(), dtype=np.float32)
+    lib = sweep.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    for v, l in zip(sweep, lib):
+        mine = orc.e2m1_value(orc.e2m1_encode(float(v)))
+        assert mine == l  # equal as values; -0 == +0 (the oracle canonicalises zero)
+        if mine == 0:
+            assert orc.e2m1_encode(float(v)) == 0
+
+
+# ---------------------------------------------------------------- E4M3 scales
+
+def test_e4m3_decode_all_bytes(orc):
+    lib = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    for b in range(256):
+        if b & 0x7F == 0x7F:
+            assert math.isnan(orc.e4m3_value(b))
+            continue
+        assert orc.e4m3_value(b) == bf.e4m3_from_bits(b) == lib[b], b
+    assert orc.e4m3_value(0x7E) == 448.0
+    assert orc.e4m3_value(0x01) == 2.0 ** -9
+
+
+def _e4m3_sweep():
+    vals = [float(v) for v in bf.E4M3_POS]
+    pts = set(vals)
+    for a, b in zip(vals, vals[1:]):
+        m = np.float32((a + b) / 2)
+        pts.update([float(m), float(np.nextafter(m, np.float32(0))), float(np.nextafter(m, np.float32(1e9)))])
+    rng = np.random.default_rng(12)
+    pts.update(float(v) for v in rng.uniform(0, 460, 2000).astype(np.float32))
+    pts.update(float(v) for v in np.exp2(rng.uniform(-12, 9, 2000)).astype(np.float32))
+    pts.update([0.0, 448.0, 450.0, 464.0, 470.0, 1e6, 1e-30, 2 ** -10, 3 * 2 ** -11])
+    return sorted(pts)
+
+
+def test_e4m3_encode_equals_exhaustive_argmin(orc):
+    for t in _e4m3_sweep():
+        assert orc.e4m3_encode(t) == bf.e4m3_nearest(t), t
+
+
+def test_e4m3_encode_saturates_and_matches_ml_dtypes_in_range(orc):
+    sweep = np.array(_e4m3_sweep(), dtype=np.float32)
+    inr = sweep[sweep <= 448]
+    lib = inr.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    for t, b in zip(inr, lib):
+        assert orc.e4m3_encode(float(t)) == int(b), t
+    for t in sweep[sweep > 448]:
+        assert orc.e4m3_encode(float(t)) == 0x7E
+
+
+# ---------------------------------------------------------------- E8M0 / MXFP4 exponent
+
+def test_e8m0_decode(orc):
+    lib = np.arange(255, dtype=np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    for b in range(255):
+        assert orc.e8m0_value(b) == lib[b] == 2.0 ** (b - 127)
+    assert math.isnan(orc.e8m0_value(255))
+
+
+def test_mx_exponent_is_floor_log2_minus_two(orc):
+    rng = np.random.default_rng(13)
+    pts = [float(v) for v in np.exp2(rng.uniform(-140, 127, 3000)).astype(np.float32) if v > 0]
+    for k in range(-149, 128):
+        p = np.float32(2.0 ** k)
+        pts += [float(p), float(np.nextafter(p, np.float32(0)))]
+    pts = [p for p in pts if p > 0 and math.isfinite(p)]
+    for a in pts:
+        want = max(-127, min(127, bf.floor_log2(a) - 2))
+        assert orc.mx_exponent(a) == want, a
+
+
+# ---------------------------------------------------------------- bf16
+
+def test_bf16_rounding_matches_ml_dtypes(orc):
+    rng = np.random.default_rng(14)
+    v = rng.standard_normal(4000).astype(np.float32) * np.float32(3.0)
+    # exact ties: a bf16 value plus half of its last place
+    base = v.astype(ml_dtypes.bfloat16).astype(np.float32)
+    ties = (base.view(np.uint32) | np.uint32(0x8000)).view(np.float32)
+    allv = np.concatenate([v, ties, np.float32([0.0, -0.0, 1e-40, -3e38])])
+    want = allv.astype(ml_dtypes.bfloat16).view(np.uint16)
+    got = orc.f32_to_bf16(allv)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- rotation
+
+def test_hadamard_is_sylvester(orc):
+    H = np.array([[orc.hadamard_entry(i, j) for j in range(32)] for i in range(32)])
+    assert np.array_equal(H, scipy.linalg.hadamard(32))
+    assert np.array_equal(H @ H.T, 32 * np.eye(32, dtype=H.dtype))
+
+
+def test_wht_constant_is_rn_of_inverse_sqrt32(orc):
+    c = np.float32(orc.wht_constant())
+    # c is the binary32 nearest to 1/sqrt(32): compare squares exactly against 1/32
+    lo, hi = np.nextafter(c, np.float32(0)), np.nextafter(c, np.float32(1))
+    target = Fraction(1, 32)
+    # the true value lies between the midpoints (lo+c)/2 and (c+hi)/2
+    assert (Fraction(float(lo)) + Fraction(float(c))) ** 2 / 4 < target
+    assert (Fraction(float(c)) + Fraction(float(hi))) ** 2 / 4 > target
+
+
+def test_wht_closed_forms(orc):
+    c = np.float32(orc.wht_constant())
+    e0 = np.zeros(32, np.float32); e0[0] = 1
+    assert np.all(orc.wht32(e0) == c)                               # delta -> flat
+    y = orc.wht32(np.ones(32, np.float32))
+    assert y[0] == np.float32(np.float32(32) * c) and np.all(y[1:] == 0)   # flat -> delta
+    H = scipy.linalg.hadamard(32).astype(np.float32)
+    for k in (1, 5, 17, 31):                                          # Walsh row k -> delta at k
+        y = orc.wht32(H[k])
+        assert y[k] == np.float32(np.float32(32) * c)
+        assert np.count_nonzero(y) == 1
+
+
+def test_wht_orthogonal_involution(orc):
+    rng = np.random.default_rng(15)
+    for _ in range(50):
+        x = rng.standard_normal(32).astype(np.float32)
+        y = orc.wht32(x)
+        assert abs(np.linalg.norm(y.astype(np.float64)) / np.linalg.norm(x.astype(np.float64)) - 1) < 1e-6
+        z = orc.wht32(y)
+        ulp = np.spacing(np.abs(x).max())
+        assert np.max(np.abs(z - x)) <= 2 * ulp
+
+
+def test_wht_equals_exact_rational_transform(orc):
+    rng = np.random.default_rng(16)
+    H = bf.sylvester_hadamard(32)
+    c = np.float32(orc.wht_constant())
+    for _ in range(20):
+        xb = (rng.standard_normal(32).astype(np.float32)).astype(ml_dtypes.bfloat16).astype(np.float32)
+        got = orc.wht32(xb)
+        for i in range(32):
+            s = sum((int(H[i, j]) * Fraction(float(xb[j])) for j in range(32)), Fraction(0))
+            assert got[i] == np.float32(bf.rn_f32(s) * c)
+
+
+# ---------------------------------------------------------------- tensor scale (two-level NVFP4)
+
+def test_tensor_scale_maps_amax_to_6x448(orc):
+    for k in range(-20, 20):
+        assert orc.tensor_scale_from_amax(2688.0 * 2.0 ** k) == 2.0 ** k
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
+def test_max_block_gets_scale_448(orc, fmt):
+    rng = np.random.default_rng(17)
+    x = (rng.standard_normal((4, 64)) * 0.02).astype(np.float32)
+    x[2, 37] = 2688.0 * 2.0 ** -7   # tensor max, exactly 6 * 448 * 2^-7
+    xb = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    codes, scales, ts, _ = orc.quantize(xb, fmt)
+    assert ts == np.float32(2.0 ** -7)
+    assert scales[2, 37 // 16] & 0x7F == 0x7E
+    nib = bf.unpack_codes(codes, 64)
+    assert nib[2, 37] == 7   # +6
+
+
+# ---------------------------------------------------------------- brute force on tiny tensors
+
+def _tiny_inputs():
+    rng = np.random.default_rng(18)
+    out = []
+    x = (rng.standard_normal((3, 64)) * 0.02).astype(np.float32)
+    x.ravel()[rng.choice(x.size, 3, replace=False)] *= 20
+    out.append(x)
+    t = rng.standard_t(3, size=(2, 64)).astype(np.float32) * np.exp(rng.standard_normal(64)).astype(np.float32)
+    out.append(t)
+    z = np.zeros((2, 32), np.float32); z[1, 5] = -3.0
+    out.append(z)
+    return [a.astype(ml_dtypes.bfloat16).view(np.uint16) for a in out]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_quantize_equals_bruteforce(orc, fmt, rotate):
+    for xb in _tiny_inputs():
+        codes, scales, ts, sse = orc.quantize(xb, fmt, rotate)
+        bcodes, bscales, bts = bf.quantize_bruteforce(xb, fmt, rotate)
+        assert np.array_equal(codes, bcodes)
+        assert np.array_equal(scales, bscales)
+        if fmt != "mxfp4":
+            assert ts == bts
+        xhat = bf.dequantize_bruteforce(bcodes, bscales, bts, fmt, rotate)
+        exact = bf.sse_exact(xb, xhat)
+        assert abs(sse - float(exact)) <= 1e-12 * max(1.0, float(exact))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_dequantize_equals_bruteforce(orc, fmt, rotate):
+    import torch
+    from activation_quantization_block_b200 import synthetic
+    codes, scales, ts = synthetic.random_packed(3, 64, fmt, seed=4)
+    codes, scales = codes.numpy(), scales.numpy()
+    ts = float(ts[0]) * 2.0 ** -6
+    y32, y16 = orc.dequantize(codes, scales, ts, fmt, rotate)
+    want = bf.dequantize_bruteforce(codes, scales, ts, fmt, rotate)
+    assert np.array_equal(y32.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(y16, want.astype(ml_dtypes.bfloat16).view(np.uint16))
+    del torch
+
+
+# ---------------------------------------------------------------- idempotence on representable inputs
+
+def _representable(fmt, rows=4, cols=64, seed=19):
+    """x = value(code) * scale exactly, with a +-6 (MXFP4: +-6 or +-4) in every block."""
+    rng = np.random.default_rng(seed)
+    B = 32 if fmt == "mxfp4" else 16
+    nb = cols // B
+    codes = rng.integers(0, 16, size=(rows, cols))
+    codes[codes == 8] = 0
+    for r in range(rows):
+        for b in range(nb):
+            codes[r, b * B + rng.integers(0, B)] = rng.choice([7, 15])
+    x = np.zeros((rows, cols), np.float64)
+    if fmt == "mxfp4":
+        ex = rng.integers(-20, 20, size=(rows, nb))
+        for r in range(rows):
+            for j in range(cols):
+                x[r, j] = bf.E2M1[codes[r, j]] * 2.0 ** ex[r, j // B]
+    else:
+        ts = 2.0 ** -9
+        sb = rng.integers(0x20, 0x7F, size=(rows, nb))
+        sb[0, 0] = 0x7E
+        for r in range(rows):
+            for b in range(nb):
+                den = bf.e4m3_from_bits(int(sb[r, b])) * ts
+                if fmt == "nvfp4_razer" and rng.random() < 0.7:
+                    sign = rng.choice([1.0, -1.0])
+                    j = b * B + (int(np.argmax(np.abs([bf.E2M1[c] for c in codes[r, b * B:(b + 1) * B]]))) + 1) % B
+                    codes[r, j] = 8
+                    x[r, j] = 5.0 * sign * den
+                for j in range(b * B, (b + 1) * B):
+                    if codes[r, j] != 8 or fmt != "nvfp4_razer":
+                        x[r, j] = bf.E2M1[codes[r, j]] * den
+    x32 = x.astype(np.float32)
+    assert np.array_equal(x32.astype(np.float64), x)
+    xb = x32.astype(ml_dtypes.bfloat16)
+    assert np.array_equal(xb.astype(np.float64), x)   # exactly representable in bf16
+    return xb.view(np.uint16)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+def test_idempotent_on_representable_inputs(orc, fmt):
+    xb = _representable(fmt)
+    codes, scales, ts, sse = orc.quantize(xb, fmt)
+    assert sse == 0.0
+    y32, y16 = orc.dequantize(codes, scales, ts, fmt)
+    assert np.array_equal(y16, xb)
+    codes2, scales2, ts2, sse2 = orc.quantize(y16, fmt)
+    assert np.array_equal(codes, codes2) and np.array_equal(scales, scales2) and ts == ts2
+    if fmt == "nvfp4_razer":
+        nib = bf.unpack_codes(codes, xb.shape[1])
+        assert (nib == 8).any()      # the +-5 entries were used
+
+
+# ---------------------------------------------------------------- RaZeR invariants and worked case
+
+def test_razer_special_values_are_the_pages_pair(orc):
+    pair = {int(r[0]): float(r[1]) for r in bf.read_golden("razer_special_values.txt")}
+    ts = 1.0
+    for sel, val in pair.items():
+        codes = np.array([[0x08] + [0] * 7], np.uint8)        # element 0 = code 0b1000
+        scales = np.array([[0x38 | (sel << 7)]], np.uint8)    # E4M3 1.0, selector bit
+        y32, _ = orc.dequantize(codes, scales, ts, "nvfp4_razer")
+        assert y32[0, 0] == val and val % 0.5 == 0
+
+
+def test_razer_worked_block(orc):
+    # one block [6d, 5d, 0, ...] with d = 448 * 2^-9: the 5d element is exactly the
+    # special value +5, so RaZeR is lossless where NVFP4 must round 5 -> 4.
+    d = 448 * 2.0 ** -9
+    x = np.zeros((1, 16), np.float32); x[0, 0] = 6 * d; x[0, 1] = 5 * d
+    xb = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    c_nv, s_nv, ts, sse_nv = orc.quantize(xb, "nvfp4")
+    c_rz, s_rz, ts2, sse_rz = orc.quantize(xb, "nvfp4_razer")
+    assert ts == ts2 == np.float32(2.0 ** -9)
+    assert s_nv[0, 0] == 0x7E and s_rz[0, 0] == 0x7E     # +5 selected: bit 7 clear
+    assert bf.unpack_codes(c_nv, 16)[0, 1] == 6          # 5 -> 4 (tie to even)
+    assert bf.unpack_codes(c_rz, 16)[0, 1] == 8
+    assert sse_rz == 0.0 and sse_nv == float((d) ** 2)
+    # the negated block picks -5 through the scale's sign bit
+    c_neg, s_neg, _, sse_neg = orc.quantize((-x).astype(ml_dtypes.bfloat16).view(np.uint16), "nvfp4_razer")
+    assert s_neg[0, 0] == 0xFE and bf.unpack_codes(c_neg, 16)[0, 1] == 8 and sse_neg == 0.0
+
+
+def test_razer_invariants_on_random_blocks(orc):
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.llm_weight(64, 256, seed=20))
+    c_nv, s_nv, ts, _ = orc.quantize(xb, "nvfp4", nthreads=2)
+    c_rz, s_rz, ts2, _ = orc.quantize(xb, "nvfp4_razer", nthreads=2)
+    assert ts == ts2
+    assert np.array_equal(s_rz & 0x7F, s_nv)
+    n_nv, n_rz = bf.unpack_codes(c_nv, 256), bf.unpack_codes(c_rz, 256)
+    differ = n_nv != n_rz
+    assert np.all(n_rz[differ] == 8)
+    assert differ.any() and (s_rz & 0x80).any()
+    # per-block squared error never grows
+    y_nv, _ = orc.dequantize(c_nv, s_nv, ts, "nvfp4")
+    y_rz, _ = orc.dequantize(c_rz, s_rz, ts, "nvfp4_razer")
+    x = bf.bits_to_f32(xb).astype(np.float64)
+    e_nv = ((x - y_nv) ** 2).reshape(64, 16, 16).sum(-1)
+    e_rz = ((x - y_rz) ** 2).reshape(64, 16, 16).sum(-1)
+    assert np.all(e_rz <= e_nv * (1 + 1e-12))
+    assert e_rz.sum() < e_nv.sum()
+
+
+def test_scale_rule_versus_best_scale_record(orc):
+    """Record, not an equality: the absmax rule is never better than the best
+    E4M3 scale found by enumerating all 126 nonzero scale bytes."""
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.llm_weight(2, 32, seed=21))
+    x = bf.bits_to_f32(xb)
+    codes, scales, ts, _ = orc.quantize(xb, "nvfp4")
+    y, _ = orc.dequantize(codes, scales, ts, "nvfp4")
+    for b in range(4):
+        r, c0 = divmod(b, 2)
+        blk = x[r, c0 * 16:(c0 + 1) * 16].astype(np.float64)
+        rule = float(((blk - y[r, c0 * 16:(c0 + 1) * 16]) ** 2).sum())
+        best = min(
+            float(((blk - np.array([bf.E2M1[bf.e2m1_nearest(float(v / (bf.e4m3_from_bits(sb) * ts)))]
+                                      for v in blk]) * bf.e4m3_from_bits(sb) * ts) ** 2).sum())
+            for sb in range(1, 0x7F))
+        # the enumeration reconstructs in double, the rule in binary32: 1e-5 slack
+        assert rule >= best * (1 - 1e-5)
+
+
+# ---------------------------------------------------------------- statistics sanity (direction only)
+
+def test_rotation_spreads_mxfp4_code_occupancy(orc):
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.activation_t3(64, 512, seed=1))
+    c0, _, _, sse0 = orc.quantize(xb, "mxfp4", False)
+    c1, _, _, sse1 = orc.quantize(xb, "mxfp4", True)
+    z0 = (bf.unpack_codes(c0, 512) & 7 == 0).mean()
+    z1 = (bf.unpack_codes(c1, 512) & 7 == 0).mean()
+    assert z1 < z0          # rotation leaves fewer elements quantized to zero
+    assert sse1 < sse0
