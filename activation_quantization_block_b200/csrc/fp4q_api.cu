@@ -1,0 +1,199 @@
+// C ABI of fp4q (declared in include/fp4q.h): argument validation, workspace
+// carving and kernel dispatch.  Validation happens on the host before any
+// launch; a rejected call enqueues nothing.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "fp4q.h"
+#include "fp4q_internal.h"
+
+using namespace fp4q;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_dev_ok[kMaxDevices];   // 0 unknown, 1 supported, -1 not supported
+
+// The kernels are built for sm_100a only: require compute capability 10.0.
+fp4q_status_t check_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FP4Q_ERROR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERROR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_dev_ok[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return FP4Q_ERROR_CUDA;
+        }
+        g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return g_dev_ok[dev] == 1 ? FP4Q_SUCCESS : FP4Q_ERROR_UNSUPPORTED_DEVICE;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int block_len(int fmt) { return fmt == FP4Q_MXFP4 ? 32 : 16; }
+
+bool valid_format(int fmt) { return fmt == FP4Q_NVFP4 || fmt == FP4Q_NVFP4_RAZER || fmt == FP4Q_MXFP4; }
+
+// Shape checks shared by every entry point.
+fp4q_status_t check_shape(int64_t rows, int64_t cols, int fmt, int rotate)
+{
+    if (!valid_format(fmt) || (rotate != 0 && rotate != 1)) return FP4Q_ERROR_INVALID_VALUE;
+    if (rows < 0 || cols < 0) return FP4Q_ERROR_INVALID_VALUE;
+    if (cols % block_len(fmt) != 0 || (rotate && cols % 32 != 0)) return FP4Q_ERROR_SHAPE;
+    if (cols > 0 && rows > ((int64_t)1 << 62) / cols) return FP4Q_ERROR_SHAPE;
+    return FP4Q_SUCCESS;
+}
+
+fp4q_status_t check_matrix(const void* p, int64_t cols, int64_t ld)
+{
+    if (p == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (ld < cols) return FP4Q_ERROR_SHAPE;
+    if (ld % 8 != 0 || !aligned(p, 16)) return FP4Q_ERROR_MISALIGNED;
+    if (ld > ((int64_t)1 << 62)) return FP4Q_ERROR_SHAPE;
+    return FP4Q_SUCCESS;
+}
+
+fp4q_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_SUCCESS : FP4Q_ERROR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int fp4q_abi_version(void) { return FP4Q_ABI_VERSION; }
+
+const char* fp4q_status_string(fp4q_status_t s)
+{
+    switch (s) {
+        case FP4Q_SUCCESS: return "success";
+        case FP4Q_ERROR_INVALID_VALUE: return "invalid value (null pointer, bad enum or flag, negative size)";
+        case FP4Q_ERROR_SHAPE: return "bad shape (cols not a multiple of the block or rotation group, ld < cols, or size overflow)";
+        case FP4Q_ERROR_MISALIGNED: return "misaligned pointer or leading dimension";
+        case FP4Q_ERROR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case FP4Q_ERROR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (compute capability 10.0)";
+        case FP4Q_ERROR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+size_t fp4q_workspace_size(int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate)
+{
+    (void)rows; (void)cols; (void)fmt; (void)rotate;
+    return kWorkspaceBytes;
+}
+
+fp4q_status_t fp4q_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                            fp4q_format_t fmt, int rotate, uint32_t flags,
+                            uint8_t* codes, uint8_t* scales, float* tensor_scale, double* mse,
+                            void* workspace, size_t workspace_bytes, fp4q_stream_t stream)
+{
+    fp4q_status_t s = check_shape(rows, cols, fmt, rotate);
+    if (s != FP4Q_SUCCESS) return s;
+    if (flags & ~FP4Q_FLAG_TENSOR_SCALE_GIVEN) return FP4Q_ERROR_INVALID_VALUE;
+    const bool nv = fmt != FP4Q_MXFP4;
+    const bool given = (flags & FP4Q_FLAG_TENSOR_SCALE_GIVEN) != 0;
+    if (nv && tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (nv && !aligned(tensor_scale, 4)) return FP4Q_ERROR_MISALIGNED;
+    if (mse != nullptr && !aligned(mse, 8)) return FP4Q_ERROR_MISALIGNED;
+    const int64_t n = rows * cols;
+    const bool need_ws = n > 0 && ((nv && !given) || mse != nullptr);
+    if (n > 0) {
+        if ((s = check_matrix(x, cols, ldx)) != FP4Q_SUCCESS) return s;
+        if (codes == nullptr || scales == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+        if (!aligned(codes, 16) || !aligned(scales, 16)) return FP4Q_ERROR_MISALIGNED;
+    }
+    if (need_ws && (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < kWorkspaceBytes))
+        return FP4Q_ERROR_WORKSPACE;
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n == 0) {
+        if (nv && !given && cudaMemsetAsync(tensor_scale, 0, sizeof(float), st) != cudaSuccess) return FP4Q_ERROR_CUDA;
+        if (mse && cudaMemsetAsync(mse, 0, sizeof(double), st) != cudaSuccess) return FP4Q_ERROR_CUDA;
+        return FP4Q_SUCCESS;
+    }
+
+    char* ws = static_cast<char*>(workspace);
+    double* sse_part = ws ? reinterpret_cast<double*>(ws + kWsSseOffset) : nullptr;
+    float* amax_part = ws ? reinterpret_cast<float*>(ws + kWsAmaxOffset) : nullptr;
+    const Geometry g = make_geometry(rows, cols, ldx);
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+
+    int n_amax = 0;
+    if (nv && !given) {
+        if ((s = from_cuda(launch_amax(xp, g, rotate, amax_part, &n_amax, st))) != FP4Q_SUCCESS) return s;
+    }
+    int n_sse = 0;
+    s = from_cuda(launch_quantize(xp, g, fmt, rotate, mse != nullptr, given ? 1 : 0, codes, scales,
+                                  tensor_scale, amax_part, n_amax, sse_part, &n_sse, st));
+    if (s != FP4Q_SUCCESS) return s;
+    if (mse) s = from_cuda(launch_sse_finalize(sse_part, n_sse, (double)n, mse, st));
+    return s;
+}
+
+fp4q_status_t fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                              int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
+                              void* y, int64_t ldy, fp4q_stream_t stream)
+{
+    fp4q_status_t s = check_shape(rows, cols, fmt, rotate);
+    if (s != FP4Q_SUCCESS) return s;
+    const bool nv = fmt != FP4Q_MXFP4;
+    if (nv && tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (nv && !aligned(tensor_scale, 4)) return FP4Q_ERROR_MISALIGNED;
+    const int64_t n = rows * cols;
+    if (n > 0) {
+        if ((s = check_matrix(y, cols, ldy)) != FP4Q_SUCCESS) return s;
+        if (codes == nullptr || scales == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+        if (!aligned(codes, 16) || !aligned(scales, 16)) return FP4Q_ERROR_MISALIGNED;
+    }
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+    if (n == 0) return FP4Q_SUCCESS;
+    const Geometry g = make_geometry(rows, cols, ldy);
+    return from_cuda(launch_dequantize(codes, scales, tensor_scale, g, fmt, rotate, static_cast<uint16_t*>(y),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status_t fp4q_error(const void* x, int64_t ldx,
+                         const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                         int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
+                         double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream)
+{
+    fp4q_status_t s = check_shape(rows, cols, fmt, rotate);
+    if (s != FP4Q_SUCCESS) return s;
+    const bool nv = fmt != FP4Q_MXFP4;
+    if (mse == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (!aligned(mse, 8)) return FP4Q_ERROR_MISALIGNED;
+    if (nv && tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (nv && !aligned(tensor_scale, 4)) return FP4Q_ERROR_MISALIGNED;
+    const int64_t n = rows * cols;
+    if (n > 0) {
+        if ((s = check_matrix(x, cols, ldx)) != FP4Q_SUCCESS) return s;
+        if (codes == nullptr || scales == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+        if (!aligned(codes, 16) || !aligned(scales, 16)) return FP4Q_ERROR_MISALIGNED;
+        if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < kWorkspaceBytes)
+            return FP4Q_ERROR_WORKSPACE;
+    }
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n == 0) return from_cuda(cudaMemsetAsync(mse, 0, sizeof(double), st));
+    char* ws = static_cast<char*>(workspace);
+    double* sse_part = reinterpret_cast<double*>(ws + kWsSseOffset);
+    const Geometry g = make_geometry(rows, cols, ldx);
+    int n_sse = 0;
+    s = from_cuda(launch_error(static_cast<const uint16_t*>(x), codes, scales, tensor_scale, g, fmt, rotate,
+                               sse_part, &n_sse, st));
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_sse_finalize(sse_part, n_sse, (double)n, mse, st));
+}
+
+}  // extern "C"

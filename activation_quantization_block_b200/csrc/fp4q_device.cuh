@@ -1,0 +1,148 @@
+// Device helpers for the fp4q kernels (sm_100a).
+//
+// Number formats follow "RaZeR: Pushing the Limits of NVFP4 Quantization with
+// Redundant Zero Remapping" (technical summary sect. 1: E2M1 elements
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit, FP8-E4M3 block scale) and
+// "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization" (sect. 1:
+// 32-element blocks with a shared power-of-two scale).  Conversions use the
+// hardware cvt instructions of sm_100a: E2M1 and E4M3 encoding round to
+// nearest even and saturate to the largest finite value, which is the
+// element and scale rounding rule of this library.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace fp4q {
+
+// RN_f32(1 / sqrt(32)), the normalisation of the 32-point Walsh-Hadamard transform.
+__device__ __forceinline__ float wht_scale() { return __uint_as_float(0x3E3504F3u); }
+
+// ---- bf16 -----------------------------------------------------------------
+
+// A 32-bit word holds elements 2k (low half) and 2k+1 (high half); widening is exact.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---- E2M1 -----------------------------------------------------------------
+
+// Eight fp32 values -> eight E2M1 nibbles (value i in bits 4i..4i+3), nearest
+// even, saturating.  Negative values that round to zero come out as 0b1000.
+__device__ __forceinline__ uint32_t e2m1x8(const float* v)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return out;
+}
+
+// Rewrite every -0 nibble (0b1000) as +0: a nibble keeps its sign bit only if
+// its magnitude is nonzero.  (mag + 7) carries into bit 3 exactly when mag >= 1,
+// and never into the next nibble.
+__device__ __forceinline__ uint32_t canonical_zero(uint32_t w)
+{
+    uint32_t nz = (w & 0x77777777u) + 0x77777777u;
+    return w & ((nz & 0x88888888u) | 0x77777777u);
+}
+
+// Two E2M1 nibbles (bits 0..3 element 2k, bits 4..7 element 2k+1) -> two fp32 values.
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte)
+{
+    uint32_t h;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h) : "r"(byte));
+    __half2 hh = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(hh);  // .x = low half = element 2k
+}
+
+// ---- E4M3 -----------------------------------------------------------------
+
+// Non-negative fp32 -> E4M3 byte, nearest even, saturating at 448 (0x7E).
+__device__ __forceinline__ uint32_t e4m3_rn_satfinite(float t)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+    return r & 0xFFu;
+}
+
+// E4M3 byte (sign included) -> fp32, exact.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte)
+{
+    uint32_t h;
+    uint16_t in = (uint16_t)(byte & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+}
+
+// ---- E8M0 -----------------------------------------------------------------
+
+// floor(log2 a) for a finite a > 0, from the binary32 fields (subnormals included).
+__device__ __forceinline__ int floor_log2_f32(float a)
+{
+    uint32_t u = __float_as_uint(a);
+    int ex = (int)((u >> 23) & 0xFFu);
+    if (ex != 0) return ex - 127;
+    return (31 - __clz((int)u)) - 149;
+}
+
+// 2^k for k in [-127, 127] as fp32 (2^-127 is subnormal).
+__device__ __forceinline__ float exp2i(int k)
+{
+    return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---- 32-point Walsh-Hadamard, in registers ----------------------------------
+
+// y <- H32 y (Sylvester order: H_ij = (-1)^popcount(i & j)), fp32 butterflies,
+// then y <- RN(y * RN(1/sqrt 32)).  The transform is its own inverse.
+__device__ __forceinline__ void wht32_inplace(float* y)
+{
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if ((i & h) == 0) {
+                float a = y[i], b = y[i + h];
+                y[i] = a + b;
+                y[i + h] = a - b;
+            }
+        }
+    }
+    const float c = wht_scale();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(y[i], c);
+}
+
+// ---- loads / stores -------------------------------------------------------
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void stg_v4(void* p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ void stg_v2(void* p, uint32_t a, uint32_t b)
+{
+    asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(a), "r"(b) : "memory");
+}
+
+}  // namespace fp4q

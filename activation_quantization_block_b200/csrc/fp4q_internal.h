@@ -1,0 +1,58 @@
+// Internal interface between the C ABI layer (fp4q_api.cu) and the kernels
+// (fp4q_kernels.cu).  Not installed; not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+constexpr int kThreads = 256;        // threads per CTA for every streaming kernel
+constexpr int kMaxPartials = 4096;   // upper bound on CTAs of one pass (per-CTA partial slots)
+
+// Workspace layout: fp64 partial sums, then fp32 partial maxima.
+constexpr size_t kWsSseOffset = 0;
+constexpr size_t kWsAmaxOffset = kMaxPartials * sizeof(double);
+constexpr size_t kWorkspaceBytes = kWsAmaxOffset + kMaxPartials * sizeof(float);
+
+// Geometry of a bf16 matrix seen as consecutive 16-element "halves" (one
+// NVFP4 block each); a unit is two consecutive halves = 32 elements.
+struct Geometry {
+    int64_t rows, cols, ld;   // ld: row stride of the bf16 matrix in elements
+    int64_t halves;           // rows * cols / 16
+    int64_t halves_per_row;   // cols / 16
+    int64_t units;            // ceil(halves / 2)
+};
+
+inline Geometry make_geometry(int64_t rows, int64_t cols, int64_t ld)
+{
+    Geometry g;
+    g.rows = rows; g.cols = cols; g.ld = ld;
+    g.halves = rows * cols / 16;
+    g.halves_per_row = cols / 16;
+    g.units = (g.halves + 1) / 2;
+    return g;
+}
+
+// Launchers: return cudaSuccess or the launch error.  `grid_out` (nullable)
+// receives the number of CTAs launched (= partial slots written).
+cudaError_t launch_amax(const uint16_t* x, const Geometry& g, int rotate, float* partials,
+                        int* grid_out, cudaStream_t st);
+
+cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int rotate, int want_sse,
+                            int scale_given, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                            const float* amax_partials, int n_amax, double* sse_partials,
+                            int* grid_out, cudaStream_t st);
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                              const Geometry& g, int fmt, int rotate, uint16_t* y, cudaStream_t st);
+
+cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t* scales,
+                         const float* tensor_scale, const Geometry& g, int fmt, int rotate,
+                         double* sse_partials, int* grid_out, cudaStream_t st);
+
+cudaError_t launch_sse_finalize(const double* partials, int n, double count, double* mse,
+                                cudaStream_t st);
+
+}  // namespace fp4q

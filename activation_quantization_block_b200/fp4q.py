@@ -1,0 +1,209 @@
+"""Python binding of the fp4q C ABI (``include/fp4q.h``).
+
+The functions named ``fp4q_*`` mirror the C entry points one to one: they only
+marshal arguments (torch tensors become device pointers, the stream becomes a
+``cudaStream_t``) and return the C status code.  The convenience wrappers
+``quantize`` / ``dequantize`` / ``error`` allocate outputs with torch, pass the
+current torch stream and raise ``Fp4qError`` on a non-success status.  Every
+step of the computation runs in the CUDA library; there is no CPU path, and a
+missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import NamedTuple
+
+import torch
+
+from . import _build
+
+NVFP4, NVFP4_RAZER, MXFP4 = 0, 1, 2
+FORMATS = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4}
+FLAG_TENSOR_SCALE_GIVEN = 0x1
+
+SUCCESS = 0
+STATUS_NAMES = {
+    0: "FP4Q_SUCCESS", 1: "FP4Q_ERROR_INVALID_VALUE", 2: "FP4Q_ERROR_SHAPE", 3: "FP4Q_ERROR_MISALIGNED",
+    4: "FP4Q_ERROR_WORKSPACE", 5: "FP4Q_ERROR_UNSUPPORTED_DEVICE", 6: "FP4Q_ERROR_CUDA",
+}
+
+# Names the C header declares; the tests check that the library exports each one.
+ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
+               "fp4q_quantize", "fp4q_dequantize", "fp4q_error")
+
+
+class Fp4qError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({fp4q_status_string(status)})")
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load (building first if the sources are newer) the in-tree libfp4q.so."""
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(_build.build())
+        vp, i64, i32, u32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
+        L.fp4q_abi_version.argtypes = []
+        L.fp4q_abi_version.restype = i32
+        L.fp4q_status_string.argtypes = [i32]
+        L.fp4q_status_string.restype = ctypes.c_char_p
+        L.fp4q_workspace_size.argtypes = [i64, i64, i32, i32]
+        L.fp4q_workspace_size.restype = sz
+        L.fp4q_quantize.argtypes = [vp, i64, i64, i64, i32, i32, u32, vp, vp, vp, vp, vp, sz, vp]
+        L.fp4q_quantize.restype = i32
+        L.fp4q_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, i64, vp]
+        L.fp4q_dequantize.restype = i32
+        L.fp4q_error.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, sz, vp]
+        L.fp4q_error.restype = i32
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _fmt(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+# ---- the C entry points, same names --------------------------------------------
+
+def fp4q_abi_version() -> int:
+    return lib().fp4q_abi_version()
+
+
+def fp4q_status_string(status: int) -> str:
+    return lib().fp4q_status_string(int(status)).decode()
+
+
+def fp4q_workspace_size(rows: int, cols: int, fmt, rotate: int) -> int:
+    return lib().fp4q_workspace_size(rows, cols, _fmt(fmt), int(rotate))
+
+
+def fp4q_quantize(x, rows, cols, ldx, fmt, rotate, flags, codes, scales, tensor_scale, mse,
+                  workspace, workspace_bytes, stream=None) -> int:
+    return lib().fp4q_quantize(_ptr(x), rows, cols, ldx, _fmt(fmt), int(rotate), flags, _ptr(codes),
+                               _ptr(scales), _ptr(tensor_scale), _ptr(mse), _ptr(workspace),
+                               workspace_bytes, _stream(stream))
+
+
+def fp4q_dequantize(codes, scales, tensor_scale, rows, cols, fmt, rotate, y, ldy, stream=None) -> int:
+    return lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, cols, _fmt(fmt),
+                                 int(rotate), _ptr(y), ldy, _stream(stream))
+
+
+def fp4q_error(x, ldx, codes, scales, tensor_scale, rows, cols, fmt, rotate, mse, workspace,
+               workspace_bytes, stream=None) -> int:
+    return lib().fp4q_error(_ptr(x), ldx, _ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, cols,
+                            _fmt(fmt), int(rotate), _ptr(mse), _ptr(workspace), workspace_bytes,
+                            _stream(stream))
+
+
+# ---- torch-level wrappers -------------------------------------------------------
+
+class Quantized(NamedTuple):
+    codes: torch.Tensor          # uint8 [rows, cols/2]
+    scales: torch.Tensor         # uint8 [rows, cols/16] or [rows, cols/32]
+    tensor_scale: torch.Tensor   # float32 [1] (zero and unused for MXFP4)
+    mse: torch.Tensor | None     # float64 [1] or None
+
+
+def block_size(fmt) -> int:
+    return 32 if _fmt(fmt) == MXFP4 else 16
+
+
+def _check(status: int, what: str):
+    if status != SUCCESS:
+        raise Fp4qError(status, what)
+
+
+_workspaces: dict = {}
+
+
+def workspace_for(device: torch.device, stream=None) -> torch.Tensor:
+    """A cached workspace tensor per (device, stream); calls on one stream are ordered."""
+    key = (device, _stream(stream))
+    ws = _workspaces.get(key)
+    if ws is None:
+        n = lib().fp4q_workspace_size(0, 0, 0, 0)
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def _rows_cols_ld(x: torch.Tensor):
+    if x.dim() != 2:
+        raise ValueError("expected a 2-D tensor")
+    if x.stride(1) != 1:
+        raise ValueError("rows must be contiguous (stride(1) == 1)")
+    return x.shape[0], x.shape[1], x.stride(0) if x.shape[0] > 1 else x.shape[1]
+
+
+def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_scale: torch.Tensor | None = None,
+             want_mse: bool = True, out: Quantized | None = None, workspace: torch.Tensor | None = None,
+             stream=None) -> Quantized:
+    """Quantize a bf16 CUDA matrix; returns codes, scales, tensor scale and (optionally) the MSE."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda:
+        raise TypeError("x must be a bf16 CUDA tensor")
+    rows, cols, ld = _rows_cols_ld(x)
+    f = _fmt(fmt)
+    B = block_size(f)
+    dev = x.device
+    if out is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(rows, cols // B, dtype=torch.uint8, device=dev)
+        ts = torch.zeros(1, dtype=torch.float32, device=dev) if tensor_scale is None else tensor_scale
+        mse = torch.empty(1, dtype=torch.float64, device=dev) if want_mse else None
+    else:
+        codes, scales, ts, mse = out
+        if tensor_scale is not None:
+            ts = tensor_scale
+    ws = workspace if workspace is not None else workspace_for(dev, stream)
+    flags = FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0
+    st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
+    _check(st, "fp4q_quantize")
+    return Quantized(codes, scales, ts, mse)
+
+
+def dequantize(q: Quantized, fmt="nvfp4_razer", rotate: bool = False, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """bf16 reconstruction of a quantized matrix."""
+    rows, cols = q.codes.shape[0], q.codes.shape[1] * 2
+    y = out if out is not None else torch.empty(rows, cols, dtype=torch.bfloat16, device=q.codes.device)
+    ldy = y.stride(0) if rows > 1 else cols
+    st = fp4q_dequantize(q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, y, ldy, stream)
+    _check(st, "fp4q_dequantize")
+    return y
+
+
+def error(x: torch.Tensor, q: Quantized, fmt="nvfp4_razer", rotate: bool = False,
+          workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """MSE (fp64 [1] on the device) of the reconstruction against x."""
+    rows, cols, ld = _rows_cols_ld(x)
+    mse = torch.empty(1, dtype=torch.float64, device=x.device)
+    ws = workspace if workspace is not None else workspace_for(x.device, stream)
+    st = fp4q_error(x, ld, q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, mse, ws,
+                    ws.numel(), stream)
+    _check(st, "fp4q_error")
+    return mse

@@ -42,6 +42,11 @@ LLAMA3_70B_MLP = (
 )
 
 
+def tensor_seed(base: int, layer: int, index: int) -> int:
+    """Seed of tensor ``index`` of layer ``layer`` in a workload whose seed is ``base``."""
+    return int(base) * 1_000_000 + int(layer) * 100 + int(index)
+
+
 def _gen(seed: int, device) -> torch.Generator:
     g = torch.Generator(device=torch.device(device))
     g.manual_seed(int(seed))

@@ -1,0 +1,160 @@
+/*
+ * fp4q -- block-scaled 4-bit quantization of bf16 matrices on NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; every pointer argument to the tensor
+ * entry points is a DEVICE pointer owned by the caller.  The library never
+ * allocates, frees or synchronises inside these calls: each call validates its
+ * arguments on the host, then enqueues kernels on `stream` and returns.
+ *
+ * Formats (element codes are 4-bit E2M1, sign in bit 3, magnitude index in
+ * bits 0..2 over {0, 0.5, 1, 1.5, 2, 3, 4, 6} -- the FP4 value set of "RaZeR:
+ * Pushing the Limits of NVFP4 Quantization with Redundant Zero Remapping",
+ * technical summary sect. 1):
+ *
+ *  FP4Q_NVFP4        16-element blocks along a row.  Block scale: one FP8
+ *                    E4M3 byte (the E4M3 block scale of RaZeR sect. 1).  Per
+ *                    tensor: one fp32 scale s_t = RN(amax / (6 * 448)), so the
+ *                    tensor maximum maps onto the largest code times the
+ *                    largest E4M3 value.  Block b: sb = E4M3_RNE_sat(
+ *                    RN(amax_b / RN(6 s_t))), den = RN(dec(sb) * s_t),
+ *                    element code = nearest E2M1 to RN(x * RN(1 / den)),
+ *                    ties to the even code, saturating at 6, zero as +0.
+ *                    Reconstruction: RN(value(code) * den).
+ *  FP4Q_NVFP4_RAZER  NVFP4 with redundant-zero remapping (RaZeR sect. 2.2):
+ *                    code 0b1000 (the spare -0) means the special value +5,
+ *                    or -5 when bit 7 of the scale byte (the spare sign bit of
+ *                    the positive E4M3 scale) is set.  Per block the encoder
+ *                    keeps the NVFP4 scale and codes, then picks the member of
+ *                    {+5, -5} that lowers the block's squared error more (ties
+ *                    and blocks with no gain keep +5 and bit 7 clear) and
+ *                    recodes every element strictly closer to it than to its
+ *                    regular value as 0b1000.  The scale magnitude is
+ *                    bits 0..6.
+ *  FP4Q_MXFP4        32-element blocks sharing one power-of-two scale ("TORQ:
+ *                    Two-Level Orthogonal Rotation for MXFP4 Quantization",
+ *                    technical summary sect. 1).  Scale byte E8M0 = e + 127
+ *                    with e = clamp(floor(log2 amax_b) - 2, -127, 127);
+ *                    element code = nearest E2M1 to x * 2^-e (exact scaling).
+ *                    No tensor scale.
+ *
+ * rotate = 1 applies, before quantization, the orthonormal 32-point
+ * Walsh-Hadamard transform y = RN(RN(H32 x) * RN(1/sqrt 32)) to every aligned
+ * group of 32 elements of a row (H32 in Sylvester order; an orthogonal
+ * intra-block rotation in the sense of TORQ sect. 2).  Quantization then acts
+ * on y.  On dequantize and error, rotate = 1 means the codes hold rotated
+ * values and the output is mapped back to the original domain with the same
+ * (self-inverse) transform.  The butterfly is summed in fp32, so rotated
+ * results can differ from an exact-sum reference by fp32 rounding.
+ *
+ * Layouts (all dense, row-major, caller-allocated, 16-byte aligned):
+ *  x, y      bf16 [rows][ld], ld >= cols, ld a multiple of 8 elements.
+ *  codes     uint8 [rows][cols/2]; element 2k in the low nibble of byte k.
+ *  scales    uint8 [rows][cols/16] (NVFP4, NVFP4_RAZER) or [rows][cols/32] (MXFP4).
+ *  tensor_scale  one fp32 (NVFP4 formats; may be NULL for MXFP4).
+ *  mse       one fp64: sum over all elements of (x - x^)^2 / (rows*cols),
+ *            x^ the fp32 reconstruction (before any bf16 rounding) in the
+ *            original domain, summed in fp64 in a fixed order.
+ *
+ * Shapes: cols must be a multiple of the block length (16 or 32) and of 32
+ * when rotating.  rows * cols == 0 is allowed: nothing is launched except the
+ * clearing of the scalar outputs (tensor_scale when computed, mse) to 0.
+ *
+ * Inputs must be finite.  NaN or infinity in x, a NaN scale byte (0x7F / 0xFF
+ * in E4M3, 0xFF in E8M0) or a non-finite tensor scale are outside the
+ * contract; the kernels do not fault on them, but the outputs are undefined.
+ *
+ * Errors: argument problems are reported before any launch as a status code,
+ * and nothing is enqueued.  FP4Q_ERROR_CUDA reports a failed launch (the
+ * library's own cudaGetLastError after its launches).  No call aborts,
+ * throws, or falls back to the CPU.
+ *
+ * Thread safety: calls may come from any host thread.  A workspace buffer
+ * must not be used by two calls that can run concurrently on the device.
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP4Q_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FP4Q_API __attribute__((visibility("default")))
+#else
+#define FP4Q_API
+#endif
+
+typedef enum {
+    FP4Q_NVFP4 = 0,
+    FP4Q_NVFP4_RAZER = 1,
+    FP4Q_MXFP4 = 2
+} fp4q_format_t;
+
+typedef enum {
+    FP4Q_SUCCESS = 0,
+    FP4Q_ERROR_INVALID_VALUE = 1,     /* null pointer, bad enum, bad flag, negative size */
+    FP4Q_ERROR_SHAPE = 2,             /* cols not a multiple of the block / rotation group, ld < cols, size overflow */
+    FP4Q_ERROR_MISALIGNED = 3,        /* pointer not 16-byte aligned, ld not a multiple of 8 */
+    FP4Q_ERROR_WORKSPACE = 4,         /* workspace missing, misaligned or smaller than fp4q_workspace_size() */
+    FP4Q_ERROR_UNSUPPORTED_DEVICE = 5,/* current device is not compute capability 10.0 (B200 / sm_100a) */
+    FP4Q_ERROR_CUDA = 6               /* a CUDA runtime call or kernel launch failed */
+} fp4q_status_t;
+
+/* NVFP4 formats: *tensor_scale is an input; the tensor-absmax pass is skipped. */
+#define FP4Q_FLAG_TENSOR_SCALE_GIVEN 0x1u
+
+/* The stream type is CUDA's cudaStream_t (a CUstream_st*); NULL is the legacy default stream. */
+typedef struct CUstream_st* fp4q_stream_t;
+
+/* FP4Q_ABI_VERSION of the loaded library. */
+FP4Q_API int fp4q_abi_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+FP4Q_API const char* fp4q_status_string(fp4q_status_t status);
+
+/* Bytes of device workspace fp4q_quantize and fp4q_error need for this shape
+ * (per-CTA partial maxima and partial sums).  Independent of the data. */
+FP4Q_API size_t fp4q_workspace_size(int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate);
+
+/* Quantize x (bf16 [rows][ldx]) into codes and scales.
+ *  fmt, rotate    as above.
+ *  flags          0 or FP4Q_FLAG_TENSOR_SCALE_GIVEN.
+ *  codes, scales  outputs, layouts above.
+ *  tensor_scale   NVFP4 formats: output (computed from the tensor absmax, of
+ *                 the rotated values when rotate = 1), or input with the flag.
+ *                 Ignored for MXFP4 (may be NULL).
+ *  mse            nullable output; when NULL the error is not computed at all.
+ *  workspace      device scratch of at least fp4q_workspace_size() bytes,
+ *                 16-byte aligned; contents on entry are ignored.
+ * Enqueues up to three kernels on `stream`: tensor absmax (NVFP4 formats
+ * without the flag), the fused quantize pass, and the mse finaliser (when mse
+ * is requested). */
+FP4Q_API fp4q_status_t fp4q_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                            fp4q_format_t fmt, int rotate, uint32_t flags,
+                            uint8_t* codes, uint8_t* scales, float* tensor_scale, double* mse,
+                            void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
+
+/* Reconstruct y (bf16 [rows][ldy], round to nearest even from the fp32
+ * reconstruction) from codes, scales and, for NVFP4 formats, *tensor_scale.
+ * One kernel; no workspace. */
+FP4Q_API fp4q_status_t fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                              int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
+                              void* y, int64_t ldy, fp4q_stream_t stream);
+
+/* Mean squared error of the reconstruction of (codes, scales, tensor_scale)
+ * against x (bf16 [rows][ldx]); *mse as in fp4q_quantize.  Two kernels. */
+FP4Q_API fp4q_status_t fp4q_error(const void* x, int64_t ldx,
+                         const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                         int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
+                         double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

@@ -1,0 +1,141 @@
+"""C ABI checks that need no GPU: the library builds and loads, exports every
+symbol include/fp4q.h declares, and rejects bad arguments on the host before
+touching the device.  Pointers here are fake addresses: every call below fails
+validation (or the device check) before any pointer is dereferenced."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from activation_quantization_block_b200 import fp4q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4q.h")
+
+ST = {name: code for code, name in fp4q.STATUS_NAMES.items()}
+A = 1 << 20          # a 16-byte-aligned fake address
+WS = fp4q.fp4q_workspace_size(0, 0, 0, 0)
+
+
+def declared_symbols() -> list[str]:
+    text = open(HEADER).read()
+    return re.findall(r"FP4Q_API\s+[\w\s\*]+?\b(fp4q_\w+)\s*\(", text)
+
+
+def test_header_declares_what_the_binding_knows():
+    assert sorted(declared_symbols()) == sorted(fp4q.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(fp4q.library_path() if os.path.exists(fp4q.library_path()) else fp4q.lib()._name)
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_version_status_strings_workspace():
+    assert fp4q.fp4q_abi_version() == 1
+    for code in range(7):
+        assert fp4q.fp4q_status_string(code)
+    assert fp4q.fp4q_status_string(99) == "unknown status"
+    assert WS >= 4096 * 12
+
+
+def q(**kw):
+    args = dict(x=A, rows=4, cols=64, ldx=64, fmt=0, rotate=0, flags=0, codes=A, scales=A, tensor_scale=A,
+                mse=None, workspace=A, workspace_bytes=WS, stream=0)
+    args.update(kw)
+    return fp4q.fp4q_quantize(**args)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(fmt=3), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(fmt=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rotate=2), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(flags=2), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(cols=40, ldx=40), "FP4Q_ERROR_SHAPE"),                 # not a multiple of 16
+    (dict(fmt=2, cols=48, ldx=48), "FP4Q_ERROR_SHAPE"),          # MXFP4 needs 32
+    (dict(rotate=1, cols=48, ldx=48), "FP4Q_ERROR_SHAPE"),       # rotation needs 32
+    (dict(ldx=32), "FP4Q_ERROR_SHAPE"),                          # ld < cols
+    (dict(rows=1 << 40, cols=1 << 30, ldx=1 << 30), "FP4Q_ERROR_SHAPE"),   # size overflow
+    (dict(x=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(codes=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(scales=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(tensor_scale=None), "FP4Q_ERROR_INVALID_VALUE"),       # NVFP4 needs it
+    (dict(x=A + 8), "FP4Q_ERROR_MISALIGNED"),
+    (dict(ldx=68), "FP4Q_ERROR_MISALIGNED"),
+    (dict(codes=A + 4), "FP4Q_ERROR_MISALIGNED"),
+    (dict(scales=A + 1), "FP4Q_ERROR_MISALIGNED"),
+    (dict(tensor_scale=A + 2), "FP4Q_ERROR_MISALIGNED"),
+    (dict(mse=A + 4), "FP4Q_ERROR_MISALIGNED"),
+    (dict(workspace=None), "FP4Q_ERROR_WORKSPACE"),
+    (dict(workspace=A + 8), "FP4Q_ERROR_WORKSPACE"),
+    (dict(workspace_bytes=WS - 1), "FP4Q_ERROR_WORKSPACE"),
+])
+def test_quantize_rejects_bad_arguments_before_launch(kw, expect):
+    assert q(**kw) == ST[expect]
+
+
+def test_quantize_argument_rules_that_relax():
+    # MXFP4 needs no tensor scale; a given tensor scale and no mse need no workspace.
+    ok_then_device = {ST["FP4Q_ERROR_CUDA"], ST["FP4Q_ERROR_UNSUPPORTED_DEVICE"], ST["FP4Q_SUCCESS"]}
+    if not _no_gpu():
+        pytest.skip("these calls would launch on a real device")
+    assert q(fmt=2, tensor_scale=None) in ok_then_device
+    assert q(flags=1, workspace=None, workspace_bytes=0) in ok_then_device
+
+
+def _no_gpu() -> bool:
+    import torch
+    return not torch.cuda.is_available()
+
+
+def test_no_cpu_fallback_without_a_device():
+    """On a machine with no GPU a valid call reports a CUDA error; nothing runs on the CPU."""
+    if not _no_gpu():
+        pytest.skip("a device is present")
+    assert q() == ST["FP4Q_ERROR_CUDA"]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(fmt=5), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(cols=24), "FP4Q_ERROR_SHAPE"),
+    (dict(y=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(y=A + 2), "FP4Q_ERROR_MISALIGNED"),
+    (dict(ldy=60), "FP4Q_ERROR_SHAPE"),
+    (dict(tensor_scale=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(codes=A + 8), "FP4Q_ERROR_MISALIGNED"),
+])
+def test_dequantize_rejects_bad_arguments(kw, expect):
+    args = dict(codes=A, scales=A, tensor_scale=A, rows=4, cols=64, fmt=1, rotate=0, y=A, ldy=64, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_dequantize(**args) == ST[expect]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(mse=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(mse=A + 4), "FP4Q_ERROR_MISALIGNED"),
+    (dict(workspace=None), "FP4Q_ERROR_WORKSPACE"),
+    (dict(workspace_bytes=16), "FP4Q_ERROR_WORKSPACE"),
+    (dict(rotate=1, cols=16), "FP4Q_ERROR_SHAPE"),
+    (dict(x=A + 16, ldx=12), "FP4Q_ERROR_SHAPE"),
+])
+def test_error_rejects_bad_arguments(kw, expect):
+    args = dict(x=A, ldx=64, codes=A, scales=A, tensor_scale=A, rows=4, cols=64, fmt=0, rotate=0, mse=A,
+                workspace=A, workspace_bytes=WS, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_error(**args) == ST[expect]
+
+
+def test_binding_has_no_oracle_or_cpu_path():
+    """The product package never imports the oracle."""
+    pkg = os.path.join(ROOT, "activation_quantization_block_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "fp4q_oracle" not in text, f
