@@ -29,7 +29,7 @@ STATUS_NAMES = {
 
 # Names the C header declares; the tests check that the library exports each one.
 ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
-               "fp4q_quantize", "fp4q_dequantize", "fp4q_error")
+               "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc")
 
 
 class Fp4qError(RuntimeError):
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.fp4q_dequantize.restype = i32
         L.fp4q_error.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, sz, vp]
         L.fp4q_error.restype = i32
+        L.fp4q_quantize_noalloc.argtypes = [vp, i64, i64, i64, i32, i32, u32, vp, vp, vp, vp, vp]
+        L.fp4q_quantize_noalloc.restype = i32
         _lib = L
     return _lib
 
@@ -118,6 +120,13 @@ def fp4q_error(x, ldx, codes, scales, tensor_scale, rows, cols, fmt, rotate, mse
     return lib().fp4q_error(_ptr(x), ldx, _ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, cols,
                             _fmt(fmt), int(rotate), _ptr(mse), _ptr(workspace), workspace_bytes,
                             _stream(stream))
+
+
+def fp4q_quantize_noalloc(x, rows, cols, ldx, fmt, rotate, flags, codes, scales, tensor_scale, mse,
+                          stream=None) -> int:
+    """fp4q_quantize with the library's static scratch: for callers that cannot allocate."""
+    return lib().fp4q_quantize_noalloc(_ptr(x), rows, cols, ldx, _fmt(fmt), int(rotate), flags, _ptr(codes),
+                                       _ptr(scales), _ptr(tensor_scale), _ptr(mse), _stream(stream))
 
 
 # ---- torch-level wrappers -------------------------------------------------------

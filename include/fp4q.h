@@ -153,6 +153,36 @@ FP4Q_API fp4q_status_t fp4q_error(const void* x, int64_t ldx,
                          int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
                          double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
 
+/* Bytes of device scratch held inside the library for fp4q_quantize_noalloc. */
+#define FP4Q_NOALLOC_SCRATCH_BYTES 49152
+
+/* fp4q_quantize for callers that cannot allocate device memory.
+ *
+ * No counterpart in the papers: this is a library convenience.  It exists for
+ * code that must not call cudaMalloc (or any allocator) where it quantizes --
+ * e.g. a plugin inside a program that owns all device memory, or a latency
+ * path that cannot afford the synchronisation an allocation can imply -- and
+ * so has no workspace to pass.  Arguments, outputs and results are those of
+ * fp4q_quantize; the scratch comes from a static device array of
+ * FP4Q_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
+ * until the process exits.  The call allocates nothing and frees nothing.
+ *
+ *  - The first call on each device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents.  Nothing in it needs clearing (each call writes every
+ *    slot it reads), but calls that can overlap on the GPU -- on different
+ *    streams without ordering between them -- race on it.  Order them on one
+ *    stream or by events.
+ *  - A shape whose scratch need (fp4q_workspace_size) exceeds the array is
+ *    rejected with FP4Q_ERROR_WORKSPACE before anything is enqueued; with the
+ *    present kernels every shape fits. */
+FP4Q_API fp4q_status_t fp4q_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                             fp4q_format_t fmt, int rotate, uint32_t flags,
+                                             uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                             double* mse, fp4q_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
