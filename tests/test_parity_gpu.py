@@ -275,14 +275,15 @@ def test_tensor_scale_given(orc, dev, fmt):
 
 
 def test_representable_inputs_are_fixed_points(orc, dev):
-    """Quantizing the reconstruction returns the same codes (all formats)."""
+    """Quantizing the bf16 reconstruction returns the same codes (all formats); what
+    remains of the error is only the bf16 rounding of the reconstruction."""
     x = synthetic.llm_weight(128, 512, seed=12, device="cpu").to(dev)
     for fmt in FMTS:
         q = fp4q.quantize(x, fmt)
         y = fp4q.dequantize(q, fmt)
         q2 = fp4q.quantize(y, fmt)
         assert torch.equal(q.codes, q2.codes) and torch.equal(q.scales, q2.scales)
-        assert q2.mse.item() == 0.0
+        assert q2.mse.item() < 1e-2 * q.mse.item()
 
 
 def test_razer_worked_block_on_gpu(orc, dev):
