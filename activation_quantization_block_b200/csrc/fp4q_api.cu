@@ -196,4 +196,18 @@ fp4q_status_t fp4q_error(const void* x, int64_t ldx,
     return from_cuda(launch_sse_finalize(sse_part, n_sse, (double)n, mse, st));
 }
 
+fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
+{
+    if (bits == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    unsigned int v = 0;
+    if (read_device_errors(&v, clear != 0) != cudaSuccess) {
+        cudaGetLastError();
+        return FP4Q_ERROR_CUDA;
+    }
+    *bits = v;
+    return FP4Q_SUCCESS;
+}
+
 }  // extern "C"

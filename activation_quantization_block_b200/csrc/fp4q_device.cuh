@@ -25,10 +25,71 @@ __device__ __forceinline__ float wht_scale() { return __uint_as_float(0x3E3504F3
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Both halves widened with the mixed-precision add (x + -0 is exact for every
+// finite x, zeros keep their sign), which runs on the FMA pipe rather than on
+// the integer pipe.
+__device__ __forceinline__ float2 bf16x2_to_f32(uint32_t w)
+{
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, 0f80000000;\n\tadd.rn.f32.bf16 %1, h, 0f80000000;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w));
+    return make_float2(lo, hi);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// max(|a|, |b|) of two bf16 pairs at once (the sign bits of the result are the
+// xor of the inputs' and carry no meaning here); exact.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// |max| of the two bf16 halves of a word, as fp32.
+__device__ __forceinline__ float bf16x2_hmax_abs(uint32_t w)
+{
+    return fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w)));
+}
+
+// ---- packed fp32 pairs (IEEE round-to-nearest per lane, no flush to zero) ----
+
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b)
+{
+    float2 r;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b)
+{
+    float2 r;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// a * b + c per lane, one rounding.
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c)
+{
+    float2 r;
+    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
 }
 
 // ---- E2M1 -----------------------------------------------------------------
@@ -56,6 +117,25 @@ __device__ __forceinline__ uint32_t canonical_zero(uint32_t w)
 {
     uint32_t nz = (w & 0x77777777u) + 0x77777777u;
     return w & ((nz & 0x88888888u) | 0x77777777u);
+}
+
+// Eight E2M1 nibbles (one word, element i in bits 4i..4i+3) -> eight fp32
+// values; the word is split into bytes inside the conversion block.
+__device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float* q)
+{
+    uint32_t h0, h1, h2, h3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(w));
+    const uint32_t h[4] = {h0, h1, h2, h3};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
+        q[2 * k] = f.x;
+        q[2 * k + 1] = f.y;
+    }
 }
 
 // Two E2M1 nibbles (bits 0..3 element 2k, bits 4..7 element 2k+1) -> two fp32 values.

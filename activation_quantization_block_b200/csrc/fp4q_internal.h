@@ -55,4 +55,8 @@ cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t*
 cudaError_t launch_sse_finalize(const double* partials, int n, double count, double* mse,
                                 cudaStream_t st);
 
+// Copy the device error word of the current device to *bits (synchronous);
+// clear it afterwards when asked.
+cudaError_t read_device_errors(unsigned int* bits, bool clear);
+
 }  // namespace fp4q

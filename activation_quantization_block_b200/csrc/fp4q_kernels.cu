@@ -1,15 +1,22 @@
 // fp4q kernels for sm_100a: tensor absmax, fused quantize, dequantize, error,
 // and the fixed-order fp64 finaliser for the squared-error sums.
 //
-// Work decomposition.  A bf16 matrix is a sequence of 16-element halves (one
-// NVFP4 block each); one thread owns a unit of two consecutive halves, i.e.
-// 32 elements = 64 bytes of input, 16 bytes of codes and 2 (NVFP4) or 1
-// (MXFP4) scale bytes.  With rotation or MXFP4 the two halves are one aligned
-// 32-group of a row, so the whole Walsh-Hadamard butterfly runs in the
-// thread's registers.  Consecutive lanes own consecutive units, so each warp
-// streams 2 KB of input and writes 512 contiguous bytes of codes per step.
-// Kernels are grid-strided over units with a grid sized to the resident
-// capacity of the device.
+// Work decomposition.  Every kernel streams 16 KB tiles of 128 rows x 64 bf16
+// through a TMA pipeline (fp4q_tma.cuh).  A contiguous matrix whose size is a
+// multiple of 64 is viewed as [N/64][64] ("flat"), so a tile is 16 KB of
+// consecutive elements; otherwise the view is [rows][cols] with the row
+// stride, and a tile is 128 rows x 64 columns.  Thread t of a CTA owns the
+// unit (tile row t/2, half t%2): 32 consecutive elements of one matrix row,
+// i.e. two NVFP4 blocks or one MXFP4 block / rotation group, 16 bytes of
+// codes and 2 (NVFP4) or 1 (MXFP4) scale bytes.  The 32-point rotation runs
+// in the thread's registers.  Grids are persistent (resident CTAs per SM x
+// SMs) and walk the tiles round-robin.
+//
+// Kernels of one call are chained with programmatic dependent launch: the
+// quantize pass starts fetching its first tiles while the absmax pass drains
+// and waits (griddepcontrol.wait) only before it reads the absmax partials;
+// the absmax pass walks the tiles forwards and the quantize pass backwards, so
+// the quantize pass begins on the tiles the absmax pass left in L2.
 //
 // Method references (title, section):
 //  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant Zero
@@ -18,8 +25,9 @@
 //   chosen per block by minimum squared error; one bit -> the pair +-5).
 //  "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization": sect. 1
 //   (32-element blocks, shared exponent, e2m1 codebook), sect. 2 (orthogonal
-//   intra-block rotation before quantization; S-step maps the block maximum
-//   to the top of the code range).
+//   intra-block rotation before quantization).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -29,52 +37,89 @@
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
+#include "fp4q_tma.cuh"
 
 namespace fp4q {
 
 enum { kNV = 0, kRZ = 1, kMX = 2 };
 
+// Device error word (bits: kErrPipelineTimeout); read and cleared through the C ABI.
+__device__ unsigned int g_device_error;
+
 // ---------------------------------------------------------------------------
-// Geometry helpers
+// Tiles and units
 // ---------------------------------------------------------------------------
 
-// Element offset of half h.  CONTIG: rows are packed (ld == cols).
-template <bool CONTIG>
-__device__ __forceinline__ int64_t half_offset(const Geometry& g, int64_t h)
-{
-    if (CONTIG) return h * 16;
-    int64_t row = h / g.halves_per_row;
-    int64_t c = h - row * g.halves_per_row;
-    return row * g.ld + c * 16;
-}
+struct Tiles {
+    int64_t count;       // number of tiles
+    int64_t col_tiles;   // 2-D view: tiles across the columns (ceil(cols / 64))
+    int64_t rows, cols;  // matrix shape
+    int64_t units;       // flat view: N / 32
+};
 
-// Load the 32 bf16 of unit u as 16 words.  PAIRED: both halves are known to
-// lie in one row (cols a multiple of 32), so the second half follows the first.
-template <bool CONTIG, bool PAIRED>
-__device__ __forceinline__ void load_unit(const uint16_t* __restrict__ x, const Geometry& g, int64_t u,
-                                          bool full, uint32_t* w)
+template <bool FLAT>
+__device__ __forceinline__ void tile_origin(const Tiles& tl, int64_t k, int& x, int& y)
 {
-    const int64_t h0 = 2 * u;
-    const uint16_t* p0 = x + half_offset<CONTIG>(g, h0);
-    uint4 a = ldg_nc_v4(p0), b = ldg_nc_v4(p0 + 8);
-    uint4 c = make_uint4(0, 0, 0, 0), d = make_uint4(0, 0, 0, 0);
-    if (full) {
-        const uint16_t* p1 = (CONTIG || PAIRED) ? p0 + 16 : x + half_offset<CONTIG>(g, h0 + 1);
-        c = ldg_nc_v4(p1);
-        d = ldg_nc_v4(p1 + 8);
+    if (FLAT) {
+        x = 0;
+        y = (int)(k * kTileRows);
+    } else {
+        const int64_t rt = k / tl.col_tiles;
+        x = (int)((k - rt * tl.col_tiles) * kTileCols);
+        y = (int)(rt * kTileRows);
     }
-    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    w[8] = c.x; w[9] = c.y; w[10] = c.z; w[11] = c.w;
-    w[12] = d.x; w[13] = d.y; w[14] = d.z; w[15] = d.w;
 }
 
-__device__ __forceinline__ void unpack32(const uint32_t* w, float* y)
+// The unit thread t owns in tile k: its row and column, whether it exists,
+// whether both 16-element halves exist, and its unit index in the flat view.
+struct Unit {
+    int64_t row, col, flat;
+    bool valid, full;
+};
+
+template <bool FLAT>
+__device__ __forceinline__ Unit unit_of(const Tiles& tl, int64_t k, int t)
 {
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        y[2 * k] = bf16_lo(w[k]);
-        y[2 * k + 1] = bf16_hi(w[k]);
+    Unit u;
+    if (FLAT) {
+        u.flat = k * (2 * kTileRows) + t;
+        u.valid = u.flat < tl.units;
+        u.full = true;
+        u.row = u.col = 0;
+    } else {
+        const int64_t rt = k / tl.col_tiles;
+        const int64_t ct = k - rt * tl.col_tiles;
+        u.row = rt * kTileRows + (t >> 1);
+        u.col = ct * kTileCols + 32 * (t & 1);
+        u.valid = u.row < tl.rows && u.col < tl.cols;
+        u.full = u.col + 32 <= tl.cols;
+        u.flat = 0;
+    }
+    return u;
+}
+
+// Offsets of a unit's codes and scale bytes in the dense layouts.
+template <bool FLAT, int FMT>
+__device__ __forceinline__ void unit_offsets(const Tiles& tl, const Unit& u, int64_t& code_off, int64_t& scale_off)
+{
+    constexpr int B = FMT == kMX ? 32 : 16;
+    if (FLAT) {
+        code_off = 16 * u.flat;
+        scale_off = (32 / B) * u.flat;
+    } else {
+        code_off = u.row * (tl.cols / 2) + u.col / 2;
+        scale_off = u.row * (tl.cols / B) + u.col / B;
+    }
+}
+
+// Store 16 (full) or 8 bytes of codes; a16 tells whether the address is 16-byte aligned.
+__device__ __forceinline__ void store_codes(uint8_t* p, const uint32_t* cw, bool full, bool a16)
+{
+    if (full && a16) {
+        stg_v4(p, make_uint4(cw[0], cw[1], cw[2], cw[3]));
+    } else {
+        stg_v2(p, cw[0], cw[1]);
+        if (full) stg_v2(p + 8, cw[2], cw[3]);
     }
 }
 
@@ -117,88 +162,228 @@ __device__ __forceinline__ double block_sum(double v, double* sh)
 }
 
 // ---------------------------------------------------------------------------
-// Per-block encoders
+// Squared error
 // ---------------------------------------------------------------------------
 
-// One 16-element NVFP4 block.  y: the (rotated) values; s_t / six_st: tensor
-// scale and RN(6 s_t).  Writes two code words and the scale byte; with SSE,
-// xh receives the fp32 reconstruction RN(q * den).
-template <bool RAZER, bool SSE>
-__device__ __forceinline__ void encode_nv16(const float* y, float s_t, float six_st, uint32_t* cw,
-                                            uint32_t& sb_out, float* xh)
+// Sum of squares of 16 differences, exact in fp64 range: the values are
+// scaled by 2^-k, 2^k the power of two at or below their largest magnitude
+// (in two exact steps, so 2^-k never overflows), squared and summed in fp32,
+// and the sum is scaled back by 2^2k in fp64.  Used when a fast fp32 sum
+// overflowed or may have lost terms to underflow (|x| near the top of the bf16
+// range, or bf16 subnormals).
+__device__ __forceinline__ double sse16_rescaled(const float* d)
 {
-    float a = 0.0f;
+    float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(y[i]));
-    const float t = six_st > 0.0f ? __fdiv_rn(a, six_st) : 0.0f;
-    uint32_t sb = e4m3_rn_satfinite(t);
-    const float den = __fmul_rn(e4m3_to_f32(sb), s_t);
-    const float r = den != 0.0f ? __frcp_rn(den) : 0.0f;   // zero scale -> every code 0
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(d[i]));
+    if (m == 0.0f || !(m <= 3.4e38f)) return m == 0.0f ? 0.0 : (double)INFINITY;
+    const int k = floor_log2_f32(m);              // in [-149, 127]
+    const int k1 = -k / 2, k2 = -k - k1;           // each in [-64, 75]
+    const float s1 = __uint_as_float((uint32_t)(k1 + 127) << 23);
+    const float s2 = __uint_as_float((uint32_t)(k2 + 127) << 23);
+    float es = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float t = __fmul_rn(__fmul_rn(d[i], s1), s2);
+        es = __fmaf_rn(t, t, es);
+    }
+    return (double)es * __longlong_as_double((long long)(2 * k + 1023) << 52);
+}
+
+// Sum of squared errors of 16 values (x - xh), the differences in fp32.
+__device__ __forceinline__ double sse16(const float* x, const float* xh)
+{
+    float2 acc = make_float2(0.0f, 0.0f);
+    float d[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 e = sub2_rn(make_float2(x[i], x[i + 1]), make_float2(xh[i], xh[i + 1]));
+        d[i] = e.x;
+        d[i + 1] = e.y;
+        acc = fma2_rn(e, e, acc);
+    }
+    const float es = acc.x + acc.y;
+    if (es >= 0x1p-100f && es <= 3.0e38f) return (double)es;
+    return sse16_rescaled(d);
+}
+
+template <int N>
+__device__ __forceinline__ double sse_of(const float* x, const float* xh)
+{
+    double e = sse16(x, xh);
+    if (N == 32) e += sse16(x + 16, xh + 16);
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// Encoders
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void unpack16(const uint32_t* w, float* y)
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float2 p = bf16x2_to_f32(w[k]);
+        y[2 * k] = p.x;
+        y[2 * k + 1] = p.y;
+    }
+}
+
+// Decode 16 codes (two words) to their E2M1 values.
+__device__ __forceinline__ void decode16(uint32_t w0, uint32_t w1, float* q)
+{
+    e2m1x8_to_f32(w0, q);
+    e2m1x8_to_f32(w1, q + 8);
+}
+
+// Per-tensor constants of the NVFP4 block-scale step, shared by a CTA: for
+// each of the 127 non-negative finite E4M3 bytes b, den[b] = RN(dec(b) * s_t)
+// and rcp[b] = RN(1 / den[b]) (0 when den[b] = 0: a zero scale zeroes every
+// code).  The quotient t = RN(a / RN(6 s_t)) uses inv6 = RN(1 / RN(6 s_t)) and
+// one correction step (Markstein's theorem: with y = RN(1/b) and a faithful
+// q = RN(a y), the residual r = a - q b is exact and RN(q + r y) = RN(a / b));
+// `exact_div` selects IEEE division when RN(6 s_t) is outside [2^-64, 2^64],
+// where the theorem's no-underflow conditions are not guaranteed.
+struct NvScale {
+    float s_t, six_st, inv6;
+    bool exact_div;
+    const float* den;
+    const float* rcp;
+};
+
+__device__ __forceinline__ NvScale nv_scale_setup(float s_t, float* den_tab, float* rcp_tab)
+{
+    NvScale c;
+    c.s_t = s_t;
+    c.six_st = __fmul_rn(6.0f, s_t);
+    c.exact_div = !(c.six_st >= 0x1p-64f && c.six_st <= 0x1p64f);
+    c.inv6 = c.exact_div ? 0.0f : __frcp_rn(c.six_st);
+    for (int b = threadIdx.x; b < 128; b += blockDim.x) {
+        const float d = b < 127 ? __fmul_rn(e4m3_to_f32((uint32_t)b), s_t) : 0.0f;
+        den_tab[b] = d;
+        rcp_tab[b] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+    }
+    __syncthreads();
+    c.den = den_tab;
+    c.rcp = rcp_tab;
+    return c;
+}
+
+// t = RN(a / RN(6 s_t)) for a >= 0.
+__device__ __forceinline__ float nv_block_ratio(const NvScale& c, float a)
+{
+    if (c.exact_div) return c.six_st > 0.0f ? __fdiv_rn(a, c.six_st) : 0.0f;
+    const float q = __fmul_rn(a, c.inv6);
+    const float r = __fmaf_rn(-q, c.six_st, a);
+    return __fmaf_rn(r, c.inv6, q);
+}
+
+// Outputs of the block encoders besides codes and scale.
+enum { kOutNone = 0, kOutSse = 1, kOutXh = 2 };
+
+// One 16-element NVFP4 block.  y: values (rotated when rotating); a: their
+// absmax.  Writes two code words and the scale byte.  OUT = kOutXh: xh receives
+// the fp32 reconstruction RN(q * den).  OUT = kOutSse: *sse receives
+// sum (y - q den)^2, each difference taken with a single rounding
+// (RN(y - q den), within half an fp32 ulp of y - RN(q den)).
+template <bool RAZER, int OUT>
+__device__ __forceinline__ void encode_nv16(const float* y, float a, const NvScale& sc, uint32_t& c0, uint32_t& c1,
+                                            uint32_t& sb_out, float* xh, double* sse)
+{
+    uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
+    const float den = sc.den[sb];
+    const float r = sc.rcp[sb];
     float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], r);
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+        v[i] = p.x;
+        v[i + 1] = p.y;
+    }
     uint32_t w0 = canonical_zero(e2m1x8(v));
     uint32_t w1 = canonical_zero(e2m1x8(v + 8));
 
-    float q[16];
-    if (SSE) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 p = e2m1x2_to_f32((w0 >> (8 * k)) & 0xFFu);
-            q[2 * k] = p.x; q[2 * k + 1] = p.y;
-            float2 s = e2m1x2_to_f32((w1 >> (8 * k)) & 0xFFu);
-            q[8 + 2 * k] = s.x; q[8 + 2 * k + 1] = s.y;
-        }
-    }
-
+    float win[16];
+    float special = 0.0f;
     if (RAZER) {
-        // Gain of remapping element i to sign(v_i) * 5: for |v_i| in (4.5, 5.5)
-        // the regular value is 4 (|v| <= 5) or 6, and
+        // Gain of remapping element i to sign(v_i) * 5.  For |v_i| in (4.5, 5.5)
+        // the regular value is 4 (|v| <= 5) or 6 and
         //   (|v| - q)^2 - (|v| - 5)^2 = 1 - 2 | |v| - 5 |,
-        // positive exactly on that open interval and clamped to 0 elsewhere.
-        // Every term is a multiple of 2^-20 in [0, 1], so the fp32 sums below
-        // are exact in any order.  S = gain(+5) - gain(-5), T = gain(+5) + gain(-5).
-        float S = 0.0f, T = 0.0f;
+        // which is positive exactly on that open interval; elsewhere it is
+        // clamped to 0.  Each term is a multiple of 2^-20 in [0, 1], so the fp32
+        // sum S = gain(+5) - gain(-5) is exact in any order.
+        float cs[16];
+        float S = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float c = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
-            S += copysignf(c, v[i]);
-            T += c;
+            cs[i] = copysignf(c, v[i]);
+            S += cs[i];
         }
-        if (T > 0.0f) {
-            const bool neg = S < 0.0f;   // -5 only when strictly better
-            uint32_t m0 = 0, m1 = 0;
+        // -5 only when its gain is strictly larger.  Winners are the candidates
+        // of the chosen sign: cs * sign >= 2^-20, so win = sat(cs * sign * 2^40)
+        // is exactly 1 for a winner and 0 otherwise (+0 or -0).
+        const float sk = S < 0.0f ? -0x1p40f : 0x1p40f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float c = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
-                const bool win = c > 0.0f && (signbit(v[i]) != 0) == neg;
-                if (win) {
-                    if (i < 8) m0 |= 0xFu << (4 * i);
-                    else m1 |= 0xFu << (4 * (i - 8));
-                    if (SSE) q[i] = neg ? -5.0f : 5.0f;
+        for (int i = 0; i < 16; ++i) win[i] = __saturatef(__fmul_rn(cs[i], sk));
+        // E2M1 of 1.0 is 0b0010 and of +-0 is 0b0000 / 0b1000: bit 1 of each
+        // nibble flags a winner; winners' codes become 0b1000.
+        const uint32_t f0 = (e2m1x8(win) >> 1) & 0x11111111u;
+        const uint32_t f1 = (e2m1x8(win + 8) >> 1) & 0x11111111u;
+        w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
+        w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
+        if (S < 0.0f) sb |= 0x80u;
+        special = S < 0.0f ? -5.0f : 5.0f;
+    }
+
+    if (OUT != kOutNone) {
+        // codes as written (RaZeR winners decode to -0 here and are fixed below)
+        float q[16];
+        decode16(w0, w1, q);
+        if (OUT == kOutSse) {
+            const float nden = -den;
+            const float nx5 = -__fmul_rn(special, den);   // -RN(special * den)
+            float2 acc = make_float2(0.0f, 0.0f);
+            float d[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float2 e = fma2_rn(make_float2(q[i], q[i + 1]), make_float2(nden, nden),
+                                   make_float2(y[i], y[i + 1]));
+                if (RAZER) e = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(nx5, nx5), e);
+                d[i] = e.x;
+                d[i + 1] = e.y;
+                acc = fma2_rn(e, e, acc);
+            }
+            const float es = acc.x + acc.y;
+            *sse = (es >= 0x1p-100f && es <= 3.0e38f) ? (double)es : sse16_rescaled(d);
+        } else {
+            if (RAZER) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    // winners: -0 + 1 * special; others: q + 0 * special
+                    const float2 n = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(special, special),
+                                             make_float2(q[i], q[i + 1]));
+                    q[i] = n.x;
+                    q[i + 1] = n.y;
                 }
             }
-            w0 = (w0 & ~m0) | (m0 & 0x88888888u);
-            w1 = (w1 & ~m1) | (m1 & 0x88888888u);
-            if (neg) sb |= 0x80u;
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(den, den));
+                xh[i] = p.x;
+                xh[i + 1] = p.y;
+            }
         }
     }
-    if (SSE) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(q[i], den);
-    }
-    cw[0] = w0;
-    cw[1] = w1;
+    c0 = w0;
+    c1 = w1;
     sb_out = sb;
 }
 
 // One 32-element MXFP4 block.
-template <bool SSE>
-__device__ __forceinline__ void encode_mx32(const float* y, uint32_t* cw, uint32_t& sb_out, float* xh)
+template <bool XH>
+__device__ __forceinline__ void encode_mx32(const float* y, float a, uint32_t* cw, uint32_t& sb_out, float* xh)
 {
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(y[i]));
     int e = -127;
     float r = 0.0f;
     uint32_t sb = 0;
@@ -210,26 +395,30 @@ __device__ __forceinline__ void encode_mx32(const float* y, uint32_t* cw, uint32
     }
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(y[i], r);
+    for (int i = 0; i < 32; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+        v[i] = p.x;
+        v[i + 1] = p.y;
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) cw[k] = canonical_zero(e2m1x8(v + 8 * k));
-    if (SSE) {
+    if (XH) {
         const float s = exp2i(e);
+        float q[32];
+        decode16(cw[0], cw[1], q);
+        decode16(cw[2], cw[3], q + 16);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float2 p = e2m1x2_to_f32((cw[k] >> (8 * j)) & 0xFFu);
-                xh[8 * k + 2 * j] = __fmul_rn(p.x, s);
-                xh[8 * k + 2 * j + 1] = __fmul_rn(p.y, s);
-            }
+        for (int i = 0; i < 32; i += 2) {
+            const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(s, s));
+            xh[i] = p.x;
+            xh[i + 1] = p.y;
         }
     }
     sb_out = sb;
 }
 
 // ---------------------------------------------------------------------------
-// Decoders (shared by dequantize and error)
+// Decoders (dequantize and error)
 // ---------------------------------------------------------------------------
 
 template <bool RAZER>
@@ -237,60 +426,34 @@ __device__ __forceinline__ void decode_nv16(uint32_t w0, uint32_t w1, uint32_t s
 {
     const float den = __fmul_rn(e4m3_to_f32(RAZER ? (sb & 0x7Fu) : sb), s_t);
     const float special = (sb & 0x80u) ? -5.0f : 5.0f;
+    float q[16];
+    decode16(w0, w1, q);
+    if (RAZER) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t b0 = (w0 >> (8 * k)) & 0xFFu, b1 = (w1 >> (8 * k)) & 0xFFu;
-        float2 p = e2m1x2_to_f32(b0);
-        float2 s = e2m1x2_to_f32(b1);
-        if (RAZER) {
-            if ((b0 & 0xFu) == 8u) p.x = special;
-            if ((b0 >> 4) == 8u) p.y = special;
-            if ((b1 & 0xFu) == 8u) s.x = special;
-            if ((b1 >> 4) == 8u) s.y = special;
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t nib = ((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu;
+            q[i] = nib == 8u ? special : q[i];
         }
-        xh[2 * k] = __fmul_rn(p.x, den);
-        xh[2 * k + 1] = __fmul_rn(p.y, den);
-        xh[8 + 2 * k] = __fmul_rn(s.x, den);
-        xh[8 + 2 * k + 1] = __fmul_rn(s.y, den);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(den, den));
+        xh[i] = p.x;
+        xh[i + 1] = p.y;
     }
 }
 
 __device__ __forceinline__ void decode_mx32(const uint32_t* cw, uint32_t sb, float* xh)
 {
     const float s = exp2i((int)sb - 127);
+    float q[32];
+    decode16(cw[0], cw[1], q);
+    decode16(cw[2], cw[3], q + 16);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 p = e2m1x2_to_f32((cw[k] >> (8 * j)) & 0xFFu);
-            xh[8 * k + 2 * j] = __fmul_rn(p.x, s);
-            xh[8 * k + 2 * j + 1] = __fmul_rn(p.y, s);
-        }
-    }
-}
-
-// Read the codes and scale bytes of unit u (dense layouts).
-template <int FMT>
-__device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                            int64_t u, bool full, uint32_t* cw, uint32_t* sb)
-{
-    if (full) {
-        uint4 c = ldg_nc_v4(codes + 16 * u);
-        cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
-    } else {
-        uint2 c = *reinterpret_cast<const uint2*>(codes + 16 * u);
-        cw[0] = c.x; cw[1] = c.y; cw[2] = 0; cw[3] = 0;
-    }
-    if (FMT == kMX) {
-        sb[0] = __ldg(scales + u);
-        sb[1] = 0;
-    } else if (full) {
-        const uint32_t two = __ldg(reinterpret_cast<const unsigned short*>(scales) + u);
-        sb[0] = two & 0xFFu;
-        sb[1] = two >> 8;
-    } else {
-        sb[0] = __ldg(scales + 2 * u);
-        sb[1] = 0;
+    for (int i = 0; i < 32; i += 2) {
+        const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(s, s));
+        xh[i] = p.x;
+        xh[i + 1] = p.y;
     }
 }
 
@@ -305,31 +468,123 @@ __device__ __forceinline__ void decode_unit(const uint32_t* cw, const uint32_t* 
     }
 }
 
-// Sum of squared errors of one unit.  The fast path squares and sums in fp32;
-// a unit whose fp32 sum overflowed or may have lost terms to underflow (|x| near
-// the top of the bf16 range, or bf16 subnormals) is recomputed in fp64.
-__device__ __forceinline__ double unit_sse(const uint32_t* w, const float* xh)
+// Read a unit's codes and scale bytes (dense layouts).
+template <int FMT>
+__device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                            int64_t code_off, int64_t scale_off, bool full, bool a16, uint32_t* cw,
+                                            uint32_t* sb)
 {
-    float e = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const float d0 = bf16_lo(w[k]) - xh[2 * k];
-        const float d1 = bf16_hi(w[k]) - xh[2 * k + 1];
-        e = __fmaf_rn(d0, d0, e);
-        e = __fmaf_rn(d1, d1, e);
-    }
-    if (e < 0x1p-100f || !(e <= 3.0e38f)) {
-        double ed = 0.0;
-#pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
-            const double d0 = (double)bf16_lo(w[k]) - (double)xh[2 * k];
-            const double d1 = (double)bf16_hi(w[k]) - (double)xh[2 * k + 1];
-            ed = fma(d0, d0, ed);
-            ed = fma(d1, d1, ed);
+    const uint8_t* cp = codes + code_off;
+    if (full && a16) {
+        const uint4 c = ldg_nc_v4(cp);
+        cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
+    } else {
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(cp));
+        cw[0] = c.x; cw[1] = c.y;
+        if (full) {
+            const uint2 d = __ldg(reinterpret_cast<const uint2*>(cp + 8));
+            cw[2] = d.x; cw[3] = d.y;
+        } else {
+            cw[2] = 0; cw[3] = 0;
         }
-        return ed;
     }
-    return (double)e;
+    sb[0] = __ldg(scales + scale_off);
+    sb[1] = (FMT != kMX && full) ? (uint32_t)__ldg(scales + scale_off + 1) : 0u;
+}
+
+// ---------------------------------------------------------------------------
+// The tile pipeline
+// ---------------------------------------------------------------------------
+
+// Shared memory of a pipelined CTA: kStages tiles (1024-byte aligned for the
+// 128-byte swizzle) followed by one mbarrier per stage.
+constexpr int kPipeSmemBytes = kStages * kTileBytes + 1024 + 64;
+
+struct Pipe {
+    uint32_t tiles;   // shared address of stage 0
+    uint32_t bars;    // shared address of the stage barriers
+};
+
+__device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
+{
+    const uint32_t base = smem_u32(smem_raw);
+    Pipe p;
+    p.tiles = (base + 1023u) & ~1023u;
+    p.bars = p.tiles + kStages * kTileBytes;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) mbar_init(p.bars + 8 * s, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    return p;
+}
+
+// Tiles of this CTA: blockIdx.x + j * gridDim.x, walked backwards when reverse.
+struct Schedule {
+    int64_t count, mine;
+    bool reverse;
+    __device__ int64_t tile(int64_t j) const
+    {
+        const int64_t i = (int64_t)blockIdx.x + j * gridDim.x;
+        return reverse ? count - 1 - i : i;
+    }
+};
+
+__device__ __forceinline__ Schedule make_schedule(int64_t count, bool reverse)
+{
+    Schedule s;
+    s.count = count;
+    s.reverse = reverse;
+    s.mine = (int64_t)blockIdx.x < count ? (count - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+    return s;
+}
+
+template <bool FLAT>
+__device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
+                                           int64_t j)
+{
+    const int s = (int)(j % kStages);
+    int x, y;
+    tile_origin<FLAT>(tl, sc.tile(j), x, y);
+    mbar_arm(p.bars + 8 * s, kTileBytes);
+    tma_load_tile(p.tiles + s * kTileBytes, map, x, y, p.bars + 8 * s);
+}
+
+// Wait for tile j (bounded); the caller consumes the tile only when this
+// returned true and then calls pipe_release.
+__device__ __forceinline__ bool pipe_wait(const Pipe& p, int64_t j)
+{
+    return mbar_wait(p.bars + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+}
+
+// End of tile j: the CTA agrees on whether any thread's wait timed out.  If so,
+// thread 0 records it and waits (bounded) for the copies still in flight, and
+// the caller stops; otherwise thread 0 refills the slot with tile j + kStages.
+template <bool FLAT>
+__device__ __forceinline__ bool pipe_release(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
+                                             int64_t j, bool ok)
+{
+    if (!__syncthreads_or(!ok)) {
+        if (threadIdx.x == 0 && j + kStages < sc.mine) pipe_issue<FLAT>(p, map, tl, sc, j + kStages);
+        return true;
+    }
+    if (threadIdx.x == 0) {
+        atomicOr(&g_device_error, kErrPipelineTimeout);
+        const int64_t last = j + kStages < sc.mine ? j + kStages : sc.mine;
+        for (int64_t q = j; q < last; ++q) mbar_wait(p.bars + 8 * (int)(q % kStages), (uint32_t)((q / kStages) & 1));
+    }
+    __syncthreads();
+    return false;
+}
+
+__device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint32_t h, uint32_t* w)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint4 v = lds128(tile_chunk(tile, r, 4 * h + c));
+        w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -337,173 +592,305 @@ __device__ __forceinline__ double unit_sse(const uint32_t* w, const float* xh)
 // ---------------------------------------------------------------------------
 
 struct AmaxArgs {
-    const uint16_t* x;
-    Geometry g;
+    Tiles tl;
     float* partials;
 };
 
-template <bool ROT, bool CONTIG, bool PAIRED>
-__global__ void __launch_bounds__(kThreads) amax_kernel(AmaxArgs a)
+// Q0: per-CTA maxima of |x| (of |H x| when rotating).
+template <bool ROT, bool FLAT>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ CUtensorMap xmap, AmaxArgs a)
 {
-    __shared__ float sh[32];
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ float shf[32];
+    const Pipe p = pipe_setup(smem_raw);
+    const Schedule sc = make_schedule(a.tl.count, false);
+    const int t = threadIdx.x;
+    if (t == 0)
+        for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT>(p, &xmap, a.tl, sc, j);
+    pdl_trigger();
     float m = 0.0f;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.g.units; u += stride) {
-        const bool full = 2 * u + 1 < a.g.halves;
-        uint32_t w[16];
-        load_unit<CONTIG, PAIRED>(a.x, a.g, u, full, w);
-        float y[32];
-        unpack32(w, y);
-        if (ROT) wht32_inplace(y);
+    for (int64_t j = 0; j < sc.mine; ++j) {
+        const bool ok = pipe_wait(p, j);
+        if (ok) {
+            const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
+            uint32_t w[16];
+            load_unit_words(tile, (uint32_t)t >> 1, (uint32_t)t & 1u, w);
+            // out-of-range parts of a tile are zero-filled, so no validity test is needed
+            if (ROT) {
+                float y[32];
+                unpack16(w, y);
+                unpack16(w + 8, y + 16);
+                wht32_inplace(y);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(y[i]));
+                for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(y[i]));
+            } else {
+                uint32_t mm = w[0];
+#pragma unroll
+                for (int i = 1; i < 16; ++i) mm = bf16x2_absmax(mm, w[i]);
+                m = fmaxf(m, bf16x2_hmax_abs(mm));
+            }
+        }
+        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
     }
-    m = block_max(m, sh);
-    if (threadIdx.x == 0) a.partials[blockIdx.x] = m;
+    m = block_max(m, shf);
+    if (t == 0) a.partials[blockIdx.x] = m;
 }
 
 struct QuantArgs {
-    const uint16_t* x;
-    Geometry g;
+    Tiles tl;
     uint8_t* codes;
     uint8_t* scales;
     float* tensor_scale;
     const float* amax_partials;
     int n_amax;
     int scale_given;
+    int reverse;
     double* sse_partials;
 };
 
-template <int FMT, bool ROT, bool SSE, bool CONTIG>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(QuantArgs a)
+// Q1-Q6: rotate, block scale, encode, RaZeR select, pack, store, SSE partials.
+template <int FMT, bool ROT, bool SSE, bool FLAT>
+__global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a)
 {
-    constexpr bool PAIRED = (FMT == kMX) || ROT;
+    extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
     __shared__ double shd[32];
+    const Pipe p = pipe_setup(smem_raw);
+    const Schedule sc = make_schedule(a.tl.count, a.reverse != 0);
+    const int t = threadIdx.x;
+    // x was complete before the preceding kernel of this call started, so the
+    // first tiles may be fetched before waiting for that kernel.
+    if (t == 0)
+        for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT>(p, &xmap, a.tl, sc, j);
+    pdl_wait();
 
-    // Tensor scale (NVFP4 formats): s_t = RN(A / (6 * 448)), A reduced from
-    // the absmax pass's per-CTA maxima in every CTA.
+    // Tensor scale (NVFP4 formats): s_t = RN(A / (6 * 448)) from the absmax partials.
     float s_t = 0.0f;
     if (FMT != kMX) {
         if (a.scale_given) {
             s_t = *a.tensor_scale;
         } else {
             float m = 0.0f;
-            for (int i = threadIdx.x; i < a.n_amax; i += kThreads) m = fmaxf(m, a.amax_partials[i]);
+            for (int i = t; i < a.n_amax; i += kThreads) m = fmaxf(m, a.amax_partials[i]);
             m = block_max(m, shf);
             s_t = __fdiv_rn(m, 2688.0f);
-            if (blockIdx.x == 0 && threadIdx.x == 0) *a.tensor_scale = s_t;
+            if (blockIdx.x == 0 && t == 0) *a.tensor_scale = s_t;
         }
     }
-    const float six_st = __fmul_rn(6.0f, s_t);
+    pdl_trigger();
+    __shared__ float den_tab[128], rcp_tab[128];
+    const NvScale nsc = nv_scale_setup(s_t, den_tab, rcp_tab);
+    const bool a16 = FLAT || (a.tl.cols % 32) == 0;
+    const uint32_t r = (uint32_t)t >> 1, h = (uint32_t)t & 1u;
 
     double acc = 0.0;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.g.units; u += stride) {
-        const bool full = 2 * u + 1 < a.g.halves;
-        uint32_t w[16];
-        load_unit<CONTIG, PAIRED>(a.x, a.g, u, full, w);
-        float y[32];
-        unpack32(w, y);
-        if (ROT) wht32_inplace(y);
-
-        uint32_t cw[4], sb0, sb1 = 0;
-        float xh[32];
-        if (FMT == kMX) {
-            encode_mx32<SSE>(y, cw, sb0, xh);
-        } else {
-            encode_nv16<FMT == kRZ, SSE>(y, s_t, six_st, cw, sb0, xh);
-            encode_nv16<FMT == kRZ, SSE>(y + 16, s_t, six_st, cw + 2, sb1, xh + 16);
+    for (int64_t j = 0; j < sc.mine; ++j) {
+        const bool ok = pipe_wait(p, j);
+        const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
+        const Unit u = unit_of<FLAT>(a.tl, sc.tile(j), t);
+        uint32_t cw[4] = {0, 0, 0, 0}, sb0 = 0, sb1 = 0;
+        if (ok && u.valid) {
+            if (FMT != kMX && !ROT) {
+                // two independent 16-element blocks, one after the other
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (half == 1 && !u.full) break;
+                    uint32_t w[8];
+                    const uint4 v0 = lds128(tile_chunk(tile, r, 4 * h + 2 * half));
+                    const uint4 v1 = lds128(tile_chunk(tile, r, 4 * h + 2 * half + 1));
+                    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+                    const uint32_t mm = bf16x2_absmax(
+                        bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
+                        bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+                    float y[16];
+                    unpack16(w, y);
+                    uint32_t sbh;
+                    double e = 0.0;
+                    encode_nv16<FMT == kRZ, SSE ? kOutSse : kOutNone>(y, bf16x2_hmax_abs(mm), nsc, cw[2 * half],
+                                                                      cw[2 * half + 1], sbh, nullptr, &e);
+                    if (half == 0) sb0 = sbh;
+                    else sb1 = sbh;
+                    if (SSE) acc += e;
+                }
+            } else {
+                float y[32], xh[32];
+                {
+                    uint32_t w[16];
+                    load_unit_words(tile, r, h, w);
+                    unpack16(w, y);
+                    unpack16(w + 8, y + 16);
+                }
+                if (ROT) wht32_inplace(y);
+                if (FMT == kMX) {
+                    float am = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(y[i]));
+                    encode_mx32<SSE>(y, am, cw, sb0, xh);
+                } else {
+                    float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        a0 = fmaxf(a0, fabsf(y[i]));
+                        a1 = fmaxf(a1, fabsf(y[16 + i]));
+                    }
+                    encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y, a0, nsc, cw[0], cw[1], sb0, xh, nullptr);
+                    encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16,
+                                                                    nullptr);
+                }
+                if (SSE) {
+                    // the original values again, from the tile still in shared memory
+                    if (ROT) wht32_inplace(xh);
+                    uint32_t w[16];
+                    load_unit_words(tile, r, h, w);
+                    unpack16(w, y);
+                    unpack16(w + 8, y + 16);
+                    acc += sse_of<32>(y, xh);
+                }
+            }
+            int64_t co, so;
+            unit_offsets<FLAT, FMT>(a.tl, u, co, so);
+            store_codes(a.codes + co, cw, u.full, a16);
+            if (FMT == kMX) {
+                a.scales[so] = (uint8_t)sb0;
+            } else if (u.full && a16) {
+                *reinterpret_cast<unsigned short*>(a.scales + so) = (unsigned short)(sb0 | (sb1 << 8));
+            } else {
+                a.scales[so] = (uint8_t)sb0;
+                if (u.full) a.scales[so + 1] = (uint8_t)sb1;
+            }
         }
-        if (SSE) {
-            if (ROT) wht32_inplace(xh);
-            acc += unit_sse(w, xh);
-        }
-        uint8_t* cp = a.codes + 16 * u;
-        if (full) {
-            stg_v4(cp, make_uint4(cw[0], cw[1], cw[2], cw[3]));
-            if (FMT == kMX) a.scales[u] = (uint8_t)sb0;
-            else reinterpret_cast<unsigned short*>(a.scales)[u] = (unsigned short)(sb0 | (sb1 << 8));
-        } else {
-            stg_v2(cp, cw[0], cw[1]);
-            a.scales[2 * u] = (uint8_t)sb0;
-        }
+        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
     }
     if (SSE) {
         acc = block_sum(acc, shd);
-        if (threadIdx.x == 0) a.sse_partials[blockIdx.x] = acc;
-    }
-}
-
-struct DeqArgs {
-    const uint8_t* codes;
-    const uint8_t* scales;
-    const float* tensor_scale;
-    Geometry g;
-    uint16_t* y;
-};
-
-template <int FMT, bool ROT, bool CONTIG>
-__global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqArgs a)
-{
-    constexpr bool PAIRED = (FMT == kMX) || ROT;
-    const float s_t = (FMT != kMX) ? *a.tensor_scale : 0.0f;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.g.units; u += stride) {
-        const bool full = 2 * u + 1 < a.g.halves;
-        uint32_t cw[4], sb[2];
-        load_packed<FMT>(a.codes, a.scales, u, full, cw, sb);
-        float xh[32];
-        decode_unit<FMT>(cw, sb, s_t, xh);
-        if (ROT) wht32_inplace(xh);
-        uint32_t o[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = pack_bf16x2_rn(xh[2 * k], xh[2 * k + 1]);
-        uint16_t* p0 = a.y + half_offset<CONTIG>(a.g, 2 * u);
-        stg_v4(p0, make_uint4(o[0], o[1], o[2], o[3]));
-        stg_v4(p0 + 8, make_uint4(o[4], o[5], o[6], o[7]));
-        if (full) {
-            uint16_t* p1 = (CONTIG || PAIRED) ? p0 + 16 : a.y + half_offset<CONTIG>(a.g, 2 * u + 1);
-            stg_v4(p1, make_uint4(o[8], o[9], o[10], o[11]));
-            stg_v4(p1 + 8, make_uint4(o[12], o[13], o[14], o[15]));
-        }
+        if (t == 0) a.sse_partials[blockIdx.x] = acc;
     }
 }
 
 struct ErrArgs {
-    const uint16_t* x;
+    Tiles tl;
     const uint8_t* codes;
     const uint8_t* scales;
     const float* tensor_scale;
-    Geometry g;
     double* sse_partials;
 };
 
-template <int FMT, bool ROT, bool CONTIG>
-__global__ void __launch_bounds__(kThreads) error_kernel(ErrArgs a)
+// Q8: squared error of a given encoding against x.
+template <int FMT, bool ROT, bool FLAT>
+__global__ void __launch_bounds__(kThreads, 3) error_kernel(const __grid_constant__ CUtensorMap xmap, ErrArgs a)
 {
-    constexpr bool PAIRED = (FMT == kMX) || ROT;
+    extern __shared__ uint8_t smem_raw[];
     __shared__ double shd[32];
+    const Pipe p = pipe_setup(smem_raw);
+    const Schedule sc = make_schedule(a.tl.count, false);
+    const int t = threadIdx.x;
+    if (t == 0)
+        for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT>(p, &xmap, a.tl, sc, j);
+    pdl_trigger();
     const float s_t = (FMT != kMX) ? *a.tensor_scale : 0.0f;
+    const bool a16 = FLAT || (a.tl.cols % 32) == 0;
+    const uint32_t r = (uint32_t)t >> 1, h = (uint32_t)t & 1u;
     double acc = 0.0;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.g.units; u += stride) {
-        const bool full = 2 * u + 1 < a.g.halves;
-        uint32_t w[16];
-        load_unit<CONTIG, PAIRED>(a.x, a.g, u, full, w);
-        uint32_t cw[4], sb[2];
-        load_packed<FMT>(a.codes, a.scales, u, full, cw, sb);
-        float xh[32];
-        decode_unit<FMT>(cw, sb, s_t, xh);
-        if (ROT) wht32_inplace(xh);
-        if (!full) {
-#pragma unroll
-            for (int i = 16; i < 32; ++i) xh[i] = 0.0f;
+    for (int64_t j = 0; j < sc.mine; ++j) {
+        const Unit u = unit_of<FLAT>(a.tl, sc.tile(j), t);
+        uint32_t cw[4] = {0, 0, 0, 0}, sb[2] = {0, 0};
+        if (u.valid) {
+            int64_t co, so;
+            unit_offsets<FLAT, FMT>(a.tl, u, co, so);
+            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
         }
-        acc += unit_sse(w, xh);
+        const bool ok = pipe_wait(p, j);
+        if (ok && u.valid) {
+            const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
+            uint32_t w[16];
+            load_unit_words(tile, r, h, w);
+            float xh[32], x[32];
+            decode_unit<FMT>(cw, sb, s_t, xh);
+            if (ROT) wht32_inplace(xh);
+            if (!u.full) {
+#pragma unroll
+                for (int i = 16; i < 32; ++i) xh[i] = 0.0f;
+            }
+            unpack16(w, x);
+            unpack16(w + 8, x + 16);
+            acc += sse_of<32>(x, xh);
+        }
+        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
     }
     acc = block_sum(acc, shd);
-    if (threadIdx.x == 0) a.sse_partials[blockIdx.x] = acc;
+    if (t == 0) a.sse_partials[blockIdx.x] = acc;
+}
+
+struct DeqArgs {
+    Tiles tl;
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* tensor_scale;
+};
+
+// Q7: reconstruct bf16 tiles in shared memory (the swizzled layout of the
+// loads) and write them with TMA stores; two output buffers alternate, and
+// the next unit's codes are fetched while the current one is written.
+template <int FMT, bool ROT, bool FLAT>
+__global__ void __launch_bounds__(kThreads) dequantize_kernel(const __grid_constant__ CUtensorMap ymap, DeqArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const Schedule sc = make_schedule(a.tl.count, false);
+    const int t = threadIdx.x;
+    pdl_trigger();
+    const float s_t = (FMT != kMX) ? *a.tensor_scale : 0.0f;
+    const bool a16 = FLAT || (a.tl.cols % 32) == 0;
+    const uint32_t r = (uint32_t)t >> 1, h = (uint32_t)t & 1u;
+
+    uint32_t cw[4] = {0, 0, 0, 0}, sb[2] = {0, 0};
+    Unit u{};
+    if (sc.mine > 0) {
+        u = unit_of<FLAT>(a.tl, sc.tile(0), t);
+        if (u.valid) {
+            int64_t co, so;
+            unit_offsets<FLAT, FMT>(a.tl, u, co, so);
+            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
+        }
+    }
+    for (int64_t j = 0; j < sc.mine; ++j) {
+        const int64_t k = sc.tile(j);
+        const Unit cur = u;
+        const uint32_t ccw[4] = {cw[0], cw[1], cw[2], cw[3]}, csb[2] = {sb[0], sb[1]};
+        if (j + 1 < sc.mine) {
+            u = unit_of<FLAT>(a.tl, sc.tile(j + 1), t);
+            if (u.valid) {
+                int64_t co, so;
+                unit_offsets<FLAT, FMT>(a.tl, u, co, so);
+                load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
+            }
+        }
+        uint32_t o[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+        if (cur.valid) {
+            float xh[32];
+            decode_unit<FMT>(ccw, csb, s_t, xh);
+            if (ROT) wht32_inplace(xh);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2_rn(xh[2 * i], xh[2 * i + 1]);
+        }
+        const uint32_t buf = base + (uint32_t)(j & 1) * kTileBytes;
+        // the TMA store issued from this buffer two tiles ago must have read it
+        if (t == 0) bulk_wait_reads_but_last();
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            sts128(tile_chunk(buf, r, 4 * h + c), make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+        fence_async_smem();
+        __syncthreads();
+        if (t == 0) {
+            int x, y;
+            tile_origin<FLAT>(a.tl, k, x, y);
+            tma_store_tile(&ymap, x, y, buf);
+            bulk_commit();
+        }
+    }
+    if (t == 0) bulk_wait_all();
 }
 
 // Sum n fp64 partials in a fixed order and write sum / count.
@@ -511,6 +898,7 @@ __global__ void __launch_bounds__(kThreads) sse_finalize_kernel(const double* pa
                                                                 double* mse)
 {
     __shared__ double sh[kThreads];
+    pdl_wait();
     double s = 0.0;
     for (int i = threadIdx.x; i < n; i += kThreads) s += partials[i];
     sh[threadIdx.x] = s;
@@ -523,7 +911,7 @@ __global__ void __launch_bounds__(kThreads) sse_finalize_kernel(const double* pa
 }
 
 // ---------------------------------------------------------------------------
-// Launch helpers
+// Host side: tensor maps, grids, launches
 // ---------------------------------------------------------------------------
 
 namespace {
@@ -531,6 +919,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_sm_count[kMaxDevices];
+std::map<std::pair<const void*, int>, int> g_occupancy;
 
 int sm_count()
 {
@@ -545,11 +934,10 @@ int sm_count()
     return g_sm_count[dev];
 }
 
-// Resident CTAs per SM for a kernel, cached per (kernel, device).
-std::map<std::pair<const void*, int>, int> g_occupancy;
-
+// Resident CTAs per SM for a kernel with `smem` bytes of dynamic shared memory,
+// cached per (kernel, device); sets the shared-memory attribute on first use.
 template <typename K>
-int ctas_per_sm(K kernel)
+int ctas_per_sm(K kernel, int smem)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -557,20 +945,90 @@ int ctas_per_sm(K kernel)
     std::lock_guard<std::mutex> lk(g_mu);
     auto it = g_occupancy.find(key);
     if (it != g_occupancy.end()) return it->second;
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, 0) != cudaSuccess || n <= 0) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess || n <= 0) n = 1;
     g_occupancy[key] = n;
     return n;
 }
 
 template <typename K>
-int grid_for(K kernel, int64_t units)
+int grid_for(K kernel, int smem, int64_t tiles)
 {
-    const int64_t need = (units + kThreads - 1) / kThreads;
-    int64_t cap = (int64_t)sm_count() * ctas_per_sm(kernel);
+    int64_t cap = (int64_t)sm_count() * ctas_per_sm(kernel, smem);
     if (cap > kMaxPartials) cap = kMaxPartials;
-    int64_t g = need < cap ? need : cap;
+    const int64_t g = tiles < cap ? tiles : cap;
     return g < 1 ? 1 : (int)g;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// The tile view of a bf16 matrix and its TMA map (box 64 x 128, 128-byte swizzle).
+bool make_view(const void* base, const Geometry& g, CUtensorMap* map, Tiles* tl)
+{
+    const int64_t n = g.rows * g.cols;
+    const bool flat = (g.ld == g.cols || g.rows == 1) && n % 64 == 0 && n / 64 < ((int64_t)1 << 31);
+    cuuint64_t dims[2];
+    cuuint64_t strides[1];
+    if (flat) {
+        dims[0] = 64;
+        dims[1] = (cuuint64_t)(n / 64);
+        strides[0] = 128;
+        tl->count = (n / 64 + kTileRows - 1) / kTileRows;
+        tl->col_tiles = 0;
+    } else {
+        if (g.rows >= ((int64_t)1 << 31) || g.cols >= ((int64_t)1 << 31)) return false;
+        dims[0] = (cuuint64_t)g.cols;
+        dims[1] = (cuuint64_t)g.rows;
+        strides[0] = (cuuint64_t)(g.ld * 2);
+        tl->col_tiles = (g.cols + kTileCols - 1) / kTileCols;
+        tl->count = tl->col_tiles * ((g.rows + kTileRows - 1) / kTileRows);
+    }
+    tl->rows = g.rows;
+    tl->cols = g.cols;
+    tl->units = n / 32;
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint32_t box[2] = {kTileCols, kTileRows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool is_flat(const Tiles& tl) { return tl.col_tiles == 0; }
+
+// Launch with `smem` bytes of dynamic shared memory; with pdl the kernel may
+// start while the previous kernel on the stream drains (it waits with
+// griddepcontrol.wait before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), int grid, int smem, bool pdl, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -578,31 +1036,32 @@ int grid_for(K kernel, int64_t units)
 cudaError_t launch_amax(const uint16_t* x, const Geometry& g, int rotate, float* partials, int* grid_out,
                         cudaStream_t st)
 {
-    AmaxArgs a{x, g, partials};
-    const bool contig = g.ld == g.cols;
-    const bool paired = (g.cols % 32) == 0;
+    CUtensorMap map;
+    AmaxArgs a;
+    if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    a.partials = partials;
     auto go = [&](auto kernel) {
-        const int grid = grid_for(kernel, g.units);
+        const int grid = grid_for(kernel, kPipeSmemBytes, a.tl.count);
         if (grid_out) *grid_out = grid;
-        kernel<<<grid, kThreads, 0, st>>>(a);
-        return cudaGetLastError();
+        return launch(kernel, grid, kPipeSmemBytes, false, st, map, a);
     };
-    if (rotate) return contig ? go(amax_kernel<true, true, true>) : go(amax_kernel<true, false, true>);
-    if (contig) return go(amax_kernel<false, true, false>);
-    return paired ? go(amax_kernel<false, false, true>) : go(amax_kernel<false, false, false>);
+    const bool flat = is_flat(a.tl);
+    if (rotate) return flat ? go(amax_kernel<true, true>) : go(amax_kernel<true, false>);
+    return flat ? go(amax_kernel<false, true>) : go(amax_kernel<false, false>);
 }
 
 template <int FMT, bool ROT>
-static cudaError_t quantize_dispatch(const QuantArgs& a, bool sse, bool contig, int* grid_out, cudaStream_t st)
+static cudaError_t quantize_dispatch(const CUtensorMap& map, const QuantArgs& a, bool sse, bool pdl, int* grid_out,
+                                     cudaStream_t st)
 {
     auto go = [&](auto kernel) {
-        const int grid = grid_for(kernel, a.g.units);
+        const int grid = grid_for(kernel, kPipeSmemBytes, a.tl.count);
         if (grid_out) *grid_out = grid;
-        kernel<<<grid, kThreads, 0, st>>>(a);
-        return cudaGetLastError();
+        return launch(kernel, grid, kPipeSmemBytes, pdl, st, map, a);
     };
-    if (sse) return contig ? go(quantize_kernel<FMT, ROT, true, true>) : go(quantize_kernel<FMT, ROT, true, false>);
-    return contig ? go(quantize_kernel<FMT, ROT, false, true>) : go(quantize_kernel<FMT, ROT, false, false>);
+    const bool flat = is_flat(a.tl);
+    if (sse) return flat ? go(quantize_kernel<FMT, ROT, true, true>) : go(quantize_kernel<FMT, ROT, true, false>);
+    return flat ? go(quantize_kernel<FMT, ROT, false, true>) : go(quantize_kernel<FMT, ROT, false, false>);
 }
 
 cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int rotate, int want_sse,
@@ -610,79 +1069,110 @@ cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int r
                             const float* amax_partials, int n_amax, double* sse_partials, int* grid_out,
                             cudaStream_t st)
 {
-    QuantArgs a{x, g, codes, scales, tensor_scale, amax_partials, n_amax, scale_given, sse_partials};
-    const bool contig = g.ld == g.cols;
+    CUtensorMap map;
+    QuantArgs a;
+    if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    a.codes = codes;
+    a.scales = scales;
+    a.tensor_scale = tensor_scale;
+    a.amax_partials = amax_partials;
+    a.n_amax = n_amax;
+    a.scale_given = scale_given;
+    // after an absmax pass: start where that pass ended (its last tiles are in L2)
+    const bool after_amax = fmt != kMX && !scale_given;
+    a.reverse = after_amax ? 1 : 0;
+    a.sse_partials = sse_partials;
     const bool sse = want_sse != 0;
     switch (fmt * 2 + (rotate ? 1 : 0)) {
-        case 0: return quantize_dispatch<kNV, false>(a, sse, contig, grid_out, st);
-        case 1: return quantize_dispatch<kNV, true>(a, sse, contig, grid_out, st);
-        case 2: return quantize_dispatch<kRZ, false>(a, sse, contig, grid_out, st);
-        case 3: return quantize_dispatch<kRZ, true>(a, sse, contig, grid_out, st);
-        case 4: return quantize_dispatch<kMX, false>(a, sse, contig, grid_out, st);
-        case 5: return quantize_dispatch<kMX, true>(a, sse, contig, grid_out, st);
+        case 0: return quantize_dispatch<kNV, false>(map, a, sse, after_amax, grid_out, st);
+        case 1: return quantize_dispatch<kNV, true>(map, a, sse, after_amax, grid_out, st);
+        case 2: return quantize_dispatch<kRZ, false>(map, a, sse, after_amax, grid_out, st);
+        case 3: return quantize_dispatch<kRZ, true>(map, a, sse, after_amax, grid_out, st);
+        case 4: return quantize_dispatch<kMX, false>(map, a, sse, after_amax, grid_out, st);
+        case 5: return quantize_dispatch<kMX, true>(map, a, sse, after_amax, grid_out, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
+constexpr int kDeqSmemBytes = 2 * kTileBytes + 1024;
+
 template <int FMT, bool ROT>
-static cudaError_t dequantize_dispatch(const DeqArgs& a, bool contig, cudaStream_t st)
+static cudaError_t dequantize_dispatch(const CUtensorMap& map, const DeqArgs& a, cudaStream_t st)
 {
     auto go = [&](auto kernel) {
-        kernel<<<grid_for(kernel, a.g.units), kThreads, 0, st>>>(a);
-        return cudaGetLastError();
+        const int grid = grid_for(kernel, kDeqSmemBytes, a.tl.count);
+        return launch(kernel, grid, kDeqSmemBytes, false, st, map, a);
     };
-    return contig ? go(dequantize_kernel<FMT, ROT, true>) : go(dequantize_kernel<FMT, ROT, false>);
+    return is_flat(a.tl) ? go(dequantize_kernel<FMT, ROT, true>) : go(dequantize_kernel<FMT, ROT, false>);
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
                               const Geometry& g, int fmt, int rotate, uint16_t* y, cudaStream_t st)
 {
-    DeqArgs a{codes, scales, tensor_scale, g, y};
-    const bool contig = g.ld == g.cols;
+    CUtensorMap map;
+    DeqArgs a;
+    if (!make_view(y, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    a.codes = codes;
+    a.scales = scales;
+    a.tensor_scale = tensor_scale;
     switch (fmt * 2 + (rotate ? 1 : 0)) {
-        case 0: return dequantize_dispatch<kNV, false>(a, contig, st);
-        case 1: return dequantize_dispatch<kNV, true>(a, contig, st);
-        case 2: return dequantize_dispatch<kRZ, false>(a, contig, st);
-        case 3: return dequantize_dispatch<kRZ, true>(a, contig, st);
-        case 4: return dequantize_dispatch<kMX, false>(a, contig, st);
-        case 5: return dequantize_dispatch<kMX, true>(a, contig, st);
+        case 0: return dequantize_dispatch<kNV, false>(map, a, st);
+        case 1: return dequantize_dispatch<kNV, true>(map, a, st);
+        case 2: return dequantize_dispatch<kRZ, false>(map, a, st);
+        case 3: return dequantize_dispatch<kRZ, true>(map, a, st);
+        case 4: return dequantize_dispatch<kMX, false>(map, a, st);
+        case 5: return dequantize_dispatch<kMX, true>(map, a, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 template <int FMT, bool ROT>
-static cudaError_t error_dispatch(const ErrArgs& a, bool contig, int* grid_out, cudaStream_t st)
+static cudaError_t error_dispatch(const CUtensorMap& map, const ErrArgs& a, int* grid_out, cudaStream_t st)
 {
     auto go = [&](auto kernel) {
-        const int grid = grid_for(kernel, a.g.units);
+        const int grid = grid_for(kernel, kPipeSmemBytes, a.tl.count);
         if (grid_out) *grid_out = grid;
-        kernel<<<grid, kThreads, 0, st>>>(a);
-        return cudaGetLastError();
+        return launch(kernel, grid, kPipeSmemBytes, false, st, map, a);
     };
-    return contig ? go(error_kernel<FMT, ROT, true>) : go(error_kernel<FMT, ROT, false>);
+    return is_flat(a.tl) ? go(error_kernel<FMT, ROT, true>) : go(error_kernel<FMT, ROT, false>);
 }
 
 cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t* scales,
                          const float* tensor_scale, const Geometry& g, int fmt, int rotate,
                          double* sse_partials, int* grid_out, cudaStream_t st)
 {
-    ErrArgs a{x, codes, scales, tensor_scale, g, sse_partials};
-    const bool contig = g.ld == g.cols;
+    CUtensorMap map;
+    ErrArgs a;
+    if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    a.codes = codes;
+    a.scales = scales;
+    a.tensor_scale = tensor_scale;
+    a.sse_partials = sse_partials;
     switch (fmt * 2 + (rotate ? 1 : 0)) {
-        case 0: return error_dispatch<kNV, false>(a, contig, grid_out, st);
-        case 1: return error_dispatch<kNV, true>(a, contig, grid_out, st);
-        case 2: return error_dispatch<kRZ, false>(a, contig, grid_out, st);
-        case 3: return error_dispatch<kRZ, true>(a, contig, grid_out, st);
-        case 4: return error_dispatch<kMX, false>(a, contig, grid_out, st);
-        case 5: return error_dispatch<kMX, true>(a, contig, grid_out, st);
+        case 0: return error_dispatch<kNV, false>(map, a, grid_out, st);
+        case 1: return error_dispatch<kNV, true>(map, a, grid_out, st);
+        case 2: return error_dispatch<kRZ, false>(map, a, grid_out, st);
+        case 3: return error_dispatch<kRZ, true>(map, a, grid_out, st);
+        case 4: return error_dispatch<kMX, false>(map, a, grid_out, st);
+        case 5: return error_dispatch<kMX, true>(map, a, grid_out, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_sse_finalize(const double* partials, int n, double count, double* mse, cudaStream_t st)
 {
-    sse_finalize_kernel<<<1, kThreads, 0, st>>>(partials, n, count, mse);
-    return cudaGetLastError();
+    return launch(sse_finalize_kernel, 1, 0, true, st, partials, n, count, mse);
+}
+
+cudaError_t read_device_errors(unsigned int* bits, bool clear)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+    }
+    return e;
 }
 
 }  // namespace fp4q

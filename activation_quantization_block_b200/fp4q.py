@@ -29,7 +29,8 @@ STATUS_NAMES = {
 
 # Names the C header declares; the tests check that the library exports each one.
 ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
-               "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc")
+               "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc",
+               "fp4q_device_errors")
 
 
 class Fp4qError(RuntimeError):
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.fp4q_error.restype = i32
         L.fp4q_quantize_noalloc.argtypes = [vp, i64, i64, i64, i32, i32, u32, vp, vp, vp, vp, vp]
         L.fp4q_quantize_noalloc.restype = i32
+        L.fp4q_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        L.fp4q_device_errors.restype = i32
         _lib = L
     return _lib
 
@@ -127,6 +130,13 @@ def fp4q_quantize_noalloc(x, rows, cols, ldx, fmt, rotate, flags, codes, scales,
     """fp4q_quantize with the library's static scratch: for callers that cannot allocate."""
     return lib().fp4q_quantize_noalloc(_ptr(x), rows, cols, ldx, _fmt(fmt), int(rotate), flags, _ptr(codes),
                                        _ptr(scales), _ptr(tensor_scale), _ptr(mse), _stream(stream))
+
+
+def fp4q_device_errors(clear: bool = False) -> tuple[int, int]:
+    """(status, error bits) of the current device; synchronous."""
+    v = ctypes.c_uint32(0)
+    st = lib().fp4q_device_errors(ctypes.byref(v), int(clear))
+    return st, v.value
 
 
 # ---- torch-level wrappers -------------------------------------------------------

@@ -153,6 +153,19 @@ FP4Q_API fp4q_status_t fp4q_error(const void* x, int64_t ldx,
                          int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
                          double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
 
+/* Bits of the device error word (fp4q_device_errors). */
+#define FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT 0x1u
+
+/* Read the device error word of the current device into *bits.
+ * Every wait of a kernel in this library on its own copy pipeline gives up
+ * after 2 s.  A CTA that gives up sets FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT in a
+ * per-device word, waits (bounded) for its copies in flight and returns, so
+ * the outputs of that call are incomplete.  This call is synchronous: it waits
+ * for the device, copies the word to the host and, when clear != 0, resets it.
+ * Returns FP4Q_ERROR_INVALID_VALUE for a null bits, FP4Q_ERROR_CUDA if the copy
+ * fails. */
+FP4Q_API fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear);
+
 /* Bytes of device scratch held inside the library for fp4q_quantize_noalloc. */
 #define FP4Q_NOALLOC_SCRATCH_BYTES 49152
 
