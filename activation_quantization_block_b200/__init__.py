@@ -7,5 +7,5 @@ holds seeded input generators.
 from .fp4q import (  # noqa: F401
     ABI_SYMBOLS, FORMATS, MXFP4, NVFP4, NVFP4_RAZER, Fp4qError, Quantized, block_size, dequantize, error,
     fp4q_abi_version, fp4q_dequantize, fp4q_error, fp4q_quantize, fp4q_status_string, fp4q_workspace_size,
-    lib, library_path, quantize,
+    lib, library_path, quantize, quantize_batch, fp4q_quantize_batch, fp4q_batch_workspace_size,
 )

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "fp4q.h"
 #include "fp4q_internal.h"
@@ -201,12 +202,64 @@ fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
     if (bits == nullptr) return FP4Q_ERROR_INVALID_VALUE;
     fp4q_status_t s = check_device();
     if (s != FP4Q_SUCCESS) return s;
-    unsigned int v = 0;
-    if (read_device_errors(&v, clear != 0) != cudaSuccess) {
+    unsigned int v = 0, w = 0;
+    if (read_device_errors(&v, clear != 0) != cudaSuccess || read_batch_device_errors(&w, clear != 0) != cudaSuccess) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }
-    *bits = v;
+    *bits = v | w;
+    return FP4Q_SUCCESS;
+}
+
+size_t fp4q_batch_workspace_size(int count, const fp4q_tensor_desc_t* tensors, fp4q_format_t fmt, int rotate)
+{
+    (void)count; (void)tensors; (void)fmt; (void)rotate;
+    return batch_workspace_bytes();
+}
+
+fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* tensors, fp4q_format_t fmt, int rotate,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes, fp4q_stream_t stream)
+{
+    if (count < 0 || (count > 0 && tensors == nullptr)) return FP4Q_ERROR_INVALID_VALUE;
+    if (flags & ~FP4Q_FLAG_TENSOR_SCALE_GIVEN) return FP4Q_ERROR_INVALID_VALUE;
+    const bool nv = fmt != FP4Q_MXFP4;
+    const bool given = (flags & FP4Q_FLAG_TENSOR_SCALE_GIVEN) != 0;
+    fp4q_status_t s;
+    for (int k = 0; k < count; ++k) {
+        const fp4q_tensor_desc_t& t = tensors[k];
+        if ((s = check_shape(t.rows, t.cols, fmt, rotate)) != FP4Q_SUCCESS) return s;
+        if (nv && t.tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+        if (nv && !aligned(t.tensor_scale, 4)) return FP4Q_ERROR_MISALIGNED;
+        if (t.mse != nullptr && !aligned(t.mse, 8)) return FP4Q_ERROR_MISALIGNED;
+        if (t.rows * t.cols > 0) {
+            if ((s = check_matrix(t.x, t.cols, t.ldx)) != FP4Q_SUCCESS) return s;
+            if (t.codes == nullptr || t.scales == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+            if (!aligned(t.codes, 16) || !aligned(t.scales, 16)) return FP4Q_ERROR_MISALIGNED;
+        }
+    }
+    if (count == 0) return FP4Q_SUCCESS;
+    if (workspace == nullptr || !aligned(workspace, 16) ||
+        workspace_bytes < fp4q_batch_workspace_size(count, tensors, fmt, rotate))
+        return FP4Q_ERROR_WORKSPACE;
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<BatchTensor> work;
+    work.reserve((size_t)count);
+    for (int k = 0; k < count; ++k) {
+        const fp4q_tensor_desc_t& t = tensors[k];
+        if (t.rows * t.cols == 0) {   // empty: the scalar outputs are 0, as with fp4q_quantize
+            if (nv && !given && cudaMemsetAsync(t.tensor_scale, 0, sizeof(float), st) != cudaSuccess) return FP4Q_ERROR_CUDA;
+            if (t.mse && cudaMemsetAsync(t.mse, 0, sizeof(double), st) != cudaSuccess) return FP4Q_ERROR_CUDA;
+            continue;
+        }
+        work.push_back(BatchTensor{t.x, t.rows, t.cols, t.ldx, t.codes, t.scales, t.tensor_scale, t.mse});
+    }
+    if (!work.empty() &&
+        launch_quantize_batch(work.data(), (int)work.size(), fmt, rotate, given ? 1 : 0, workspace, st) != cudaSuccess) {
+        cudaGetLastError();
+        return FP4Q_ERROR_CUDA;
+    }
     return FP4Q_SUCCESS;
 }
 

@@ -1,0 +1,302 @@
+// Batch quantization: a chain of persistent kernels with programmatic
+// dependent launch, one kernel per tensor.
+//
+// With the tensor scale computed (NVFP4 formats), kernel j of a batch of n
+// tensors streams, interleaved in proportion to their tile counts:
+//   - the quantize tiles of tensor j-1 (its tensor scale comes from the
+//     absmax partials kernel j-1 wrote), and
+//   - the absmax tiles of tensor j (partials for kernel j+1),
+// and its CTA 0 turns the error partials of tensor j-2 into its MSE.  So the
+// memory-bound absmax pass of one tensor runs inside the same SMs as the
+// ALU-bound quantize pass of the previous one, every dependency crosses a
+// kernel boundary (griddepcontrol.wait), and no CTA ever waits on another.
+// Kernel 0 holds only absmax tiles, kernel n only quantize tiles, and kernel
+// n+1 only finalises.  With the scale given, or for MXFP4, kernel j quantizes
+// tensor j and finalises tensor j-1.
+//
+// Every kernel fetches its first tiles before waiting for its predecessor:
+// all inputs were complete when the first kernel of the batch started, and a
+// kernel lets its successor launch only after it has passed that wait, so a
+// kernel never starts before its predecessor's predecessor has finished.
+// Partial buffers rotate over three slots: kernel j reads slot j-1 and writes
+// slot j, so a kernel overlapping its predecessor's tail never writes a slot
+// that is still being read.  Tiles are assigned to CTAs round-robin (a fixed
+// schedule), so every partial sum is formed in a fixed order.
+//
+// Method references (title, section): as fp4q_common.cuh.
+#include <new>
+#include <vector>
+
+#include "fp4q_launch.cuh"
+
+namespace fp4q {
+
+constexpr int kRing = 3;   // rotating partial-buffer slots
+
+struct ChainArgs {
+    // quantize part
+    Tiles qtl;
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tensor_scale;
+    const float* amax_in;   // absmax partials of the quantized tensor (computed scale)
+    double* sse_out;        // this kernel's per-CTA error partials of the quantized tensor
+    int32_t n_amax_in;
+    int32_t has_q, q_flat, computed;
+    // absmax part
+    Tiles atl;
+    float* amax_out;        // this kernel's per-CTA absmax partials
+    int32_t has_a, a_flat;
+    // finaliser part
+    const double* sse_in;
+    double* fin_mse;
+    double fin_count;
+    int32_t n_sse_in;
+    int32_t has_fin;
+};
+
+template <int FMT, bool ROT, bool SSE>
+__global__ void __launch_bounds__(kThreads, 3)
+    chain_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap amap, ChainArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ float shf[32];
+    __shared__ double shd[kThreads];
+    __shared__ float den_tab[128], rcp_tab[128];
+    __shared__ int64_t slot_tile[kStages];   // item of each pipeline slot, decoded once by thread 0
+    __shared__ int32_t slot_q[kStages];
+    const Pipe p = pipe_setup(smem_raw);
+    const int t = threadIdx.x;
+
+    // Items of this kernel: nq quantize tiles (walked backwards) and na absmax
+    // tiles, interleaved in proportion; CTA b takes items b, b + G, b + 2G, ...
+    const int64_t nq = a.has_q ? a.qtl.count : 0;
+    const int64_t na = a.has_a ? a.atl.count : 0;
+    const int64_t tot = nq + na;
+    const int64_t G = gridDim.x, b = blockIdx.x;
+    const int64_t mine = b < tot ? (tot - 1 - b) / G + 1 : 0;
+    auto item = [&](int64_t jj, bool& is_q, int64_t& tile) {
+        const int64_t i = b + jj * G;
+        const int64_t qb = i * nq / tot;
+        is_q = (i + 1) * nq / tot > qb;
+        tile = is_q ? nq - 1 - qb : i - qb;
+    };
+    auto issue = [&](int64_t jj) {
+        bool is_q;
+        int64_t tile;
+        item(jj, is_q, tile);
+        const int s = (int)(jj % kStages);
+        slot_q[s] = is_q ? 1 : 0;
+        slot_tile[s] = tile;
+        int x, y;
+        if (is_q) {
+            if (a.q_flat) tile_origin<true>(a.qtl, tile, x, y);
+            else tile_origin<false>(a.qtl, tile, x, y);
+        } else {
+            if (a.a_flat) tile_origin<true>(a.atl, tile, x, y);
+            else tile_origin<false>(a.atl, tile, x, y);
+        }
+        mbar_arm(p.bars + 8 * s, kTileBytes);
+        tma_load_tile(p.tiles + s * kTileBytes, is_q ? &qmap : &amap, x, y, p.bars + 8 * s);
+    };
+    if (t == 0)
+        for (int64_t jj = 0; jj < mine && jj < kStages; ++jj) issue(jj);
+    pdl_wait();
+
+    // Tensor scale of the quantized tensor, from its absmax partials.
+    float s_t = 0.0f;
+    if (a.has_q && FMT != kMX) {
+        if (a.computed) {
+            float mx = 0.0f;
+            for (int i = t; i < a.n_amax_in; i += kThreads) mx = fmaxf(mx, a.amax_in[i]);
+            mx = block_max(mx, shf);
+            s_t = __fdiv_rn(mx, 2688.0f);
+            if (b == 0 && t == 0) *a.tensor_scale = s_t;
+        } else {
+            s_t = *a.tensor_scale;
+        }
+    }
+    // Finaliser: fixed-order sum of the previous kernel's error partials.
+    if (a.has_fin && b == 0) {
+        double s = 0.0;
+        for (int i = t; i < a.n_sse_in; i += kThreads) s += a.sse_in[i];
+        shd[t] = s;
+        __syncthreads();
+        for (int o = kThreads / 2; o > 0; o >>= 1) {
+            if (t < o) shd[t] += shd[t + o];
+            __syncthreads();
+        }
+        if (t == 0) *a.fin_mse = a.fin_count > 0.0 ? shd[0] / a.fin_count : 0.0;
+    }
+    pdl_trigger();
+    NvScale nsc;
+    nsc.den = den_tab;
+    nsc.rcp = rcp_tab;
+    if (a.has_q && FMT != kMX) nsc = nv_scale_setup(s_t, den_tab, rcp_tab);
+    __syncthreads();   // the slot items written by thread 0 are visible from here on
+
+    double acc = 0.0;
+    float m = 0.0f;
+    for (int64_t jj = 0; jj < mine; ++jj) {
+        const int s = (int)(jj % kStages);
+        const bool ok = mbar_wait(p.bars + 8 * s, (uint32_t)((jj / kStages) & 1));
+        const bool is_q = slot_q[s] != 0;
+        const int64_t tile = slot_tile[s];
+        const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
+        if (ok) {
+            if (is_q) {
+                if (a.q_flat) acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc);
+                else acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc);
+            } else {
+                m = fmaxf(m, amax_tile<ROT>(tp));
+            }
+        }
+        // end of the tile: agree on timeouts, then refill the slot
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) {
+                atomicOr(&g_device_error, kErrPipelineTimeout);
+                const int64_t last = jj + kStages < mine ? jj + kStages : mine;
+                for (int64_t q = jj + 1; q < last; ++q)
+                    mbar_wait(p.bars + 8 * (int)(q % kStages), (uint32_t)((q / kStages) & 1));
+            }
+            __syncthreads();
+            break;
+        }
+        if (t == 0 && jj + kStages < mine) issue(jj + kStages);
+    }
+    if (a.has_a) {
+        m = block_max(m, shf);
+        if (t == 0) a.amax_out[b] = m;
+    }
+    if (a.has_q && SSE) {
+        acc = block_sum(acc, shd);
+        if (t == 0) a.sse_out[b] = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+template <int FMT, bool ROT, bool SSE>
+cudaError_t chain_go(const CUtensorMap& qmap, const CUtensorMap& amap, const ChainArgs& a, int64_t tiles, bool pdl,
+                     int* grid_out, cudaStream_t st)
+{
+    auto kernel = chain_kernel<FMT, ROT, SSE>;
+    const int grid = grid_for(kernel, kPipeSmemBytes, tiles);
+    *grid_out = grid;
+    return launch(kernel, grid, kPipeSmemBytes, pdl, st, qmap, amap, a);
+}
+
+cudaError_t chain_dispatch(int fmt, bool rotate, bool sse, const CUtensorMap& qmap, const CUtensorMap& amap,
+                           const ChainArgs& a, int64_t tiles, bool pdl, int* grid_out, cudaStream_t st)
+{
+    switch (fmt * 4 + (rotate ? 2 : 0) + (sse ? 1 : 0)) {
+        case 0: return chain_go<kNV, false, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 1: return chain_go<kNV, false, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 2: return chain_go<kNV, true, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 3: return chain_go<kNV, true, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 4: return chain_go<kRZ, false, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 5: return chain_go<kRZ, false, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 6: return chain_go<kRZ, true, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 7: return chain_go<kRZ, true, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 8: return chain_go<kMX, false, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 9: return chain_go<kMX, false, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 10: return chain_go<kMX, true, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 11: return chain_go<kMX, true, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+struct View {
+    CUtensorMap map;
+    Tiles tl;
+};
+
+}  // namespace
+
+size_t batch_workspace_bytes() { return (size_t)kRing * kMaxPartials * (sizeof(float) + sizeof(double)); }
+
+cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, void* workspace,
+                                  cudaStream_t st)
+{
+    if (n <= 0) return cudaSuccess;
+    const bool computed = fmt != kMX && !scale_given;
+    bool sse = false;
+    for (int k = 0; k < n; ++k) sse = sse || ts[k].mse != nullptr;
+    char* ws = static_cast<char*>(workspace);
+    auto amax_slot = [&](int64_t j) { return reinterpret_cast<float*>(ws + (j % kRing) * kMaxPartials * 4); };
+    auto sse_slot = [&](int64_t j) {
+        return reinterpret_cast<double*>(ws + (size_t)kRing * kMaxPartials * 4 + (j % kRing) * kMaxPartials * 8);
+    };
+    std::vector<View> views((size_t)n);
+    for (int k = 0; k < n; ++k) {
+        const Geometry g = make_geometry(ts[k].rows, ts[k].cols, ts[k].ldx);
+        if (!make_view(ts[k].x, g, &views[(size_t)k].map, &views[(size_t)k].tl)) return cudaErrorInvalidValue;
+    }
+    const int lag = computed ? 1 : 0;            // kernel j quantizes tensor j - lag
+    std::vector<int> grids((size_t)n + 2, 0);    // CTAs (= partials written) of kernel j
+    for (int64_t j = 0; j < n + lag + 1; ++j) {
+        ChainArgs a = {};
+        const int64_t kq = j - lag;              // tensor quantized by kernel j
+        const int64_t ka = computed ? j : -1;    // tensor whose absmax pass kernel j runs
+        const int64_t kf = j - lag - 1;          // tensor whose MSE kernel j finalises
+        a.has_q = kq >= 0 && kq < n;
+        a.has_a = ka >= 0 && ka < n;
+        a.has_fin = kf >= 0 && kf < n && ts[kf].mse != nullptr;
+        if (!a.has_q && !a.has_a && !a.has_fin) continue;
+        const CUtensorMap* qmap = &views[0].map;
+        const CUtensorMap* amap = &views[0].map;
+        int64_t tiles = 0;
+        if (a.has_q) {
+            const View& v = views[(size_t)kq];
+            qmap = &v.map;
+            a.qtl = v.tl;
+            a.q_flat = is_flat(v.tl) ? 1 : 0;
+            a.codes = ts[kq].codes;
+            a.scales = ts[kq].scales;
+            a.tensor_scale = ts[kq].tensor_scale;
+            a.computed = computed ? 1 : 0;
+            if (computed) {
+                a.amax_in = amax_slot(kq);
+                a.n_amax_in = grids[(size_t)kq];
+            }
+            a.sse_out = sse_slot(j);
+            tiles += v.tl.count;
+        }
+        if (a.has_a) {
+            const View& v = views[(size_t)ka];
+            amap = &v.map;
+            a.atl = v.tl;
+            a.a_flat = is_flat(v.tl) ? 1 : 0;
+            a.amax_out = amax_slot(j);
+            tiles += v.tl.count;
+        }
+        if (a.has_fin) {
+            a.sse_in = sse_slot(j - 1);
+            a.n_sse_in = grids[(size_t)(j - 1)];
+            a.fin_count = (double)(ts[kf].rows * ts[kf].cols);
+            a.fin_mse = ts[kf].mse;
+        }
+        int grid = 0;
+        const cudaError_t e = chain_dispatch(fmt, rotate != 0, sse, *qmap, *amap, a, tiles, j > 0, &grid, st);
+        if (e != cudaSuccess) return e;
+        grids[(size_t)j] = grid;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t read_batch_device_errors(unsigned int* bits, bool clear)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace fp4q

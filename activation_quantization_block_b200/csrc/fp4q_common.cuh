@@ -1,0 +1,690 @@
+// Device code shared by the single-tensor kernels (fp4q_kernels.cu) and the
+// batch scheduler (fp4q_batch.cu): tile and unit geometry, block encoders and
+// decoders, error sums, CTA reductions and the TMA tile pipeline.
+//
+// Method references (title, section):
+//  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant Zero
+//   Remapping": sect. 1 (E2M1 set, E4M3 block scale from the block absmax,
+//   unused scale sign bit), sect. 2.2 (-0 code remapped to a special value
+//   chosen per block by minimum squared error; one bit -> the pair +-5).
+//  "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization": sect. 1
+//   (32-element blocks, shared exponent, e2m1 codebook), sect. 2 (orthogonal
+//   intra-block rotation before quantization).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp4q_device.cuh"
+#include "fp4q_internal.h"
+#include "fp4q_tma.cuh"
+
+namespace fp4q {
+
+enum { kNV = 0, kRZ = 1, kMX = 2 };
+
+// Device error word of a translation unit (bits: kErrPipelineTimeout); each
+// unit that launches kernels reads and clears its own copy for the C ABI.
+static __device__ unsigned int g_device_error;
+
+// ---------------------------------------------------------------------------
+// Tiles and units
+// ---------------------------------------------------------------------------
+
+struct Tiles {
+    int64_t count;       // number of tiles
+    int64_t col_tiles;   // 2-D view: tiles across the columns (ceil(cols / 64))
+    int64_t rows, cols;  // matrix shape
+    int64_t units;       // flat view: N / 32
+};
+
+template <bool FLAT>
+__device__ __forceinline__ void tile_origin(const Tiles& tl, int64_t k, int& x, int& y)
+{
+    if (FLAT) {
+        x = 0;
+        y = (int)(k * kTileRows);
+    } else {
+        const int64_t rt = k / tl.col_tiles;
+        x = (int)((k - rt * tl.col_tiles) * kTileCols);
+        y = (int)(rt * kTileRows);
+    }
+}
+
+// The unit thread t owns in tile k: its row and column, whether it exists,
+// whether both 16-element halves exist, and its unit index in the flat view.
+struct Unit {
+    int64_t row, col, flat;
+    bool valid, full;
+};
+
+template <bool FLAT>
+__device__ __forceinline__ Unit unit_of(const Tiles& tl, int64_t k, int t)
+{
+    Unit u;
+    if (FLAT) {
+        u.flat = k * (2 * kTileRows) + t;
+        u.valid = u.flat < tl.units;
+        u.full = true;
+        u.row = u.col = 0;
+    } else {
+        const int64_t rt = k / tl.col_tiles;
+        const int64_t ct = k - rt * tl.col_tiles;
+        u.row = rt * kTileRows + (t >> 1);
+        u.col = ct * kTileCols + 32 * (t & 1);
+        u.valid = u.row < tl.rows && u.col < tl.cols;
+        u.full = u.col + 32 <= tl.cols;
+        u.flat = 0;
+    }
+    return u;
+}
+
+// Offsets of a unit's codes and scale bytes in the dense layouts.
+template <bool FLAT, int FMT>
+__device__ __forceinline__ void unit_offsets(const Tiles& tl, const Unit& u, int64_t& code_off, int64_t& scale_off)
+{
+    constexpr int B = FMT == kMX ? 32 : 16;
+    if (FLAT) {
+        code_off = 16 * u.flat;
+        scale_off = (32 / B) * u.flat;
+    } else {
+        code_off = u.row * (tl.cols / 2) + u.col / 2;
+        scale_off = u.row * (tl.cols / B) + u.col / B;
+    }
+}
+
+// Store 16 (full) or 8 bytes of codes; a16 tells whether the address is 16-byte aligned.
+__device__ __forceinline__ void store_codes(uint8_t* p, const uint32_t* cw, bool full, bool a16)
+{
+    if (full && a16) {
+        stg_v4(p, make_uint4(cw[0], cw[1], cw[2], cw[3]));
+    } else {
+        stg_v2(p, cw[0], cw[1]);
+        if (full) stg_v2(p + 8, cw[2], cw[3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Block reductions (fixed order within a CTA)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float block_max(float v, float* sh)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    v = (threadIdx.x < (blockDim.x >> 5)) ? sh[threadIdx.x] : 0.0f;
+    if (warp == 0) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if (lane == 0) sh[0] = v;
+    }
+    __syncthreads();
+    return sh[0];
+}
+
+__device__ __forceinline__ double block_sum(double v, double* sh)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    v = (threadIdx.x < (blockDim.x >> 5)) ? sh[threadIdx.x] : 0.0;
+    if (warp == 0) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    }
+    return v;  // valid in thread 0
+}
+
+// ---------------------------------------------------------------------------
+// Squared error
+// ---------------------------------------------------------------------------
+
+// Sum of squares of 16 differences, exact in fp64 range: the values are
+// scaled by 2^-k, 2^k the power of two at or below their largest magnitude
+// (in two exact steps, so 2^-k never overflows), squared and summed in fp32,
+// and the sum is scaled back by 2^2k in fp64.  Used when a fast fp32 sum
+// overflowed or may have lost terms to underflow (|x| near the top of the bf16
+// range, or bf16 subnormals).
+__device__ __forceinline__ double sse16_rescaled(const float* d)
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(d[i]));
+    if (m == 0.0f || !(m <= 3.4e38f)) return m == 0.0f ? 0.0 : (double)INFINITY;
+    const int k = floor_log2_f32(m);              // in [-149, 127]
+    const int k1 = -k / 2, k2 = -k - k1;           // each in [-64, 75]
+    const float s1 = __uint_as_float((uint32_t)(k1 + 127) << 23);
+    const float s2 = __uint_as_float((uint32_t)(k2 + 127) << 23);
+    float es = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float t = __fmul_rn(__fmul_rn(d[i], s1), s2);
+        es = __fmaf_rn(t, t, es);
+    }
+    return (double)es * __longlong_as_double((long long)(2 * k + 1023) << 52);
+}
+
+// Sum of squared errors of 16 values (x - xh), the differences in fp32.
+__device__ __forceinline__ double sse16(const float* x, const float* xh)
+{
+    float2 acc = make_float2(0.0f, 0.0f);
+    float d[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 e = sub2_rn(make_float2(x[i], x[i + 1]), make_float2(xh[i], xh[i + 1]));
+        d[i] = e.x;
+        d[i + 1] = e.y;
+        acc = fma2_rn(e, e, acc);
+    }
+    const float es = acc.x + acc.y;
+    if (es >= 0x1p-100f && es <= 3.0e38f) return (double)es;
+    return sse16_rescaled(d);
+}
+
+template <int N>
+__device__ __forceinline__ double sse_of(const float* x, const float* xh)
+{
+    double e = sse16(x, xh);
+    if (N == 32) e += sse16(x + 16, xh + 16);
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// Encoders
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void unpack16(const uint32_t* w, float* y)
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float2 p = bf16x2_to_f32(w[k]);
+        y[2 * k] = p.x;
+        y[2 * k + 1] = p.y;
+    }
+}
+
+// Decode 16 codes (two words) to their E2M1 values.
+__device__ __forceinline__ void decode16(uint32_t w0, uint32_t w1, float* q)
+{
+    e2m1x8_to_f32(w0, q);
+    e2m1x8_to_f32(w1, q + 8);
+}
+
+// Per-tensor constants of the NVFP4 block-scale step, shared by a CTA: for
+// each of the 127 non-negative finite E4M3 bytes b, den[b] = RN(dec(b) * s_t)
+// and rcp[b] = RN(1 / den[b]) (0 when den[b] = 0: a zero scale zeroes every
+// code).  The quotient t = RN(a / RN(6 s_t)) uses inv6 = RN(1 / RN(6 s_t)) and
+// one correction step (Markstein's theorem: with y = RN(1/b) and a faithful
+// q = RN(a y), the residual r = a - q b is exact and RN(q + r y) = RN(a / b));
+// `exact_div` selects IEEE division when RN(6 s_t) is outside [2^-64, 2^64],
+// where the theorem's no-underflow conditions are not guaranteed.
+struct NvScale {
+    float s_t, six_st, inv6;
+    bool exact_div;
+    const float* den;
+    const float* rcp;
+};
+
+__device__ __forceinline__ NvScale nv_scale_setup(float s_t, float* den_tab, float* rcp_tab)
+{
+    NvScale c;
+    c.s_t = s_t;
+    c.six_st = __fmul_rn(6.0f, s_t);
+    c.exact_div = !(c.six_st >= 0x1p-64f && c.six_st <= 0x1p64f);
+    c.inv6 = c.exact_div ? 0.0f : __frcp_rn(c.six_st);
+    for (int b = threadIdx.x; b < 128; b += blockDim.x) {
+        const float d = b < 127 ? __fmul_rn(e4m3_to_f32((uint32_t)b), s_t) : 0.0f;
+        den_tab[b] = d;
+        rcp_tab[b] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+    }
+    __syncthreads();
+    c.den = den_tab;
+    c.rcp = rcp_tab;
+    return c;
+}
+
+// t = RN(a / RN(6 s_t)) for a >= 0.
+__device__ __forceinline__ float nv_block_ratio(const NvScale& c, float a)
+{
+    if (c.exact_div) return c.six_st > 0.0f ? __fdiv_rn(a, c.six_st) : 0.0f;
+    const float q = __fmul_rn(a, c.inv6);
+    const float r = __fmaf_rn(-q, c.six_st, a);
+    return __fmaf_rn(r, c.inv6, q);
+}
+
+// Outputs of the block encoders besides codes and scale.
+enum { kOutNone = 0, kOutSse = 1, kOutXh = 2 };
+
+// One 16-element NVFP4 block.  y: values (rotated when rotating); a: their
+// absmax.  Writes two code words and the scale byte.  OUT = kOutXh: xh receives
+// the fp32 reconstruction RN(q * den).  OUT = kOutSse: *sse receives
+// sum (y - q den)^2, each difference taken with a single rounding
+// (RN(y - q den), within half an fp32 ulp of y - RN(q den)).
+template <bool RAZER, int OUT>
+__device__ __forceinline__ void encode_nv16(const float* y, float a, const NvScale& sc, uint32_t& c0, uint32_t& c1,
+                                            uint32_t& sb_out, float* xh, double* sse)
+{
+    uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
+    const float den = sc.den[sb];
+    const float r = sc.rcp[sb];
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+        v[i] = p.x;
+        v[i + 1] = p.y;
+    }
+    uint32_t w0 = canonical_zero(e2m1x8(v));
+    uint32_t w1 = canonical_zero(e2m1x8(v + 8));
+
+    float win[16];
+    float special = 0.0f;
+    if (RAZER) {
+        // Gain of remapping element i to sign(v_i) * 5.  For |v_i| in (4.5, 5.5)
+        // the regular value is 4 (|v| <= 5) or 6 and
+        //   (|v| - q)^2 - (|v| - 5)^2 = 1 - 2 | |v| - 5 |,
+        // which is positive exactly on that open interval; elsewhere it is
+        // clamped to 0.  Each term is a multiple of 2^-20 in [0, 1], so the fp32
+        // sum S = gain(+5) - gain(-5) is exact in any order.
+        float cs[16];
+        float S = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float c = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
+            cs[i] = copysignf(c, v[i]);
+            S += cs[i];
+        }
+        // -5 only when its gain is strictly larger.  Winners are the candidates
+        // of the chosen sign: cs * sign >= 2^-20, so win = sat(cs * sign * 2^40)
+        // is exactly 1 for a winner and 0 otherwise (+0 or -0).
+        const float sk = S < 0.0f ? -0x1p40f : 0x1p40f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) win[i] = __saturatef(__fmul_rn(cs[i], sk));
+        // E2M1 of 1.0 is 0b0010 and of +-0 is 0b0000 / 0b1000: bit 1 of each
+        // nibble flags a winner; winners' codes become 0b1000.
+        const uint32_t f0 = (e2m1x8(win) >> 1) & 0x11111111u;
+        const uint32_t f1 = (e2m1x8(win + 8) >> 1) & 0x11111111u;
+        w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
+        w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
+        if (S < 0.0f) sb |= 0x80u;
+        special = S < 0.0f ? -5.0f : 5.0f;
+    }
+
+    if (OUT != kOutNone) {
+        // codes as written (RaZeR winners decode to -0 here and are fixed below)
+        float q[16];
+        decode16(w0, w1, q);
+        if (OUT == kOutSse) {
+            const float nden = -den;
+            const float nx5 = -__fmul_rn(special, den);   // -RN(special * den)
+            float2 acc = make_float2(0.0f, 0.0f);
+            float d[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float2 e = fma2_rn(make_float2(q[i], q[i + 1]), make_float2(nden, nden),
+                                   make_float2(y[i], y[i + 1]));
+                if (RAZER) e = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(nx5, nx5), e);
+                d[i] = e.x;
+                d[i + 1] = e.y;
+                acc = fma2_rn(e, e, acc);
+            }
+            const float es = acc.x + acc.y;
+            *sse = (es >= 0x1p-100f && es <= 3.0e38f) ? (double)es : sse16_rescaled(d);
+        } else {
+            if (RAZER) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    // winners: -0 + 1 * special; others: q + 0 * special
+                    const float2 n = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(special, special),
+                                             make_float2(q[i], q[i + 1]));
+                    q[i] = n.x;
+                    q[i + 1] = n.y;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(den, den));
+                xh[i] = p.x;
+                xh[i + 1] = p.y;
+            }
+        }
+    }
+    c0 = w0;
+    c1 = w1;
+    sb_out = sb;
+}
+
+// One 32-element MXFP4 block.
+template <bool XH>
+__device__ __forceinline__ void encode_mx32(const float* y, float a, uint32_t* cw, uint32_t& sb_out, float* xh)
+{
+    int e = -127;
+    float r = 0.0f;
+    uint32_t sb = 0;
+    if (a > 0.0f) {
+        e = floor_log2_f32(a) - 2;          // 2 = exponent of the largest E2M1 value
+        e = e < -127 ? -127 : (e > 127 ? 127 : e);
+        sb = (uint32_t)(e + 127);
+        r = exp2i(-e);
+    }
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+        v[i] = p.x;
+        v[i + 1] = p.y;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cw[k] = canonical_zero(e2m1x8(v + 8 * k));
+    if (XH) {
+        const float s = exp2i(e);
+        float q[32];
+        decode16(cw[0], cw[1], q);
+        decode16(cw[2], cw[3], q + 16);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(s, s));
+            xh[i] = p.x;
+            xh[i + 1] = p.y;
+        }
+    }
+    sb_out = sb;
+}
+
+// ---------------------------------------------------------------------------
+// Decoders (dequantize and error)
+// ---------------------------------------------------------------------------
+
+template <bool RAZER>
+__device__ __forceinline__ void decode_nv16(uint32_t w0, uint32_t w1, uint32_t sb, float s_t, float* xh)
+{
+    const float den = __fmul_rn(e4m3_to_f32(RAZER ? (sb & 0x7Fu) : sb), s_t);
+    const float special = (sb & 0x80u) ? -5.0f : 5.0f;
+    float q[16];
+    decode16(w0, w1, q);
+    if (RAZER) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t nib = ((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu;
+            q[i] = nib == 8u ? special : q[i];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(den, den));
+        xh[i] = p.x;
+        xh[i + 1] = p.y;
+    }
+}
+
+__device__ __forceinline__ void decode_mx32(const uint32_t* cw, uint32_t sb, float* xh)
+{
+    const float s = exp2i((int)sb - 127);
+    float q[32];
+    decode16(cw[0], cw[1], q);
+    decode16(cw[2], cw[3], q + 16);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(s, s));
+        xh[i] = p.x;
+        xh[i + 1] = p.y;
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void decode_unit(const uint32_t* cw, const uint32_t* sb, float s_t, float* xh)
+{
+    if (FMT == kMX) {
+        decode_mx32(cw, sb[0], xh);
+    } else {
+        decode_nv16<FMT == kRZ>(cw[0], cw[1], sb[0], s_t, xh);
+        decode_nv16<FMT == kRZ>(cw[2], cw[3], sb[1], s_t, xh + 16);
+    }
+}
+
+// Read a unit's codes and scale bytes (dense layouts).
+template <int FMT>
+__device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                            int64_t code_off, int64_t scale_off, bool full, bool a16, uint32_t* cw,
+                                            uint32_t* sb)
+{
+    const uint8_t* cp = codes + code_off;
+    if (full && a16) {
+        const uint4 c = ldg_nc_v4(cp);
+        cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
+    } else {
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(cp));
+        cw[0] = c.x; cw[1] = c.y;
+        if (full) {
+            const uint2 d = __ldg(reinterpret_cast<const uint2*>(cp + 8));
+            cw[2] = d.x; cw[3] = d.y;
+        } else {
+            cw[2] = 0; cw[3] = 0;
+        }
+    }
+    sb[0] = __ldg(scales + scale_off);
+    sb[1] = (FMT != kMX && full) ? (uint32_t)__ldg(scales + scale_off + 1) : 0u;
+}
+
+// ---------------------------------------------------------------------------
+// The tile pipeline
+// ---------------------------------------------------------------------------
+
+// Shared memory of a pipelined CTA: kStages tiles (1024-byte aligned for the
+// 128-byte swizzle) followed by one mbarrier per stage.
+constexpr int kPipeSmemBytes = kStages * kTileBytes + 1024 + 64;
+
+struct Pipe {
+    uint32_t tiles;   // shared address of stage 0
+    uint32_t bars;    // shared address of the stage barriers
+};
+
+__device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
+{
+    const uint32_t base = smem_u32(smem_raw);
+    Pipe p;
+    p.tiles = (base + 1023u) & ~1023u;
+    p.bars = p.tiles + kStages * kTileBytes;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) mbar_init(p.bars + 8 * s, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    return p;
+}
+
+// Tiles of this CTA: blockIdx.x + j * gridDim.x, walked backwards when reverse.
+struct Schedule {
+    int64_t count, mine;
+    bool reverse;
+    __device__ int64_t tile(int64_t j) const
+    {
+        const int64_t i = (int64_t)blockIdx.x + j * gridDim.x;
+        return reverse ? count - 1 - i : i;
+    }
+};
+
+__device__ __forceinline__ Schedule make_schedule(int64_t count, bool reverse)
+{
+    Schedule s;
+    s.count = count;
+    s.reverse = reverse;
+    s.mine = (int64_t)blockIdx.x < count ? (count - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+    return s;
+}
+
+template <bool FLAT>
+__device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
+                                           int64_t j)
+{
+    const int s = (int)(j % kStages);
+    int x, y;
+    tile_origin<FLAT>(tl, sc.tile(j), x, y);
+    mbar_arm(p.bars + 8 * s, kTileBytes);
+    tma_load_tile(p.tiles + s * kTileBytes, map, x, y, p.bars + 8 * s);
+}
+
+// Wait for tile j (bounded); the caller consumes the tile only when this
+// returned true and then calls pipe_release.
+__device__ __forceinline__ bool pipe_wait(const Pipe& p, int64_t j)
+{
+    return mbar_wait(p.bars + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+}
+
+// End of tile j: the CTA agrees on whether any thread's wait timed out.  If so,
+// thread 0 records it and waits (bounded) for the copies still in flight, and
+// the caller stops; otherwise thread 0 refills the slot with tile j + kStages.
+template <bool FLAT>
+__device__ __forceinline__ bool pipe_release(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
+                                             int64_t j, bool ok)
+{
+    if (!__syncthreads_or(!ok)) {
+        if (threadIdx.x == 0 && j + kStages < sc.mine) pipe_issue<FLAT>(p, map, tl, sc, j + kStages);
+        return true;
+    }
+    if (threadIdx.x == 0) {
+        atomicOr(&g_device_error, kErrPipelineTimeout);
+        const int64_t last = j + kStages < sc.mine ? j + kStages : sc.mine;
+        for (int64_t q = j; q < last; ++q) mbar_wait(p.bars + 8 * (int)(q % kStages), (uint32_t)((q / kStages) & 1));
+    }
+    __syncthreads();
+    return false;
+}
+
+__device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint32_t h, uint32_t* w)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint4 v = lds128(tile_chunk(tile, r, 4 * h + c));
+        w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Per-tile work (shared by the single-tensor kernels and the batch scheduler)
+// ---------------------------------------------------------------------------
+
+// Q1-Q6 on the unit this thread owns in tile k (shared address `tile`):
+// rotate, block scales, encode, RaZeR select, pack and store codes and scales.
+// Returns the unit's squared error when SSE.
+template <int FMT, bool ROT, bool SSE, bool FLAT>
+__device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, int64_t k, uint8_t* codes,
+                                                uint8_t* scales, const NvScale& nsc)
+{
+    const int t = threadIdx.x;
+    const bool a16 = FLAT || (tl.cols % 32) == 0;
+    const uint32_t r = (uint32_t)t >> 1, h = (uint32_t)t & 1u;
+    double acc = 0.0;
+    const Unit u = unit_of<FLAT>(tl, k, t);
+    uint32_t cw[4] = {0, 0, 0, 0}, sb0 = 0, sb1 = 0;
+    if (u.valid) {
+        if (FMT != kMX && !ROT) {
+            // two independent 16-element blocks, one after the other
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1 && !u.full) break;
+                uint32_t w[8];
+                const uint4 v0 = lds128(tile_chunk(tile, r, 4 * h + 2 * half));
+                const uint4 v1 = lds128(tile_chunk(tile, r, 4 * h + 2 * half + 1));
+                w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+                const uint32_t mm = bf16x2_absmax(
+                    bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
+                    bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+                float y[16];
+                unpack16(w, y);
+                uint32_t sbh;
+                double e = 0.0;
+                encode_nv16<FMT == kRZ, SSE ? kOutSse : kOutNone>(y, bf16x2_hmax_abs(mm), nsc, cw[2 * half],
+                                                                  cw[2 * half + 1], sbh, nullptr, &e);
+                if (half == 0) sb0 = sbh;
+                else sb1 = sbh;
+                if (SSE) acc += e;
+            }
+        } else {
+            float y[32], xh[32];
+            {
+                uint32_t w[16];
+                load_unit_words(tile, r, h, w);
+                unpack16(w, y);
+                unpack16(w + 8, y + 16);
+            }
+            if (ROT) wht32_inplace(y);
+            if (FMT == kMX) {
+                float am = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(y[i]));
+                encode_mx32<SSE>(y, am, cw, sb0, xh);
+            } else {
+                float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    a0 = fmaxf(a0, fabsf(y[i]));
+                    a1 = fmaxf(a1, fabsf(y[16 + i]));
+                }
+                encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y, a0, nsc, cw[0], cw[1], sb0, xh, nullptr);
+                encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16,
+                                                                nullptr);
+            }
+            if (SSE) {
+                // the original values again, from the tile still in shared memory
+                if (ROT) wht32_inplace(xh);
+                uint32_t w[16];
+                load_unit_words(tile, r, h, w);
+                unpack16(w, y);
+                unpack16(w + 8, y + 16);
+                acc += sse_of<32>(y, xh);
+            }
+        }
+        int64_t co, so;
+        unit_offsets<FLAT, FMT>(tl, u, co, so);
+        store_codes(codes + co, cw, u.full, a16);
+        if (FMT == kMX) {
+            scales[so] = (uint8_t)sb0;
+        } else if (u.full && a16) {
+            *reinterpret_cast<unsigned short*>(scales + so) = (unsigned short)(sb0 | (sb1 << 8));
+        } else {
+            scales[so] = (uint8_t)sb0;
+            if (u.full) scales[so + 1] = (uint8_t)sb1;
+        }
+    }
+    return acc;
+}
+
+// Q0 on the unit this thread owns in a tile: max |x| (of |H x| when rotating).
+// Out-of-range parts of a tile are zero-filled, so no validity test is needed.
+template <bool ROT>
+__device__ __forceinline__ float amax_tile(uint32_t tile)
+{
+    const int t = threadIdx.x;
+    uint32_t w[16];
+    load_unit_words(tile, (uint32_t)t >> 1, (uint32_t)t & 1u, w);
+    float m = 0.0f;
+    if (ROT) {
+        float y[32];
+        unpack16(w, y);
+        unpack16(w + 8, y + 16);
+        wht32_inplace(y);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(y[i]));
+    } else {
+        uint32_t mm = w[0];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) mm = bf16x2_absmax(mm, w[i]);
+        m = bf16x2_hmax_abs(mm);
+    }
+    return m;
+}
+
+}  // namespace fp4q

@@ -56,7 +56,29 @@ cudaError_t launch_sse_finalize(const double* partials, int n, double count, dou
                                 cudaStream_t st);
 
 // Copy the device error word of the current device to *bits (synchronous);
-// clear it afterwards when asked.
+// clear it afterwards when asked.  One word per kernel translation unit.
 cudaError_t read_device_errors(unsigned int* bits, bool clear);
+cudaError_t read_batch_device_errors(unsigned int* bits, bool clear);
+
+// Tile count of a bf16 matrix's view (see make_view): 16 KB tiles.
+int64_t view_tiles(const Geometry& g);
+
+// One tensor of a batch (device pointers; mse may be null).
+struct BatchTensor {
+    const void* x;
+    int64_t rows, cols, ldx;
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tensor_scale;
+    double* mse;
+};
+
+// Batch workspace: three rotating slots of per-CTA absmax and error partials.
+size_t batch_workspace_bytes();
+
+// Quantize n non-empty tensors as a chain of persistent kernels, one per tensor
+// (absmax pass of tensor j interleaved with the quantize pass of tensor j-1).
+cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, void* workspace,
+                                  cudaStream_t st);
 
 }  // namespace fp4q

@@ -30,7 +30,14 @@ STATUS_NAMES = {
 # Names the C header declares; the tests check that the library exports each one.
 ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc",
-               "fp4q_device_errors")
+               "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch")
+
+
+class TensorDesc(ctypes.Structure):
+    """fp4q_tensor_desc_t: one tensor of a batch (device pointers)."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ldx", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("mse", ctypes.c_void_p)]
 
 
 class Fp4qError(RuntimeError):
@@ -68,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.fp4q_quantize_noalloc.restype = i32
         L.fp4q_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         L.fp4q_device_errors.restype = i32
+        L.fp4q_batch_workspace_size.argtypes = [i32, ctypes.POINTER(TensorDesc), i32, i32]
+        L.fp4q_batch_workspace_size.restype = sz
+        L.fp4q_quantize_batch.argtypes = [i32, ctypes.POINTER(TensorDesc), i32, i32, u32, vp, sz, vp]
+        L.fp4q_quantize_batch.restype = i32
         _lib = L
     return _lib
 
@@ -139,6 +150,33 @@ def fp4q_device_errors(clear: bool = False) -> tuple[int, int]:
     return st, v.value
 
 
+def _descs(descs):
+    if isinstance(descs, ctypes.Array):
+        return descs
+    arr = (TensorDesc * max(1, len(descs)))()
+    for i, d in enumerate(descs):
+        arr[i] = d
+    return arr
+
+
+def fp4q_batch_workspace_size(count, descs, fmt, rotate) -> int:
+    return lib().fp4q_batch_workspace_size(count, _descs(descs), _fmt(fmt), int(rotate))
+
+
+def fp4q_quantize_batch(count, descs, fmt, rotate, flags, workspace, workspace_bytes, stream=None) -> int:
+    return lib().fp4q_quantize_batch(count, _descs(descs), _fmt(fmt), int(rotate), flags, _ptr(workspace),
+                                     workspace_bytes, _stream(stream))
+
+
+def tensor_desc(x, q: "Quantized") -> TensorDesc:
+    """Descriptor of bf16 matrix x and its outputs q (torch tensors)."""
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    return TensorDesc(x.data_ptr(), rows, cols, ld, q.codes.data_ptr(), q.scales.data_ptr(),
+                      q.tensor_scale.data_ptr() if q.tensor_scale is not None else None,
+                      q.mse.data_ptr() if q.mse is not None else None)
+
+
 # ---- torch-level wrappers -------------------------------------------------------
 
 class Quantized(NamedTuple):
@@ -203,6 +241,34 @@ def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_sc
     st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize")
     return Quantized(codes, scales, ts, mse)
+
+
+def empty_like_quantized(x: torch.Tensor, fmt, want_mse: bool = True) -> Quantized:
+    rows, cols = x.shape
+    B = block_size(fmt)
+    return Quantized(torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device),
+                     torch.empty(rows, cols // B, dtype=torch.uint8, device=x.device),
+                     torch.zeros(1, dtype=torch.float32, device=x.device),
+                     torch.empty(1, dtype=torch.float64, device=x.device) if want_mse else None)
+
+
+def quantize_batch(xs, fmt="nvfp4_razer", rotate: bool = False, outs=None, scale_given: bool = False,
+                   want_mse: bool = True, workspace: torch.Tensor | None = None, stream=None) -> list:
+    """Quantize a list of bf16 CUDA matrices with one fp4q_quantize_batch call.
+
+    With scale_given, each out's tensor_scale holds the input scale."""
+    if not xs:
+        return []
+    dev = xs[0].device
+    if outs is None:
+        outs = [empty_like_quantized(x, fmt, want_mse) for x in xs]
+    descs = _descs([tensor_desc(x, q) for x, q in zip(xs, outs)])
+    need = fp4q_batch_workspace_size(len(xs), descs, fmt, rotate)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+    flags = FLAG_TENSOR_SCALE_GIVEN if scale_given else 0
+    st = fp4q_quantize_batch(len(xs), descs, fmt, rotate, flags, ws, ws.numel(), stream)
+    _check(st, "fp4q_quantize_batch")
+    return outs
 
 
 def dequantize(q: Quantized, fmt="nvfp4_razer", rotate: bool = False, out: torch.Tensor | None = None,

@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--mode", choices=["batch", "per-call"], default="batch",
+                   help="batch: fp4q_quantize_batch over 16 layers (112 tensors) per call; "
+                        "per-call: one fp4q_quantize per tensor")
     return p.parse_args()
 
 
@@ -244,17 +247,40 @@ def main():
     ws = torch.zeros(fp4q.fp4q_workspace_size(0, 0, FMT, 0), dtype=torch.uint8, device=dev)
     L = fp4q.lib()
     fmt = fp4q.FORMATS[FMT]
-    calls = [(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), q.codes.data_ptr(), q.scales.data_ptr(),
-              q.tensor_scale.data_ptr(), q.mse.data_ptr(), x.numel()) for _, x, q in tensors]
-    launches_per_call = 3   # absmax, quantize, mse finaliser
+    if args.mode == "per-call":
+        calls = [(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), q.codes.data_ptr(), q.scales.data_ptr(),
+                  q.tensor_scale.data_ptr(), q.mse.data_ptr(), x.numel()) for _, x, q in tensors]
+        launches_per_call = 3   # absmax, quantize, mse finaliser
+        call_elements = [c[-1] for c in calls]
+        kernel_desc = "fp4q_quantize call: absmax pass + quantize pass + mse finaliser"
 
-    def step(events=None):
-        for k, (xp, r, c, ld, cp, sp, tp, mp, n) in enumerate(calls):
-            if events is not None:
-                events[2 * k].record(stream)
+        def one_call(k):
+            xp, r, c, ld, cp, sp, tp, mp, n = calls[k]
             st = L.fp4q_quantize(xp, r, c, ld, fmt, 0, 0, cp, sp, tp, mp, ws.data_ptr(), ws.numel(), sh)
             if st != 0:
                 raise fp4q.Fp4qError(st, "fp4q_quantize")
+    else:
+        groups = [tensors]                      # the whole weight set in one call
+        descs = [fp4q._descs([fp4q.tensor_desc(x, q) for _, x, q in g]) for g in groups]
+        ws_need = max(fp4q.fp4q_batch_workspace_size(len(g), d, FMT, 0) for g, d in zip(groups, descs))
+        bws = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        calls = list(range(len(groups)))
+        launches_per_call = len(tensors) + 2    # one chained kernel per tensor, plus the first and last
+        call_elements = [sum(x.numel() for _, x, _ in g) for g in groups]
+        kernel_desc = ("fp4q_quantize_batch over the weight set: chain of persistent kernels, each the absmax "
+                       "pass of one tensor interleaved with the quantize pass of the previous (PDL-chained); "
+                       "per-launch figures = call totals / launches")
+
+        def one_call(k):
+            st = L.fp4q_quantize_batch(len(groups[k]), descs[k], fmt, 0, 0, bws.data_ptr(), bws.numel(), sh)
+            if st != 0:
+                raise fp4q.Fp4qError(st, "fp4q_quantize_batch")
+
+    def step(events=None):
+        for k in range(len(calls)):
+            if events is not None:
+                events[2 * k].record(stream)
+            one_call(k)
             if events is not None:
                 events[2 * k + 1].record(stream)
 
@@ -286,17 +312,17 @@ def main():
     ms_per_step = ms / args.steps
     value = elements * world / (ms / 1e3) * args.steps
 
-    # per-call durations -> roofline of the quantize call (absmax + quantize + finaliser)
+    # per-call durations -> roofline of the call (its launches run back to back on the stream)
     call_ms = [ev[s][2 * k].elapsed_time(ev[s][2 * k + 1]) for s in range(args.steps) for k in range(len(calls))]
     avg_call_ms = statistics.mean(call_ms)
-    avg_call_bytes = BYTES_PER_ELEMENT * elements / len(calls)
+    avg_call_bytes = BYTES_PER_ELEMENT * statistics.mean(call_elements)
     peak, peak_kind = peaks()
     achieved = avg_call_bytes / (avg_call_ms / 1e3) / 1e9
     dram_bpe = traffic_record("quantize_nvfp4_razer_sse")
-    roofline = {"bound": "hbm", "kernel": "fp4q_quantize call: absmax pass + quantize pass + mse finaliser",
+    roofline = {"bound": "hbm", "kernel": kernel_desc,
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_kind": f"{peak_kind} copy bandwidth",
-                "traffic": (dram_bpe * elements / len(calls)) if dram_bpe else None,
+                "traffic": (dram_bpe * statistics.mean(call_elements)) if dram_bpe else None,
                 "algorithmic_bytes_per_launch": avg_call_bytes, "avg_launch_ms": avg_call_ms}
 
     # ---- check a result, outside the timed region ---------------------------------
@@ -316,6 +342,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "elements_per_step": elements * world, "layers": args.layers,
+                   "api": "fp4q_quantize_batch, one call per step" if args.mode == "batch" else
+                          "fp4q_quantize, one call per tensor",
                    "parallelism": f"dp{world} (independent weight sets, no collective)" if world > 1 else "1 GPU",
                    "l2": f"no flush: each step reads {elements * 2 / 1e9:.2f} GB of inputs (> 126 MB L2)"},
         "achieved_gbs": BYTES_PER_ELEMENT * elements * world / (ms_per_step / 1e3) / 1e9,
@@ -336,10 +364,14 @@ def main():
 
 
 def run_e2e(args, tensors, fmt, L, dev):
-    """Same metric from pinned host buffers: every step copies each tensor in, quantizes it
-    and copies codes, scales, tensor scale and MSE back; copies overlap the kernels."""
+    """Same metric from pinned host buffers: every step copies each group of
+    tensors in (one layer in batch mode, one tensor per call otherwise),
+    quantizes it and copies codes, scales, tensor scales and MSEs back; copies
+    of one group overlap the kernels of the other (two buffer sets, 3 streams)."""
     import torch
     from activation_quantization_block_b200 import fp4q
+    per = len(layer_shapes()) if args.mode == "batch" else 1
+    groups = [list(range(i, min(i + per, len(tensors)))) for i in range(0, len(tensors), per)]
     host_in = []
     for _, x, _ in tensors:
         h = torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -349,16 +381,19 @@ def run_e2e(args, tensors, fmt, L, dev):
                                torch.empty(q.scales.shape, dtype=torch.uint8, pin_memory=True),
                                torch.empty(1, dtype=torch.float32, pin_memory=True),
                                torch.empty(1, dtype=torch.float64, pin_memory=True)) for _, _, q in tensors]
-    big = max(x.numel() for _, x, _ in tensors)
-    staging = [torch.empty(big, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    outs = [fp4q.Quantized(torch.empty(big // 2, dtype=torch.uint8, device=dev),
-                           torch.empty(big // 16, dtype=torch.uint8, device=dev),
-                           torch.empty(1, dtype=torch.float32, device=dev),
-                           torch.empty(1, dtype=torch.float64, device=dev)) for _ in range(2)]
-    ws = torch.zeros(fp4q.fp4q_workspace_size(0, 0, fmt, 0), dtype=torch.uint8, device=dev)
-    h2d = torch.cuda.Stream(dev)
-    comp = torch.cuda.Stream(dev)
-    d2h = torch.cuda.Stream(dev)
+    # two buffer sets, each holding one group's inputs and outputs (by position in the group)
+    shapes = [[tensors[k][1].shape for k in g] for g in groups]
+    biggest = max(range(len(groups)), key=lambda i: sum(s[0] * s[1] for s in shapes[i]))
+    bufs = []
+    for _ in range(2):
+        xs = [torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in shapes[biggest]]
+        qs = [fp4q.empty_like_quantized(x, FMT) for x in xs]
+        bufs.append((xs, qs))
+    ws_bytes = max(fp4q.fp4q_batch_workspace_size(len(g), [fp4q.tensor_desc(x, q) for x, q in zip(*bufs[0])][:len(g)],
+                                                  FMT, 0) for g in groups)
+    ws_bytes = max(ws_bytes, fp4q.fp4q_workspace_size(0, 0, FMT, 0))
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    h2d, comp, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     in_ready = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
     out_free = [torch.cuda.Event() for _ in range(2)]
@@ -368,29 +403,35 @@ def run_e2e(args, tensors, fmt, L, dev):
         e.record(comp)
 
     def step():
-        for k, hx in enumerate(host_in):
-            b = k & 1
-            n = hx.numel()
-            r, c = hx.shape
-            h2d.wait_event(comp_done[b])          # staging[b] no longer read by an earlier quantize
+        for gi, g in enumerate(groups):
+            b = gi & 1
+            xs, qs = bufs[b]
+            h2d.wait_event(comp_done[b])          # buffer set b no longer read by an earlier call
             with torch.cuda.stream(h2d):
-                staging[b][:n].copy_(hx.view(-1), non_blocking=True)
+                for j, k in enumerate(g):
+                    xs[j].copy_(host_in[k], non_blocking=True)
                 in_ready[b].record(h2d)
             comp.wait_event(in_ready[b])
-            comp.wait_event(out_free[b])          # outs[b] copied out by an earlier D2H
-            st = L.fp4q_quantize(staging[b].data_ptr(), r, c, c, fmt, 0, 0, outs[b].codes.data_ptr(),
-                                 outs[b].scales.data_ptr(), outs[b].tensor_scale.data_ptr(),
-                                 outs[b].mse.data_ptr(), ws.data_ptr(), ws.numel(), comp.cuda_stream)
+            comp.wait_event(out_free[b])          # outputs of set b copied out by an earlier D2H
+            if args.mode == "batch":
+                d = fp4q._descs([fp4q.tensor_desc(xs[j], qs[j]) for j in range(len(g))])
+                st = L.fp4q_quantize_batch(len(g), d, fmt, 0, 0, ws.data_ptr(), ws.numel(), comp.cuda_stream)
+            else:
+                x, q = xs[0], qs[0]
+                st = L.fp4q_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.shape[1], fmt, 0, 0, q.codes.data_ptr(),
+                                     q.scales.data_ptr(), q.tensor_scale.data_ptr(), q.mse.data_ptr(), ws.data_ptr(),
+                                     ws.numel(), comp.cuda_stream)
             if st != 0:
-                raise fp4q.Fp4qError(st, "fp4q_quantize")
+                raise fp4q.Fp4qError(st, "quantize")
             comp_done[b].record(comp)
             d2h.wait_event(comp_done[b])
             with torch.cuda.stream(d2h):
-                ho = host_out[k]
-                ho.codes.view(-1).copy_(outs[b].codes[:n // 2], non_blocking=True)
-                ho.scales.view(-1).copy_(outs[b].scales[:n // 16], non_blocking=True)
-                ho.tensor_scale.copy_(outs[b].tensor_scale, non_blocking=True)
-                ho.mse.copy_(outs[b].mse, non_blocking=True)
+                for j, k in enumerate(g):
+                    ho = host_out[k]
+                    ho.codes.copy_(qs[j].codes, non_blocking=True)
+                    ho.scales.copy_(qs[j].scales, non_blocking=True)
+                    ho.tensor_scale.copy_(qs[j].tensor_scale, non_blocking=True)
+                    ho.mse.copy_(qs[j].mse, non_blocking=True)
                 out_free[b].record(d2h)
 
     step()
@@ -409,8 +450,10 @@ def run_e2e(args, tensors, fmt, L, dev):
     ok = all(torch.equal(host_out[k].codes, tensors[k][2].codes.cpu()) for k in (0, len(tensors) - 1))
     return {"value": elements / dt, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
             "d2h_bytes_per_step": d2h_bytes, "ms_per_step": dt * 1e3, "steps": args.e2e_steps,
-            "path": "pinned host bf16 -> H2D -> fp4q_quantize -> D2H codes/scales/scale/mse, 3 streams, "
-                    "double-buffered", "matches_device_results": bool(ok)}
+            "path": ("pinned host bf16 -> H2D -> fp4q_quantize_batch per layer" if args.mode == "batch" else
+                     "pinned host bf16 -> H2D -> fp4q_quantize per tensor") +
+                    " -> D2H codes/scales/scale/mse; two buffer sets, 3 streams",
+            "matches_device_results": bool(ok)}
 
 
 if __name__ == "__main__":

@@ -153,6 +153,41 @@ FP4Q_API fp4q_status_t fp4q_error(const void* x, int64_t ldx,
                          int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
                          double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
 
+/* One tensor of a batch: as the arguments of fp4q_quantize (device pointers;
+ * mse may be NULL, tensor_scale may be NULL for MXFP4). */
+typedef struct fp4q_tensor_desc {
+    const void* x;
+    int64_t rows, cols, ldx;
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tensor_scale;
+    double* mse;
+} fp4q_tensor_desc_t;
+
+/* Bytes of workspace fp4q_quantize_batch needs (independent of the tensors):
+ * three rotating slots of per-CTA partial maxima and partial sums. */
+FP4Q_API size_t fp4q_batch_workspace_size(int count, const fp4q_tensor_desc_t* tensors, fp4q_format_t fmt,
+                                          int rotate);
+
+/* Quantize `count` tensors, all in one format.  Results are those of calling
+ * fp4q_quantize on each tensor in order with the same fmt, rotate and flags
+ * (bit-identical codes, scales and tensor scales; each mse within fp64
+ * summation order).  `tensors` is a HOST array read during the call.
+ *
+ * The call enqueues one persistent kernel per tensor (plus one), chained with
+ * programmatic dependent launch: with the tensor scale computed, kernel j
+ * runs the absmax pass of tensor j interleaved with the quantize pass of
+ * tensor j-1 in the same SMs, so memory-bound and ALU-bound work overlap and
+ * each kernel's start overlaps its predecessor's tail; kernel j also
+ * finalises the MSE of tensor j-2.  The workspace (at least
+ * fp4q_batch_workspace_size bytes, 16-byte aligned) needs no clearing; calls
+ * sharing a workspace must not overlap on the device.  Errors as
+ * fp4q_quantize; the first invalid tensor's status is returned before
+ * anything is enqueued. */
+FP4Q_API fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* tensors, fp4q_format_t fmt,
+                                           int rotate, uint32_t flags, void* workspace, size_t workspace_bytes,
+                                           fp4q_stream_t stream);
+
 /* Bits of the device error word (fp4q_device_errors). */
 #define FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT 0x1u
 

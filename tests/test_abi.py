@@ -139,3 +139,36 @@ def test_binding_has_no_oracle_or_cpu_path():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "fp4q_oracle" not in text, f
+
+
+def _desc(**kw):
+    d = dict(x=A, rows=4, cols=64, ldx=64, codes=A, scales=A, tensor_scale=A, mse=None)
+    d.update(kw)
+    return fp4q.TensorDesc(**d)
+
+
+def test_batch_workspace_size_is_fixed():
+    one = fp4q.fp4q_batch_workspace_size(1, [_desc(rows=128, cols=8192, ldx=8192)], 1, 0)
+    two = fp4q.fp4q_batch_workspace_size(2, [_desc(rows=128, cols=8192, ldx=8192)] * 2, 1, 0)
+    assert one == two == 3 * 4096 * (4 + 8)     # three slots of per-CTA partials
+
+
+@pytest.mark.parametrize("descs,kw,expect", [
+    ([_desc()], dict(count=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    ([_desc()], dict(flags=4), "FP4Q_ERROR_INVALID_VALUE"),
+    ([_desc(), _desc(cols=40, ldx=40)], {}, "FP4Q_ERROR_SHAPE"),
+    ([_desc(), _desc(x=A + 8)], {}, "FP4Q_ERROR_MISALIGNED"),
+    ([_desc(tensor_scale=None)], {}, "FP4Q_ERROR_INVALID_VALUE"),
+    ([_desc(codes=None)], {}, "FP4Q_ERROR_INVALID_VALUE"),
+    ([_desc()], dict(workspace=None), "FP4Q_ERROR_WORKSPACE"),
+    ([_desc()], dict(workspace_bytes=100), "FP4Q_ERROR_WORKSPACE"),
+])
+def test_batch_rejects_bad_arguments(descs, kw, expect):
+    args = dict(count=len(descs), descs=descs, fmt=0, rotate=0, flags=0, workspace=A, workspace_bytes=1 << 20,
+                stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_quantize_batch(**args) == ST[expect]
+
+
+def test_batch_of_nothing_is_a_no_op():
+    assert fp4q.fp4q_quantize_batch(0, [], 0, 0, 0, None, 0, 0) == ST["FP4Q_SUCCESS"]
