@@ -20,8 +20,8 @@
 // kernel never starts before its predecessor's predecessor has finished.
 // Partial buffers rotate over three slots: kernel j reads slot j-1 and writes
 // slot j, so a kernel overlapping its predecessor's tail never writes a slot
-// that is still being read.  Tiles are assigned to CTAs round-robin (a fixed
-// schedule), so every partial sum is formed in a fixed order.
+// that is still being read.  Tiles are assigned to CTAs by a fixed schedule,
+// so every partial sum is formed in a fixed order.
 //
 // Method references (title, section): as fp4q_common.cuh.
 #include <new>
@@ -69,17 +69,21 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int t = threadIdx.x;
 
     // Items of this kernel: nq quantize tiles (walked backwards) and na absmax
-    // tiles, interleaved in proportion; CTA b takes items b, b + G, b + 2G, ...
+    // tiles.  CTA b owns quantize tiles b, b + G, ... and absmax tiles
+    // G-1-b, 2G-1-b, ... (so a CTA with one quantize tile more than another
+    // tends to have one absmax tile less), and walks its two lists
+    // interleaved in proportion to their lengths.  Each CTA thus gets an even
+    // share of both kinds, whatever the parity of G.
     const int64_t nq = a.has_q ? a.qtl.count : 0;
     const int64_t na = a.has_a ? a.atl.count : 0;
-    const int64_t tot = nq + na;
-    const int64_t G = gridDim.x, b = blockIdx.x;
-    const int64_t mine = b < tot ? (tot - 1 - b) / G + 1 : 0;
+    const int64_t G = gridDim.x, b = blockIdx.x, ab = G - 1 - b;
+    const int64_t my_q = b < nq ? (nq - 1 - b) / G + 1 : 0;
+    const int64_t my_a = ab < na ? (na - 1 - ab) / G + 1 : 0;
+    const int64_t mine = my_q + my_a;
     auto item = [&](int64_t jj, bool& is_q, int64_t& tile) {
-        const int64_t i = b + jj * G;
-        const int64_t qb = i * nq / tot;
-        is_q = (i + 1) * nq / tot > qb;
-        tile = is_q ? nq - 1 - qb : i - qb;
+        const int64_t k = jj * my_q / mine;   // quantize items before item jj
+        is_q = (jj + 1) * my_q / mine > k;
+        tile = is_q ? nq - 1 - (b + k * G) : ab + (jj - k) * G;
     };
     auto issue = [&](int64_t jj) {
         bool is_q;
@@ -96,8 +100,8 @@ __global__ void __launch_bounds__(kThreads, 3)
             if (a.a_flat) tile_origin<true>(a.atl, tile, x, y);
             else tile_origin<false>(a.atl, tile, x, y);
         }
-        mbar_arm(p.bars + 8 * s, kTileBytes);
-        tma_load_tile(p.tiles + s * kTileBytes, is_q ? &qmap : &amap, x, y, p.bars + 8 * s);
+        mbar_arm(p.full + 8 * s, kTileBytes);
+        tma_load_tile(p.tiles + s * kTileBytes, is_q ? &qmap : &amap, x, y, p.full + 8 * s);
     };
     if (t == 0)
         for (int64_t jj = 0; jj < mine && jj < kStages; ++jj) issue(jj);
@@ -138,31 +142,28 @@ __global__ void __launch_bounds__(kThreads, 3)
     double acc = 0.0;
     float m = 0.0f;
     for (int64_t jj = 0; jj < mine; ++jj) {
+        if (!pipe_acquire(p, jj)) {
+            pipe_fail(p, jj, jj + kStages < mine ? jj + kStages : mine);
+            break;
+        }
         const int s = (int)(jj % kStages);
-        const bool ok = mbar_wait(p.bars + 8 * s, (uint32_t)((jj / kStages) & 1));
         const bool is_q = slot_q[s] != 0;
         const int64_t tile = slot_tile[s];
         const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
-        if (ok) {
-            if (is_q) {
-                if (a.q_flat) acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc);
-                else acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc);
-            } else {
-                m = fmaxf(m, amax_tile<ROT>(tp));
-            }
+        if (is_q) {
+            if (a.q_flat) acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc);
+            else acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc);
+        } else {
+            m = fmaxf(m, amax_tile<ROT>(tp));
         }
-        // end of the tile: agree on timeouts, then refill the slot
-        if (__syncthreads_or(!ok)) {
-            if (t == 0) {
-                atomicOr(&g_device_error, kErrPipelineTimeout);
-                const int64_t last = jj + kStages < mine ? jj + kStages : mine;
-                for (int64_t q = jj + 1; q < last; ++q)
-                    mbar_wait(p.bars + 8 * (int)(q % kStages), (uint32_t)((q / kStages) & 1));
+        pipe_release(p, jj);
+        if (t == 0 && jj + kStages < mine) {
+            if (!pipe_stage_free(p, jj)) {
+                pipe_fail(p, jj + 1, jj + kStages);
+                break;
             }
-            __syncthreads();
-            break;
+            issue(jj + kStages);
         }
-        if (t == 0 && jj + kStages < mine) issue(jj + kStages);
     }
     if (a.has_a) {
         m = block_max(m, shf);

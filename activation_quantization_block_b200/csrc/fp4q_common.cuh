@@ -480,12 +480,18 @@ __device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, c
 // ---------------------------------------------------------------------------
 
 // Shared memory of a pipelined CTA: kStages tiles (1024-byte aligned for the
-// 128-byte swizzle) followed by one mbarrier per stage.
-constexpr int kPipeSmemBytes = kStages * kTileBytes + 1024 + 64;
+// 128-byte swizzle), then a "full" and an "empty" mbarrier per stage.
+constexpr int kPipeSmemBytes = kStages * kTileBytes + 1024 + 128;
+constexpr int kWarps = kThreads / 32;
 
+// Stage s is "full" when its copy has landed (one arrival by thread 0 with the
+// byte count, completed by the copy) and "empty" when every warp has finished
+// reading it (one arrival per warp).  Warps consume tiles independently; only
+// thread 0, which refills the stages, waits for a stage to become empty.
 struct Pipe {
     uint32_t tiles;   // shared address of stage 0
-    uint32_t bars;    // shared address of the stage barriers
+    uint32_t full;    // shared address of the full barriers
+    uint32_t empty;   // shared address of the empty barriers
 };
 
 __device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
@@ -493,10 +499,14 @@ __device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
     const uint32_t base = smem_u32(smem_raw);
     Pipe p;
     p.tiles = (base + 1023u) & ~1023u;
-    p.bars = p.tiles + kStages * kTileBytes;
+    p.full = p.tiles + kStages * kTileBytes;
+    p.empty = p.full + 8 * kStages;
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) mbar_init(p.bars + 8 * s, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(p.full + 8 * s, 1);
+            mbar_init(p.empty + 8 * s, kWarps);
+        }
         mbar_init_fence();
     }
     __syncthreads();
@@ -523,6 +533,7 @@ __device__ __forceinline__ Schedule make_schedule(int64_t count, bool reverse)
     return s;
 }
 
+// Thread 0: start the copy of the j-th tile of the schedule into its stage.
 template <bool FLAT>
 __device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
                                            int64_t j)
@@ -530,35 +541,37 @@ __device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map
     const int s = (int)(j % kStages);
     int x, y;
     tile_origin<FLAT>(tl, sc.tile(j), x, y);
-    mbar_arm(p.bars + 8 * s, kTileBytes);
-    tma_load_tile(p.tiles + s * kTileBytes, map, x, y, p.bars + 8 * s);
+    mbar_arm(p.full + 8 * s, kTileBytes);
+    tma_load_tile(p.tiles + s * kTileBytes, map, x, y, p.full + 8 * s);
 }
 
-// Wait for tile j (bounded); the caller consumes the tile only when this
-// returned true and then calls pipe_release.
-__device__ __forceinline__ bool pipe_wait(const Pipe& p, int64_t j)
+// Every thread: wait (bounded) until the j-th tile has landed.
+__device__ __forceinline__ bool pipe_acquire(const Pipe& p, int64_t j)
 {
-    return mbar_wait(p.bars + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+    return mbar_wait(p.full + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
 }
 
-// End of tile j: the CTA agrees on whether any thread's wait timed out.  If so,
-// thread 0 records it and waits (bounded) for the copies still in flight, and
-// the caller stops; otherwise thread 0 refills the slot with tile j + kStages.
-template <bool FLAT>
-__device__ __forceinline__ bool pipe_release(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
-                                             int64_t j, bool ok)
+// Every warp, after its last read of the j-th tile: release the stage.
+__device__ __forceinline__ void pipe_release(const Pipe& p, int64_t j)
 {
-    if (!__syncthreads_or(!ok)) {
-        if (threadIdx.x == 0 && j + kStages < sc.mine) pipe_issue<FLAT>(p, map, tl, sc, j + kStages);
-        return true;
-    }
-    if (threadIdx.x == 0) {
-        atomicOr(&g_device_error, kErrPipelineTimeout);
-        const int64_t last = j + kStages < sc.mine ? j + kStages : sc.mine;
-        for (int64_t q = j; q < last; ++q) mbar_wait(p.bars + 8 * (int)(q % kStages), (uint32_t)((q / kStages) & 1));
-    }
-    __syncthreads();
-    return false;
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(p.empty + 8 * (int)(j % kStages)) : "memory");
+}
+
+// Thread 0: wait (bounded) until every warp has released the j-th tile's stage.
+__device__ __forceinline__ bool pipe_stage_free(const Pipe& p, int64_t j)
+{
+    return mbar_wait(p.empty + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+}
+
+// After a timeout: record it; thread 0 waits (bounded) for the copies it issued
+// that may still be in flight, tiles [from, to) of the schedule.
+__device__ __forceinline__ void pipe_fail(const Pipe& p, int64_t from, int64_t to)
+{
+    if ((threadIdx.x & 31) == 0) atomicOr(&g_device_error, kErrPipelineTimeout);
+    if (threadIdx.x == 0)
+        for (int64_t q = from; q < to; ++q) pipe_acquire(p, q);
 }
 
 __device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint32_t h, uint32_t* w)

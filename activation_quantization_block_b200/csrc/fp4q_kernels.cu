@@ -62,9 +62,19 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ 
     pdl_trigger();
     float m = 0.0f;
     for (int64_t j = 0; j < sc.mine; ++j) {
-        const bool ok = pipe_wait(p, j);
-        if (ok) m = fmaxf(m, amax_tile<ROT>(p.tiles + (uint32_t)(j % kStages) * kTileBytes));
-        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
+        if (!pipe_acquire(p, j)) {
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            break;
+        }
+        m = fmaxf(m, amax_tile<ROT>(p.tiles + (uint32_t)(j % kStages) * kTileBytes));
+        pipe_release(p, j);
+        if (t == 0 && j + kStages < sc.mine) {
+            if (!pipe_stage_free(p, j)) {
+                pipe_fail(p, j + 1, j + kStages);
+                break;
+            }
+            pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
+        }
     }
     m = block_max(m, shf);
     if (t == 0) a.partials[blockIdx.x] = m;
@@ -117,10 +127,20 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_cons
 
     double acc = 0.0;
     for (int64_t j = 0; j < sc.mine; ++j) {
-        const bool ok = pipe_wait(p, j);
+        if (!pipe_acquire(p, j)) {
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            break;
+        }
         const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
-        if (ok) acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc);
-        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
+        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc);
+        pipe_release(p, j);
+        if (t == 0 && j + kStages < sc.mine) {
+            if (!pipe_stage_free(p, j)) {
+                pipe_fail(p, j + 1, j + kStages);
+                break;
+            }
+            pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
+        }
     }
     if (SSE) {
         acc = block_sum(acc, shd);
@@ -160,8 +180,11 @@ __global__ void __launch_bounds__(kThreads, 3) error_kernel(const __grid_constan
             unit_offsets<FLAT, FMT>(a.tl, u, co, so);
             load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
         }
-        const bool ok = pipe_wait(p, j);
-        if (ok && u.valid) {
+        if (!pipe_acquire(p, j)) {
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            break;
+        }
+        if (u.valid) {
             const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
             uint32_t w[16];
             load_unit_words(tile, r, h, w);
@@ -176,7 +199,14 @@ __global__ void __launch_bounds__(kThreads, 3) error_kernel(const __grid_constan
             unpack16(w + 8, x + 16);
             acc += sse_of<32>(x, xh);
         }
-        if (!pipe_release<FLAT>(p, &xmap, a.tl, sc, j, ok)) break;
+        pipe_release(p, j);
+        if (t == 0 && j + kStages < sc.mine) {
+            if (!pipe_stage_free(p, j)) {
+                pipe_fail(p, j + 1, j + kStages);
+                break;
+            }
+            pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
+        }
     }
     acc = block_sum(acc, shd);
     if (t == 0) a.sse_partials[blockIdx.x] = acc;
