@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
     __shared__ double shd[kThreads];
-    __shared__ float den_tab[128], rcp_tab[128];
+    __shared__ NvTable nvt;
     __shared__ int64_t slot_tile[kStages];   // item of each pipeline slot, decoded once by thread 0
     __shared__ int32_t slot_q[kStages];
     const Pipe p = pipe_setup(smem_raw);
@@ -133,11 +133,12 @@ __global__ void __launch_bounds__(kThreads, 3)
         if (t == 0) *a.fin_mse = a.fin_count > 0.0 ? shd[0] / a.fin_count : 0.0;
     }
     pdl_trigger();
-    NvScale nsc;
-    nsc.den = den_tab;
-    nsc.rcp = rcp_tab;
-    if (a.has_q && FMT != kMX) nsc = nv_scale_setup(s_t, den_tab, rcp_tab);
-    __syncthreads();   // the slot items written by thread 0 are visible from here on
+    NvScale nsc{};
+    if (a.has_q && FMT != kMX) nsc = nv_scale_setup(s_t, &nvt);
+    // The first items, written by thread 0, are visible after this barrier; a
+    // refill's item is written before thread 0 arms its stage, and the
+    // consumers' acquire of the landed phase makes it visible.
+    __syncthreads();
 
     double acc = 0.0;
     float m = 0.0f;

@@ -15,6 +15,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdint>
 
 #include "fp4q_device.cuh"
@@ -220,21 +221,26 @@ __device__ __forceinline__ void decode16(uint32_t w0, uint32_t w1, float* q)
 }
 
 // Per-tensor constants of the NVFP4 block-scale step, shared by a CTA: for
-// each of the 127 non-negative finite E4M3 bytes b, den[b] = RN(dec(b) * s_t)
-// and rcp[b] = RN(1 / den[b]) (0 when den[b] = 0: a zero scale zeroes every
-// code).  The quotient t = RN(a / RN(6 s_t)) uses inv6 = RN(1 / RN(6 s_t)) and
-// one correction step (Markstein's theorem: with y = RN(1/b) and a faithful
-// q = RN(a y), the residual r = a - q b is exact and RN(q + r y) = RN(a / b));
-// `exact_div` selects IEEE division when RN(6 s_t) is outside [2^-64, 2^64],
-// where the theorem's no-underflow conditions are not guaranteed.
+// each of the 127 non-negative finite E4M3 bytes b, den[b] = RN(dec(b) * s_t),
+// rcp[b] = RN(1 / den[b]) (0 when den[b] = 0: a zero scale zeroes every code)
+// and den[b]^2 (exact in binary64).  The quotient t = RN(a / RN(6 s_t)) uses
+// inv6 = RN(1 / RN(6 s_t)) and one correction step (Markstein's theorem: with
+// y = RN(1/b) and a faithful q = RN(a y), the residual r = a - q b is exact and
+// RN(q + r y) = RN(a / b)); `exact_div` selects IEEE division when RN(6 s_t)
+// is outside [2^-64, 2^64], where the theorem's no-underflow conditions are
+// not guaranteed.
+struct NvTable {
+    float2 dr[128];       // {den, rcp}
+    double den2[128];     // den^2
+};
+
 struct NvScale {
     float s_t, six_st, inv6;
     bool exact_div;
-    const float* den;
-    const float* rcp;
+    uint32_t tab;         // shared address of the CTA's NvTable
 };
 
-__device__ __forceinline__ NvScale nv_scale_setup(float s_t, float* den_tab, float* rcp_tab)
+__device__ __forceinline__ NvScale nv_scale_setup(float s_t, NvTable* tab)
 {
     NvScale c;
     c.s_t = s_t;
@@ -243,13 +249,28 @@ __device__ __forceinline__ NvScale nv_scale_setup(float s_t, float* den_tab, flo
     c.inv6 = c.exact_div ? 0.0f : __frcp_rn(c.six_st);
     for (int b = threadIdx.x; b < 128; b += blockDim.x) {
         const float d = b < 127 ? __fmul_rn(e4m3_to_f32((uint32_t)b), s_t) : 0.0f;
-        den_tab[b] = d;
-        rcp_tab[b] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        tab->dr[b] = make_float2(d, d != 0.0f ? __frcp_rn(d) : 0.0f);
+        tab->den2[b] = (double)d * (double)d;
     }
     __syncthreads();
-    c.den = den_tab;
-    c.rcp = rcp_tab;
+    c.tab = smem_u32(tab);
     return c;
+}
+
+// {den, rcp} of scale byte sb (bit 7 clear).
+__device__ __forceinline__ float2 nv_den_rcp(const NvScale& c, uint32_t sb)
+{
+    float2 v;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(c.tab + 8u * sb));
+    return v;
+}
+
+// den^2 of scale byte sb (bit 7 clear).
+__device__ __forceinline__ double nv_den2(const NvScale& c, uint32_t sb)
+{
+    double v;
+    asm("ld.shared.f64 %0, [%1];" : "=d"(v) : "r"(c.tab + (uint32_t)offsetof(NvTable, den2) + 8u * sb));
+    return v;
 }
 
 // t = RN(a / RN(6 s_t)) for a >= 0.
@@ -261,21 +282,64 @@ __device__ __forceinline__ float nv_block_ratio(const NvScale& c, float a)
     return __fmaf_rn(r, c.inv6, q);
 }
 
-// Outputs of the block encoders besides codes and scale.
-enum { kOutNone = 0, kOutSse = 1, kOutXh = 2 };
+// RaZeR remap of one block given cs[i] = sign(v_i) * gain_i, the signed gains
+// of remapping element i to sign(v_i) * 5 (multiples of 2^-20 in [-1, 1]),
+// and their exact sum S = gain(+5) - gain(-5): -5 only when its gain is
+// strictly larger.  Winners are the candidates of the chosen sign.  With
+// x = cs * (+-2^40), every candidate has |x| >= 2^20 and encodes (saturating)
+// as +6 = 0b0111 when it wins and as -6 = 0b1111 otherwise, and every other
+// element as +-0; so bit 0 and not bit 3 of a nibble flags a winner, whose
+// code becomes 0b1000.
+__device__ __forceinline__ void razer_apply(const float* cs, float S, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+{
+    const float sk = S < 0.0f ? -0x1p40f : 0x1p40f;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(cs[i], cs[i + 1]), make_float2(sk, sk));
+        x[i] = p.x;
+        x[i + 1] = p.y;
+    }
+    const uint32_t k0 = e2m1x8(x), k1 = e2m1x8(x + 8);
+    const uint32_t f0 = k0 & ~(k0 >> 3) & 0x11111111u;
+    const uint32_t f1 = k1 & ~(k1 >> 3) & 0x11111111u;
+    w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
+    w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
+    if (S < 0.0f) sb |= 0x80u;
+}
 
-// One 16-element NVFP4 block.  y: values (rotated when rotating); a: their
-// absmax.  Writes two code words and the scale byte.  OUT = kOutXh: xh receives
-// the fp32 reconstruction RN(q * den).  OUT = kOutSse: *sse receives
-// sum (y - q den)^2, each difference taken with a single rounding
-// (RN(y - q den), within half an fp32 ulp of y - RN(q den)).
-template <bool RAZER, int OUT>
+// RaZeR selection from the scaled values alone (any magnitude).  For |v| in
+// (4.5, 5.5) the regular value is 4 (|v| <= 5) or 6 and
+//   (|v| - q)^2 - (|v| - 5)^2 = 1 - 2 | |v| - 5 |,
+// positive exactly on that open interval; elsewhere the gain is clamped to 0.
+// |v| - 5 is exact there, so each gain is a multiple of 2^-20 and every sum of
+// them is exact in any order.
+__device__ __forceinline__ void razer_tent(const float* v, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+{
+    float cs[16];
+    float2 sp[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        cs[i] = copysignf(__saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f)), v[i]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sp[i] = make_float2(cs[2 * i], cs[2 * i + 1]);
+#pragma unroll
+    for (int k = 4; k > 0; k >>= 1)
+#pragma unroll
+        for (int i = 0; i < k; ++i) sp[i] = add2_rn(sp[i], sp[i + k]);
+    razer_apply(cs, sp[0].x + sp[0].y, w0, w1, sb);
+}
+
+// One 16-element NVFP4 / RaZeR block of values y (rotated ones, on the rotated
+// path) with absmax a: two code words and the scale byte and, when XH, the
+// fp32 reconstruction xh = RN(q den) (RaZeR winners: RN(+-5 den)).
+template <bool RAZER, bool XH>
 __device__ __forceinline__ void encode_nv16(const float* y, float a, const NvScale& sc, uint32_t& c0, uint32_t& c1,
-                                            uint32_t& sb_out, float* xh, double* sse)
+                                            uint32_t& sb_out, float* xh)
 {
     uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
-    const float den = sc.den[sb];
-    const float r = sc.rcp[sb];
+    const float2 dr = nv_den_rcp(sc, sb);
+    const float den = dr.x, r = dr.y;
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
@@ -285,82 +349,175 @@ __device__ __forceinline__ void encode_nv16(const float* y, float a, const NvSca
     }
     uint32_t w0 = canonical_zero(e2m1x8(v));
     uint32_t w1 = canonical_zero(e2m1x8(v + 8));
-
-    float win[16];
-    float special = 0.0f;
-    if (RAZER) {
-        // Gain of remapping element i to sign(v_i) * 5.  For |v_i| in (4.5, 5.5)
-        // the regular value is 4 (|v| <= 5) or 6 and
-        //   (|v| - q)^2 - (|v| - 5)^2 = 1 - 2 | |v| - 5 |,
-        // which is positive exactly on that open interval; elsewhere it is
-        // clamped to 0.  Each term is a multiple of 2^-20 in [0, 1], so the fp32
-        // sum S = gain(+5) - gain(-5) is exact in any order.
-        float cs[16];
-        float S = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float c = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
-            cs[i] = copysignf(c, v[i]);
-            S += cs[i];
-        }
-        // -5 only when its gain is strictly larger.  Winners are the candidates
-        // of the chosen sign: cs * sign >= 2^-20, so win = sat(cs * sign * 2^40)
-        // is exactly 1 for a winner and 0 otherwise (+0 or -0).
-        const float sk = S < 0.0f ? -0x1p40f : 0x1p40f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) win[i] = __saturatef(__fmul_rn(cs[i], sk));
-        // E2M1 of 1.0 is 0b0010 and of +-0 is 0b0000 / 0b1000: bit 1 of each
-        // nibble flags a winner; winners' codes become 0b1000.
-        const uint32_t f0 = (e2m1x8(win) >> 1) & 0x11111111u;
-        const uint32_t f1 = (e2m1x8(win + 8) >> 1) & 0x11111111u;
-        w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
-        w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
-        if (S < 0.0f) sb |= 0x80u;
-        special = S < 0.0f ? -5.0f : 5.0f;
-    }
-
-    if (OUT != kOutNone) {
-        // codes as written (RaZeR winners decode to -0 here and are fixed below)
+    if (RAZER) razer_tent(v, w0, w1, sb);
+    if (XH) {
         float q[16];
         decode16(w0, w1, q);
-        if (OUT == kOutSse) {
-            const float nden = -den;
-            const float nx5 = -__fmul_rn(special, den);   // -RN(special * den)
-            float2 acc = make_float2(0.0f, 0.0f);
-            float d[16];
+        const float special = (sb & 0x80u) ? -5.0f : 5.0f;
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                float2 e = fma2_rn(make_float2(q[i], q[i + 1]), make_float2(nden, nden),
-                                   make_float2(y[i], y[i + 1]));
-                if (RAZER) e = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(nx5, nx5), e);
-                d[i] = e.x;
-                d[i + 1] = e.y;
-                acc = fma2_rn(e, e, acc);
-            }
-            const float es = acc.x + acc.y;
-            *sse = (es >= 0x1p-100f && es <= 3.0e38f) ? (double)es : sse16_rescaled(d);
-        } else {
+        for (int i = 0; i < 16; i += 2) {
+            float q0 = q[i], q1 = q[i + 1];
             if (RAZER) {
-#pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    // winners: -0 + 1 * special; others: q + 0 * special
-                    const float2 n = fma2_rn(make_float2(win[i], win[i + 1]), make_float2(special, special),
-                                             make_float2(q[i], q[i + 1]));
-                    q[i] = n.x;
-                    q[i + 1] = n.y;
-                }
+                if ((((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu) == 8u) q0 = special;
+                if ((((i < 8 ? w0 : w1) >> (4 * ((i + 1) & 7))) & 0xFu) == 8u) q1 = special;
             }
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(den, den));
-                xh[i] = p.x;
-                xh[i + 1] = p.y;
-            }
+            const float2 p = mul2_rn(make_float2(q0, q1), make_float2(den, den));
+            xh[i] = p.x;
+            xh[i + 1] = p.y;
         }
     }
     c0 = w0;
     c1 = w1;
     sb_out = sb;
+}
+
+// ---------------------------------------------------------------------------
+// Unrotated NVFP4 / RaZeR blocks straight from the bf16 tile
+// ---------------------------------------------------------------------------
+
+struct BlockOut {
+    uint32_t w0, w1, sb;
+    double sse;
+};
+
+// One block recomputed in full from its bf16 words in shared memory (chunks
+// at a0 and a1), given its unsigned scale byte and {den, rcp}: codes, scale
+// byte and the squared error in the original domain, each difference
+// y - RN(q den) taken in fp32 (zero when the element is reproduced) and
+// squared and summed in fp64.  Taken for the rare blocks the fast path below
+// does not cover.
+template <bool RAZER>
+__device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32_t sb, float den, float r)
+{
+    uint32_t w[8];
+    const uint4 c0 = lds128(a0), c1 = lds128(a1);
+    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+    w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+    float y[16], v[16];
+    unpack16(w, y);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+        v[i] = p.x;
+        v[i + 1] = p.y;
+    }
+    BlockOut o;
+    o.w0 = canonical_zero(e2m1x8(v));
+    o.w1 = canonical_zero(e2m1x8(v + 8));
+    o.sb = sb;
+    if (RAZER) razer_tent(v, o.w0, o.w1, o.sb);
+    float q[16];
+    decode16(o.w0, o.w1, q);
+    const float special = (o.sb & 0x80u) ? -5.0f : 5.0f;
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t nib = ((i < 8 ? o.w0 : o.w1) >> (4 * (i & 7))) & 0xFu;
+        const float qi = (RAZER && nib == 8u) ? special : q[i];
+        const double d = (double)(y[i] - __fmul_rn(qi, den));
+        s = fma(d, d, s);
+    }
+    o.sse = s;
+    return o;
+}
+
+// One unrotated 16-element NVFP4 / RaZeR block from its eight bf16x2 words w
+// (chunks a0, a1 of the tile): two code words, the scale byte and, when SSE,
+// the block's squared error.
+//
+// The squared error is formed in the scaled domain.  With v = RN(y r) the
+// scaled values and q the regular grid values, e = q - v is exact (see
+// e2m1x8_diff) and the block's error is den^2 (sum e^2 - G), where G is the
+// total gain of the RaZeR winners (0 for NVFP4).  For a candidate (|v| in
+// (4.5, 5.5), q = +-4 or +-6) the gain 1 - 2||v| - 5| equals 2|e| - 1, and
+// sat(2|e| - 1) is 0 for every other element as long as |v| <= 6.5, so gains,
+// decision and G come from e with no further per-element work.  den v differs
+// from y by at most 2^-23 |y| (two roundings), the only departure from the
+// exact error besides fp32 rounding of the sum.
+//
+// Blocks outside the fast path's assumptions are recomputed by
+// nv_block_exact: max |v| > 6.5 (a saturated scale byte, or a subnormal one
+// far below the block absmax), a fast sum below 2^-30 (the block is reproduced
+// exactly or almost, and the exact sum keeps a zero error zero), or one that
+// is not finite (an infinite reciprocal).
+template <bool RAZER, bool SSE>
+__device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_t a1, const NvScale& sc,
+                                         uint32_t& c0, uint32_t& c1, uint32_t& sb_out, double& sse)
+{
+    const uint32_t mm = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
+                                      bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+    const float a = bf16x2_hmax_abs(mm);
+    uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
+    const float2 dr = nv_den_rcp(sc, sb);
+    float v[16];
+    {
+        float y[16];
+        unpack16(w, y);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(dr.y, dr.y));
+            v[i] = p.x;
+            v[i + 1] = p.y;
+        }
+    }
+    if (!SSE) {
+        uint32_t w0 = canonical_zero(e2m1x8(v)), w1 = canonical_zero(e2m1x8(v + 8));
+        if (RAZER) razer_tent(v, w0, w1, sb);
+        c0 = w0;
+        c1 = w1;
+        sb_out = sb;
+        return;
+    }
+    float e[16];
+    uint32_t w0 = e2m1x8_diff(v, e), w1 = e2m1x8_diff(v + 8, e + 8);
+    float2 sq[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        sq[i] = mul2_rn(make_float2(e[2 * i], e[2 * i + 1]), make_float2(e[2 * i], e[2 * i + 1]));
+        sq[i] = fma2_rn(make_float2(e[2 * i + 8], e[2 * i + 9]), make_float2(e[2 * i + 8], e[2 * i + 9]), sq[i]);
+    }
+    sq[0] = add2_rn(add2_rn(sq[0], sq[1]), add2_rn(sq[2], sq[3]));
+    float sv = sq[0].x + sq[0].y;
+    w0 = canonical_zero(w0);
+    w1 = canonical_zero(w1);
+    const uint32_t sb0 = sb;
+    if (RAZER) {
+        float cs[16];
+        float2 gp[8], sp[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float g0 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i]), -1.0f));
+            const float g1 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i + 1]), -1.0f));
+            cs[i] = copysignf(g0, v[i]);
+            cs[i + 1] = copysignf(g1, v[i + 1]);
+            gp[i / 2] = make_float2(g0, g1);
+            sp[i / 2] = make_float2(cs[i], cs[i + 1]);
+        }
+        // pairwise sums (exact in any order)
+#pragma unroll
+        for (int k = 4; k > 0; k >>= 1)
+#pragma unroll
+            for (int i = 0; i < k; ++i) {
+                gp[i] = add2_rn(gp[i], gp[i + k]);
+                sp[i] = add2_rn(sp[i], sp[i + k]);
+            }
+        const float S = sp[0].x + sp[0].y;
+        sv -= 0.5f * ((gp[0].x + gp[0].y) + fabsf(S));   // G = max(gain(+5), gain(-5))
+        razer_apply(cs, S, w0, w1, sb);
+    }
+    const bool fast = sv >= 0x1p-30f && sv <= 0x1p64f && (!RAZER || __fmul_rn(a, dr.y) <= 6.5f);
+    if (fast) {
+        c0 = w0;
+        c1 = w1;
+        sb_out = sb;
+        sse = (double)sv * nv_den2(sc, sb0);
+    } else {
+        const BlockOut o = nv_block_exact<RAZER>(a0, a1, sb0, dr.x, dr.y);
+        c0 = o.w0;
+        c1 = o.w1;
+        sb_out = o.sb;
+        sse = o.sse;
+    }
 }
 
 // One 32-element MXFP4 block.
@@ -608,19 +765,14 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
             for (int half = 0; half < 2; ++half) {
                 if (half == 1 && !u.full) break;
                 uint32_t w[8];
-                const uint4 v0 = lds128(tile_chunk(tile, r, 4 * h + 2 * half));
-                const uint4 v1 = lds128(tile_chunk(tile, r, 4 * h + 2 * half + 1));
+                const uint32_t a0 = tile_chunk(tile, r, 4 * h + 2 * half);
+                const uint32_t a1 = tile_chunk(tile, r, 4 * h + 2 * half + 1);
+                const uint4 v0 = lds128(a0), v1 = lds128(a1);
                 w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
                 w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-                const uint32_t mm = bf16x2_absmax(
-                    bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
-                    bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
-                float y[16];
-                unpack16(w, y);
                 uint32_t sbh;
                 double e = 0.0;
-                encode_nv16<FMT == kRZ, SSE ? kOutSse : kOutNone>(y, bf16x2_hmax_abs(mm), nsc, cw[2 * half],
-                                                                  cw[2 * half + 1], sbh, nullptr, &e);
+                nv_block<FMT == kRZ, SSE>(w, a0, a1, nsc, cw[2 * half], cw[2 * half + 1], sbh, e);
                 if (half == 0) sb0 = sbh;
                 else sb1 = sbh;
                 if (SSE) acc += e;
@@ -646,9 +798,8 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                     a0 = fmaxf(a0, fabsf(y[i]));
                     a1 = fmaxf(a1, fabsf(y[16 + i]));
                 }
-                encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y, a0, nsc, cw[0], cw[1], sb0, xh, nullptr);
-                encode_nv16<FMT == kRZ, SSE ? kOutXh : kOutNone>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16,
-                                                                nullptr);
+                encode_nv16<FMT == kRZ, SSE>(y, a0, nsc, cw[0], cw[1], sb0, xh);
+                encode_nv16<FMT == kRZ, SSE>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16);
             }
             if (SSE) {
                 // the original values again, from the tile still in shared memory

@@ -81,6 +81,16 @@ __device__ __forceinline__ float2 sub2_rn(float2 a, float2 b)
     return r;
 }
 
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b)
+{
+    float2 r;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
 // a * b + c per lane, one rounding.
 __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c)
 {
@@ -106,6 +116,35 @@ __device__ __forceinline__ uint32_t e2m1x8(const float* v)
         "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return out;
+}
+
+// As e2m1x8, and e[i] = q_i - v[i] with q_i the grid value of nibble i (the
+// codes are decoded back to f16 and subtracted in one mixed-precision
+// rounding).  The difference is exact: q_i is the grid point nearest v[i],
+// or +-6 when |v[i]| > 6, so q_i - v[i] is a multiple of ulp(v[i]) and no
+// larger than max(|v[i]|, 1).
+__device__ __forceinline__ uint32_t e2m1x8_diff(const float* v, float* e)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+        ".reg .b16 l0, u0, l1, u1, l2, u2, l3, u3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %12, %11;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %14, %13;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %16, %15;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h0, b0;\n\tcvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, b2;\n\tcvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+        "mov.b32 {l0, u0}, h0;\n\tmov.b32 {l1, u1}, h1;\n\t"
+        "mov.b32 {l2, u2}, h2;\n\tmov.b32 {l3, u3}, h3;\n\t"
+        "sub.rn.f32.f16 %1, l0, %9;\n\tsub.rn.f32.f16 %2, u0, %10;\n\t"
+        "sub.rn.f32.f16 %3, l1, %11;\n\tsub.rn.f32.f16 %4, u1, %12;\n\t"
+        "sub.rn.f32.f16 %5, l2, %13;\n\tsub.rn.f32.f16 %6, u2, %14;\n\t"
+        "sub.rn.f32.f16 %7, l3, %15;\n\tsub.rn.f32.f16 %8, u3, %16;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out), "=f"(e[0]), "=f"(e[1]), "=f"(e[2]), "=f"(e[3]), "=f"(e[4]), "=f"(e[5]), "=f"(e[6]),
+          "=f"(e[7])
         : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return out;
 }

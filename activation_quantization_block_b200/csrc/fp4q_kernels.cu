@@ -122,8 +122,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_cons
         }
     }
     pdl_trigger();
-    __shared__ float den_tab[128], rcp_tab[128];
-    const NvScale nsc = nv_scale_setup(s_t, den_tab, rcp_tab);
+    __shared__ NvTable nvt;
+    const NvScale nsc = nv_scale_setup(s_t, &nvt);
 
     double acc = 0.0;
     for (int64_t j = 0; j < sc.mine; ++j) {
