@@ -318,7 +318,7 @@ def main():
     avg_call_bytes = BYTES_PER_ELEMENT * statistics.mean(call_elements)
     peak, peak_kind = peaks()
     achieved = avg_call_bytes / (avg_call_ms / 1e3) / 1e9
-    dram_bpe = traffic_record("quantize_nvfp4_razer_sse")
+    dram_bpe = traffic_record("quantize_batch_nvfp4_razer_sse" if args.mode == "batch" else "quantize_nvfp4_razer_sse")
     roofline = {"bound": "hbm", "kernel": kernel_desc,
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_kind": f"{peak_kind} copy bandwidth",
