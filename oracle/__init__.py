@@ -20,8 +20,8 @@ import subprocess
 
 import numpy as np
 
-NVFP4, NVFP4_RAZER, MXFP4 = 0, 1, 2
-FORMAT_NAMES = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4}
+NVFP4, NVFP4_RAZER, MXFP4, NVFP4_RAZER_W = 0, 1, 2, 3
+FORMAT_NAMES = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4, "nvfp4_razer_w": NVFP4_RAZER_W}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4q_oracle.c")
@@ -54,6 +54,11 @@ def lib() -> ctypes.CDLL:
         L.orc_e2m1_encode.argtypes = [f32]; L.orc_e2m1_encode.restype = i32
         L.orc_e4m3_value.argtypes = [i32]; L.orc_e4m3_value.restype = f64
         L.orc_e4m3_encode.argtypes = [f32]; L.orc_e4m3_encode.restype = i32
+        L.orc_e3m3_value.argtypes = [i32]; L.orc_e3m3_value.restype = f64
+        L.orc_e3m3_encode.argtypes = [f32]; L.orc_e3m3_encode.restype = i32
+        L.orc_set_razer_w_pair.argtypes = [f64]; L.orc_set_razer_w_pair.restype = None
+        L.orc_razer_w_pair.argtypes = []; L.orc_razer_w_pair.restype = f64
+        L.orc_tensor_scale_from_amax_w.argtypes = [f32]; L.orc_tensor_scale_from_amax_w.restype = f32
         L.orc_e8m0_value.argtypes = [i32]; L.orc_e8m0_value.restype = f64
         L.orc_mx_exponent.argtypes = [f32]; L.orc_mx_exponent.restype = i32
         L.orc_hadamard_entry.argtypes = [i32, i32]; L.orc_hadamard_entry.restype = i32
@@ -105,6 +110,24 @@ def e4m3_value(byte: int) -> float:
 
 def e4m3_encode(t: float) -> int:
     return lib().orc_e4m3_encode(float(t))
+
+
+def e3m3_value(byte6: int) -> float:
+    return lib().orc_e3m3_value(int(byte6))
+
+
+def e3m3_encode(t: float) -> int:
+    return lib().orc_e3m3_encode(float(t))
+
+
+def razer_w_pair() -> float:
+    """The second special-value pair (+-s2) of the RaZeR weight mode."""
+    return lib().orc_razer_w_pair()
+
+
+def set_razer_w_pair(s2: float) -> None:
+    """Change the weight mode's second pair (the offline search only)."""
+    lib().orc_set_razer_w_pair(float(s2))
 
 
 def e8m0_value(byte: int) -> float:
@@ -161,7 +184,9 @@ def tensor_amax(x: np.ndarray, rotate: bool = False, nthreads: int | None = None
                                  nthreads or default_threads())
 
 
-def tensor_scale_from_amax(amax: float) -> float:
+def tensor_scale_from_amax(amax: float, fmt="nvfp4") -> float:
+    if _fmt(fmt) == NVFP4_RAZER_W:
+        return lib().orc_tensor_scale_from_amax_w(float(amax))
     return lib().orc_tensor_scale_from_amax(float(amax))
 
 

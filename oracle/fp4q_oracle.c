@@ -37,6 +37,15 @@
  *     Sylvester-ordered +-1 Hadamard matrix; the sum is taken in double.
  *  R6 layout: codes row-major, element 2k in the low nibble of byte k; scales
  *     dense row-major [rows][cols / block].
+ *  R7 RaZeR weight mode [RaZeR sect. 2.1, 2.2: weights take a 6-bit E3M3 block
+ *     scale, and the two freed bits choose among four special values, two
+ *     pairs fixed offline, all multiples of 0.5]: E3M3 is unsigned, exponent
+ *     bias 3, exponent field 0 subnormal (m * 2^-5), no NaN, largest value 30;
+ *     the scale byte holds the E3M3 value in bits 0..5 and the selector in bits
+ *     6..7 (0: +5, 1: -5, 2: +s2, 3: -s2); the first level is
+ *     s_t = RN(A / (6 * 30)); per block the special value with the largest
+ *     squared-error gain wins, ties going to the lower selector; s2 is the
+ *     second pair found by the offline search in oracle/razer_weight_pair.py.
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC
  * -pthread.  Floating point is IEEE binary32/binary64 with round-to-nearest
@@ -51,6 +60,14 @@
 #define ORC_NVFP4 0
 #define ORC_NVFP4_RAZER 1
 #define ORC_MXFP4 2
+#define ORC_NVFP4_RAZER_W 3
+
+/* The second special-value pair of the RaZeR weight mode (R7): the winner of
+ * the offline search over multiples of 0.5 (oracle/razer_weight_pair.py).
+ * The search itself changes it through orc_set_razer_w_pair. */
+static double razer_w_pair = 2.5;
+void orc_set_razer_w_pair(double s2) { razer_w_pair = s2; }
+double orc_razer_w_pair(void) { return razer_w_pair; }
 
 /* ------------------------------------------------------------------------ */
 /* bf16 and fp32 bit helpers                                                 */
@@ -148,6 +165,44 @@ int orc_e4m3_encode(float t)
     int mant = (int)r, ex = k + 7;
     if (mant == 8) { mant = 0; ex += 1; }
     if (ex > 15 || (ex == 15 && mant > 6)) return 0x7E;
+    return (ex << 3) | mant;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E3M3 block scale of the RaZeR weight mode (R7)                             */
+/* ------------------------------------------------------------------------ */
+
+double orc_e3m3_value(int byte6)
+{
+    int e = (byte6 >> 3) & 7, m = byte6 & 7;
+    if (e == 0) return ldexp((double)m, -5);
+    return ldexp(1.0 + m / 8.0, e - 3);
+}
+
+/* Round a non-negative fp32 to E3M3: nearest, ties to even mantissa,
+ * saturating at 30 (0x3F).  As orc_e4m3_encode with bias 3. */
+int orc_e3m3_encode(float t)
+{
+    double x = (double)t;
+    if (!(x > 0.0)) return 0;
+    if (x >= 30.0) return 0x3F;
+    int k;
+    double f = frexp(x, &k);       /* x = f * 2^k, f in [0.5, 1) */
+    k -= 1;                        /* x = (2f) * 2^k, 2f in [1, 2) */
+    if (k < -2) {                  /* subnormal range: quantum 2^-5 */
+        double q = x / ldexp(1.0, -5);
+        double r = floor(q);
+        double frac = q - r;
+        if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+        return (int)r;             /* r in [0, 8]; 8 encodes the smallest normal */
+    }
+    double q = (2.0 * f - 1.0) * 8.0;
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    int mant = (int)r, ex = k + 3;
+    if (mant == 8) { mant = 0; ex += 1; }
+    if (ex > 7) return 0x3F;
     return (ex << 3) | mant;
 }
 
@@ -268,6 +323,14 @@ float orc_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx
  * largest E4M3 value (448). */
 float orc_tensor_scale_from_amax(float amax) { return amax / 2688.0f; }
 
+/* R7: the weight mode maps it onto 6 times the largest E3M3 value (30). */
+float orc_tensor_scale_from_amax_w(float amax) { return amax / 180.0f; }
+
+static float tensor_scale_for(int fmt, float amax)
+{
+    return fmt == ORC_NVFP4_RAZER_W ? orc_tensor_scale_from_amax_w(amax) : orc_tensor_scale_from_amax(amax);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Block decode: the fp32 reconstruction of one element                      */
 /* ------------------------------------------------------------------------ */
@@ -277,14 +340,27 @@ float orc_tensor_scale_from_amax(float amax) { return amax / 2688.0f; }
  * for +5 (scale bit 7 clear) or -5 (bit 7 set)  [RaZeR sect. 2.2]. */
 static float nv_den(int fmt, int sbyte, float s_t)
 {
-    double sv = orc_e4m3_value(fmt == ORC_NVFP4_RAZER ? (sbyte & 0x7F) : sbyte);
+    double sv = fmt == ORC_NVFP4_RAZER_W ? orc_e3m3_value(sbyte & 0x3F)
+                                         : orc_e4m3_value(fmt == ORC_NVFP4_RAZER ? (sbyte & 0x7F) : sbyte);
     return (float)sv * s_t;
+}
+
+/* The special value code 0b1000 stands for in a block with scale byte sbyte. */
+static double special_value(int fmt, int sbyte)
+{
+    if (fmt == ORC_NVFP4_RAZER) return (sbyte & 0x80) ? -5.0 : 5.0;
+    switch ((sbyte >> 6) & 3) {
+        case 0: return 5.0;
+        case 1: return -5.0;
+        case 2: return razer_w_pair;
+        default: return -razer_w_pair;
+    }
 }
 
 static float nv_decode(int fmt, int code, int sbyte, float den)
 {
     double q;
-    if (fmt == ORC_NVFP4_RAZER && code == 8) q = (sbyte & 0x80) ? -5.0 : 5.0;
+    if ((fmt == ORC_NVFP4_RAZER || fmt == ORC_NVFP4_RAZER_W) && code == 8) q = special_value(fmt, sbyte);
     else q = orc_e2m1_value(code);
     return (float)q * den;
 }
@@ -311,26 +387,30 @@ static int get_code(const uint8_t* row_codes, int64_t j)
     return (j & 1) ? (b >> 4) : (b & 0x0F);
 }
 
-/* RaZeR selection for one 16-block given the scaled values v[] and the
- * regular codes q[] (R4).  Squared errors are formed in double; every
- * difference involved is exact in binary32 and every square and sum of the
- * candidates is exact in binary64, so the comparison is exact.  Returns
- * 0 (use +5) or 1 (use -5) and rewrites the winning elements to 0b1000. */
-static int razer_select(const float* v, int* q, int n)
+/* RaZeR selection for one 16-block given the scaled values v[], the regular
+ * codes q[] and the candidate special values sv[0..ns) (R4, R7).  Squared
+ * errors are formed in double; every difference involved is exact in binary32
+ * and every square and sum of the candidates is exact in binary64, so the
+ * comparison is exact.  Returns the index of the candidate with the largest
+ * total gain (ties: the lower index) and rewrites its winning elements, those
+ * strictly closer to it than to their regular value, to 0b1000. */
+static int razer_select(const float* v, int* q, int n, const double* sv, int ns)
 {
-    double gain[2] = {0.0, 0.0};
-    const double special[2] = {5.0, -5.0};
-    for (int s = 0; s < 2; ++s)
+    double best = 0.0;
+    int pick = 0;
+    for (int s = 0; s < ns; ++s) {
+        double gain = 0.0;
         for (int i = 0; i < n; ++i) {
             double e_reg = (double)v[i] - orc_e2m1_value(q[i]);
-            double e_sp = (double)v[i] - special[s];
+            double e_sp = (double)v[i] - sv[s];
             if (fabs(e_sp) < fabs(e_reg))           /* strictly closer: remap */
-                gain[s] += e_reg * e_reg - e_sp * e_sp;
+                gain += e_reg * e_reg - e_sp * e_sp;
         }
-    int pick = gain[1] > gain[0] ? 1 : 0;           /* ties keep +5 */
+        if (s == 0 || gain > best) { best = gain; pick = s; }
+    }
     for (int i = 0; i < n; ++i) {
         double e_reg = (double)v[i] - orc_e2m1_value(q[i]);
-        double e_sp = (double)v[i] - special[pick];
+        double e_sp = (double)v[i] - sv[pick];
         if (fabs(e_sp) < fabs(e_reg)) q[i] = 8;
     }
     return pick;
@@ -360,18 +440,26 @@ static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
                 for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
             }
         } else {
-            /* RaZeR sect. 1 / R2: block scale from the block absmax */
+            /* RaZeR sect. 1 / R2: block scale from the block absmax (R7: E3M3
+             * for the weight mode) */
             float six_st = 6.0f * s_t;
             float t = (six_st > 0.0f) ? a / six_st : 0.0f;
-            sbyte = orc_e4m3_encode(t);
-            float den = (float)orc_e4m3_value(sbyte) * s_t;
+            const int wmode = fmt == ORC_NVFP4_RAZER_W;
+            sbyte = wmode ? orc_e3m3_encode(t) : orc_e4m3_encode(t);
+            float den = (float)(wmode ? orc_e3m3_value(sbyte) : orc_e4m3_value(sbyte)) * s_t;
             if (sbyte == 0 || den == 0.0f) {
                 /* a zero (or underflowed) scale decodes every element to 0 */
                 for (int i = 0; i < B; ++i) q[i] = 0;
             } else {
                 float r = 1.0f / den;
                 for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
-                if (fmt == ORC_NVFP4_RAZER && razer_select(v, q, B)) sbyte |= 0x80;
+                if (fmt == ORC_NVFP4_RAZER) {
+                    const double pair[2] = {5.0, -5.0};
+                    sbyte |= razer_select(v, q, B, pair, 2) << 7;
+                } else if (wmode) {
+                    const double four[4] = {5.0, -5.0, razer_w_pair, -razer_w_pair};
+                    sbyte |= razer_select(v, q, B, four, 4) << 6;
+                }
             }
         }
         row_scales[b0 / B] = (uint8_t)sbyte;
@@ -476,7 +564,7 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
     if (fmt != ORC_MXFP4) {
         if (scale_given) s_t = *tensor_scale;
         else {
-            s_t = orc_tensor_scale_from_amax(orc_tensor_amax(x, rows, cols, ldx, rotate, nthreads));
+            s_t = tensor_scale_for(fmt, orc_tensor_amax(x, rows, cols, ldx, rotate, nthreads));
             *tensor_scale = s_t;
         }
     }

@@ -43,8 +43,15 @@ def e4m3_from_bits(byte: int) -> float:
     return -mag if s else mag
 
 
+def e3m3_from_bits(byte6: int) -> float:
+    """E3M3 (6 bits, unsigned): bias 3, exponent 0 subnormal, no NaN."""
+    e, m = (byte6 >> 3) & 7, byte6 & 7
+    return m * 2.0 ** -5 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 3)
+
+
 E2M1 = [e2m1_from_bits(c) for c in range(16)]
 E4M3_POS = [e4m3_from_bits(b) for b in range(0x7F)]  # 0x00 .. 0x7E, increasing
+E3M3 = [e3m3_from_bits(b) for b in range(64)]        # increasing
 
 
 def e2m1_nearest(v: float) -> int:
@@ -69,6 +76,40 @@ def e4m3_nearest(t: float) -> int:
         if best is None or key < best[0]:
             best = (key, b)
     return best[1]
+
+
+def e3m3_nearest(t: float) -> int:
+    """Argmin over the 64 E3M3 values; ties to the even byte."""
+    best = None
+    ft = Fraction(t)
+    for b, val in enumerate(E3M3):
+        key = (abs(ft - Fraction(val)), b & 1)
+        if best is None or key < best[0]:
+            best = (key, b)
+    return best[1]
+
+
+def razer_pick(v, q, specials):
+    """Exact per-block special-value choice: for each candidate, elements strictly
+    closer to it than to their regular value move to it; the candidate with the
+    lowest total squared error wins (ties: the earlier candidate).  Returns
+    (index, codes)."""
+    best = None
+    for idx, sv in enumerate(specials):
+        tot = Fraction(0)
+        ch = []
+        for vi, qi in zip(v, q):
+            er = (Fraction(float(vi)) - Fraction(E2M1[qi])) ** 2
+            es = (Fraction(float(vi)) - Fraction(sv)) ** 2
+            if es < er:
+                tot += es
+                ch.append(8)
+            else:
+                tot += er
+                ch.append(qi)
+        if best is None or tot < best[0]:
+            best = (tot, idx, ch)
+    return best[1], best[2]
 
 
 def floor_log2(a: float) -> int:
@@ -115,9 +156,10 @@ def unpack_codes(codes: np.ndarray, cols: int) -> np.ndarray:
     return out
 
 
-def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool):
+def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool, pair2: float = 2.5):
     """Quantize by enumeration: every scale byte and every element code is the
-    argmin of its own exhaustive search; rotation sums are exact rationals."""
+    argmin of its own exhaustive search; rotation sums are exact rationals.
+    ``pair2``: the second special-value pair of the weight mode."""
     x = bits_to_f32(xbits).astype(np.float32)
     rows, cols = x.shape
     y = x.copy()
@@ -134,9 +176,10 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool):
     codes = np.zeros((rows, cols), dtype=np.int64)
     scales = np.zeros((rows, cols // B), dtype=np.int64)
     ts = np.float32(0)
+    wmode = fmt == "nvfp4_razer_w"
     if fmt != "mxfp4":
         A = np.float32(np.max(np.abs(y))) if y.size else np.float32(0)
-        ts = np.float32(A / np.float32(2688))
+        ts = np.float32(A / np.float32(180 if wmode else 2688))
     for r in range(rows):
         for b in range(cols // B):
             blk = y[r, b * B:(b + 1) * B]
@@ -150,8 +193,8 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool):
             else:
                 six = np.float32(np.float32(6) * ts)
                 t = np.float32(a / six) if six > 0 else np.float32(0)
-                sb = e4m3_nearest(float(t))
-                den = np.float32(np.float32(E4M3_POS[sb]) * ts)
+                sb = e3m3_nearest(float(t)) if wmode else e4m3_nearest(float(t))
+                den = np.float32(np.float32(E3M3[sb] if wmode else E4M3_POS[sb]) * ts)
                 scales[r, b] = sb
                 if sb == 0 or den == 0:
                     continue
@@ -159,32 +202,18 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool):
                 v = [np.float32(val * rr) for val in blk]
             q = [e2m1_nearest(float(vi)) for vi in v]
             if fmt == "nvfp4_razer":
-                sse = {}
-                choice = {}
-                for sv in (5.0, -5.0):
-                    tot = Fraction(0)
-                    ch = []
-                    for vi, qi in zip(v, q):
-                        er = (Fraction(float(vi)) - Fraction(E2M1[qi])) ** 2
-                        es = (Fraction(float(vi)) - Fraction(sv)) ** 2
-                        if es < er:
-                            tot += es
-                            ch.append(8)
-                        else:
-                            tot += er
-                            ch.append(qi)
-                    sse[sv], choice[sv] = tot, ch
-                pick = -5.0 if sse[-5.0] < sse[5.0] else 5.0
-                q = choice[pick]
-                if pick < 0:
-                    scales[r, b] |= 0x80
+                idx, q = razer_pick(v, q, (5.0, -5.0))
+                scales[r, b] |= idx << 7
+            elif wmode:
+                idx, q = razer_pick(v, q, (5.0, -5.0, pair2, -pair2))
+                scales[r, b] |= idx << 6
             codes[r, b * B:(b + 1) * B] = q
     packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
     return packed, scales.astype(np.uint8), ts
 
 
 def dequantize_bruteforce(codes: np.ndarray, scales: np.ndarray, ts: float, fmt: str,
-                          rotate: bool) -> np.ndarray:
+                          rotate: bool, pair2: float = 2.5) -> np.ndarray:
     """fp32 reconstruction from the bit-field definitions (exact rationals for rotation)."""
     rows, cols = codes.shape[0], codes.shape[1] * 2
     nib = unpack_codes(codes, cols)
@@ -197,11 +226,15 @@ def dequantize_bruteforce(codes: np.ndarray, scales: np.ndarray, ts: float, fmt:
             if fmt == "mxfp4":
                 out[r, j] = np.float32(E2M1[code] * 2.0 ** (sb - 127))
             else:
-                mag = sb & 0x7F if fmt == "nvfp4_razer" else sb
-                sval = e4m3_from_bits(mag)
+                if fmt == "nvfp4_razer_w":
+                    sval = e3m3_from_bits(sb & 0x3F)
+                else:
+                    sval = e4m3_from_bits(sb & 0x7F if fmt == "nvfp4_razer" else sb)
                 den = np.float32(np.float32(sval) * np.float32(ts))
                 if fmt == "nvfp4_razer" and code == 8:
                     qv = -5.0 if sb & 0x80 else 5.0
+                elif fmt == "nvfp4_razer_w" and code == 8:
+                    qv = (5.0, -5.0, pair2, -pair2)[(sb >> 6) & 3]
                 else:
                     qv = E2M1[code]
                 out[r, j] = np.float32(np.float32(qv) * den)

@@ -243,22 +243,22 @@ def _tiny_inputs():
     return [a.astype(ml_dtypes.bfloat16).view(np.uint16) for a in out]
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_quantize_equals_bruteforce(orc, fmt, rotate):
     for xb in _tiny_inputs():
         codes, scales, ts, sse = orc.quantize(xb, fmt, rotate)
-        bcodes, bscales, bts = bf.quantize_bruteforce(xb, fmt, rotate)
+        bcodes, bscales, bts = bf.quantize_bruteforce(xb, fmt, rotate, pair2=orc.razer_w_pair())
         assert np.array_equal(codes, bcodes)
         assert np.array_equal(scales, bscales)
         if fmt != "mxfp4":
             assert ts == bts
-        xhat = bf.dequantize_bruteforce(bcodes, bscales, bts, fmt, rotate)
+        xhat = bf.dequantize_bruteforce(bcodes, bscales, bts, fmt, rotate, pair2=orc.razer_w_pair())
         exact = bf.sse_exact(xb, xhat)
         assert abs(sse - float(exact)) <= 1e-12 * max(1.0, float(exact))
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_dequantize_equals_bruteforce(orc, fmt, rotate):
     import torch
@@ -267,7 +267,7 @@ def test_dequantize_equals_bruteforce(orc, fmt, rotate):
     codes, scales = codes.numpy(), scales.numpy()
     ts = float(ts[0]) * 2.0 ** -6
     y32, y16 = orc.dequantize(codes, scales, ts, fmt, rotate)
-    want = bf.dequantize_bruteforce(codes, scales, ts, fmt, rotate)
+    want = bf.dequantize_bruteforce(codes, scales, ts, fmt, rotate, pair2=orc.razer_w_pair())
     assert np.array_equal(y32.view(np.uint32), want.view(np.uint32))
     assert np.array_equal(y16, want.astype(ml_dtypes.bfloat16).view(np.uint16))
     del torch
@@ -409,3 +409,97 @@ def test_rotation_spreads_mxfp4_code_occupancy(orc):
     z1 = (bf.unpack_codes(c1, 512) & 7 == 0).mean()
     assert z1 < z0          # rotation leaves fewer elements quantized to zero
     assert sse1 < sse0
+
+
+# ---------------------------------------------------------------- RaZeR weight mode (E3M3 scale, four specials)
+
+def test_e3m3_decode(orc):
+    """64 values: the normal ones are exactly the E4M3 values (ml_dtypes) whose
+    exponent field is 4 higher (same 3-bit mantissa, bias 3 instead of 7), the
+    subnormal ones the multiples of 2^-5 below the smallest normal 0.25."""
+    vals = [orc.e3m3_value(b) for b in range(64)]
+    assert vals == [bf.e3m3_from_bits(b) for b in range(64)]
+    e4 = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    for b in range(64):
+        e, m = b >> 3, b & 7
+        if e:
+            assert vals[b] == e4[((e + 4) << 3) | m]
+        else:
+            assert vals[b] == m * 2.0 ** -5
+    assert vals[0x3F] == 30.0 and vals[8] == 0.25 and vals[1] == 2.0 ** -5
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+
+
+def test_e3m3_encode_equals_exhaustive_argmin(orc):
+    vals = sorted(set(bf.E3M3))
+    probes = [0.0, 1e-9, 40.0, 30.0, 31.0, 1e30]
+    for a, b in zip(vals, vals[1:]):
+        mid = np.float32((a + b) / 2)
+        probes += [a, b, float(mid), float(np.nextafter(mid, np.float32(0))), float(np.nextafter(mid, np.float32(99)))]
+    for t in probes:
+        assert orc.e3m3_encode(np.float32(t)) == bf.e3m3_nearest(min(float(np.float32(t)), 30.0)), t
+
+
+def test_weight_mode_tensor_scale_maps_amax_to_6x30(orc):
+    for k in range(-20, 20):
+        assert orc.tensor_scale_from_amax(180.0 * 2.0 ** k, "nvfp4_razer_w") == np.float32(2.0 ** k)
+    assert orc.tensor_scale_from_amax(1.0, "nvfp4_razer_w") == np.float32(1.0) / np.float32(180.0)
+
+
+def test_weight_mode_worked_blocks(orc):
+    """[6d, 2.5d, 0...] is lossless with the second pair (selector 2, or 3 for the
+    negated block); [6d, 5d, 0...] with the first (selector 0 / 1)."""
+    d = 2.0 ** -4        # with A = 6d, s_t = A / 180, so the block scale is 30 (E3M3 0x3F)
+    for special, sel in ((orc.razer_w_pair(), 2), (5.0, 0)):
+        x = np.zeros((1, 16), np.float32); x[0, 0] = 6 * d; x[0, 3] = special * d
+        for sign, s_sel in ((1.0, sel), (-1.0, sel + 1)):
+            xb = (sign * x).astype(ml_dtypes.bfloat16).view(np.uint16)
+            codes, scales, ts, sse = orc.quantize(xb, "nvfp4_razer_w")
+            assert ts == np.float32(6 * d / 180.0)
+            assert scales[0, 0] == (s_sel << 6) | 0x3F
+            assert bf.unpack_codes(codes, 16)[0, 3] == 8 and sse == 0.0
+            y32, _ = orc.dequantize(codes, scales, ts, "nvfp4_razer_w")
+            assert np.array_equal(y32, (sign * x).astype(np.float32))
+
+
+def test_weight_mode_invariants_on_random_blocks(orc):
+    """Against NVFP4 with the same (E3M3-rounded) block scales, the weight mode
+    only moves elements to code 0b1000 and never raises a block's error."""
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.llm_weight(64, 256, seed=22))
+    x = bf.bits_to_f32(xb).astype(np.float64)
+    c_w, s_w, ts, _ = orc.quantize(xb, "nvfp4_razer_w", nthreads=2)
+    y_w, _ = orc.dequantize(c_w, s_w, ts, "nvfp4_razer_w")
+    n_w = bf.unpack_codes(c_w, 256)
+    sels = (s_w >> 6) & 3
+    assert {0, 1, 2, 3} <= set(np.unique(sels).tolist())
+    # the same scales with every special code read as its regular E2M1 neighbour:
+    # plain rounding of the scaled values, block by block
+    for r in range(8):
+        for b in range(16):
+            sb = int(s_w[r, b]) & 0x3F
+            den = np.float32(np.float32(bf.E3M3[sb]) * ts)
+            rr = np.float32(np.float32(1) / den)
+            blk = x[r, 16 * b:16 * b + 16].astype(np.float32)
+            v = [np.float32(val * rr) for val in blk]
+            q = [bf.e2m1_nearest(float(vi)) for vi in v]
+            got = n_w[r, 16 * b:16 * b + 16]
+            assert all(g == qi or g == 8 for g, qi in zip(got, q))
+            plain = float(((blk.astype(np.float64) - np.array([bf.E2M1[qi] for qi in q]) * float(den)) ** 2).sum())
+            mine = float(((blk.astype(np.float64) - y_w[r, 16 * b:16 * b + 16]) ** 2).sum())
+            assert mine <= plain * (1 + 1e-6)
+
+
+def test_weight_mode_second_pair_wins_a_reduced_search(orc):
+    """The second pair is the minimum of the offline search; a smaller sample of
+    the same synthetic weights gives the same winner."""
+    from oracle import razer_weight_pair
+    from activation_quantization_block_b200 import synthetic
+    mats = [synthetic.bf16_bits(synthetic.llm_weight(256, 2048, seed=300 + k, device="cpu")) for k in range(2)]
+    keep = orc.razer_w_pair()
+    try:
+        table = {s2: razer_weight_pair.total_sse(mats, s2) for s2 in razer_weight_pair.CANDIDATES}
+    finally:
+        orc.set_razer_w_pair(keep)
+    assert min(table, key=table.get) == keep == 2.5
+    assert all(keep % 0.5 == 0 for keep in table)
