@@ -44,7 +44,10 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int block_len(int fmt) { return fmt == FP4Q_MXFP4 ? 32 : 16; }
 
-bool valid_format(int fmt) { return fmt == FP4Q_NVFP4 || fmt == FP4Q_NVFP4_RAZER || fmt == FP4Q_MXFP4; }
+bool valid_format(int fmt)
+{
+    return fmt == FP4Q_NVFP4 || fmt == FP4Q_NVFP4_RAZER || fmt == FP4Q_MXFP4 || fmt == FP4Q_NVFP4_RAZER_W;
+}
 
 // Shape checks shared by every entry point.
 fp4q_status_t check_shape(int64_t rows, int64_t cols, int fmt, int rotate)

@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 3)
             float mx = 0.0f;
             for (int i = t; i < a.n_amax_in; i += kThreads) mx = fmaxf(mx, a.amax_in[i]);
             mx = block_max(mx, shf);
-            s_t = __fdiv_rn(mx, 2688.0f);
+            s_t = tensor_scale_of<FMT>(mx);
             if (b == 0 && t == 0) *a.tensor_scale = s_t;
         } else {
             s_t = *a.tensor_scale;
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
     pdl_trigger();
     NvScale nsc{};
-    if (a.has_q && FMT != kMX) nsc = nv_scale_setup(s_t, &nvt);
+    if (a.has_q && FMT != kMX) nsc = nv_scale_setup<FMT>(s_t, &nvt);
     // The first items, written by thread 0, are visible after this barrier; a
     // refill's item is written before thread 0 arms its stage, and the
     // consumers' acquire of the landed phase makes it visible.
@@ -208,6 +208,10 @@ cudaError_t chain_dispatch(int fmt, bool rotate, bool sse, const CUtensorMap& qm
         case 9: return chain_go<kMX, false, true>(qmap, amap, a, tiles, pdl, grid_out, st);
         case 10: return chain_go<kMX, true, false>(qmap, amap, a, tiles, pdl, grid_out, st);
         case 11: return chain_go<kMX, true, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 12: return chain_go<kRW, false, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 13: return chain_go<kRW, false, true>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 14: return chain_go<kRW, true, false>(qmap, amap, a, tiles, pdl, grid_out, st);
+        case 15: return chain_go<kRW, true, true>(qmap, amap, a, tiles, pdl, grid_out, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -6,7 +6,8 @@
 //  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant Zero
 //   Remapping": sect. 1 (E2M1 set, E4M3 block scale from the block absmax,
 //   unused scale sign bit), sect. 2.2 (-0 code remapped to a special value
-//   chosen per block by minimum squared error; one bit -> the pair +-5).
+//   chosen per block by minimum squared error; one bit -> the pair +-5;
+//   weights: a 6-bit E3M3 block scale and two bits -> four special values).
 //  "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization": sect. 1
 //   (32-element blocks, shared exponent, e2m1 codebook), sect. 2 (orthogonal
 //   intra-block rotation before quantization).
@@ -24,7 +25,22 @@
 
 namespace fp4q {
 
-enum { kNV = 0, kRZ = 1, kMX = 2 };
+// Formats, numbered as the C ABI's: NVFP4, RaZeR (activation mode: +-5),
+// MXFP4, RaZeR weight mode (E3M3 scale, +-5 and +-2.5).
+enum { kNV = 0, kRZ = 1, kMX = 2, kRW = 3 };
+
+template <int FMT> constexpr bool kRazer = FMT == kRZ || FMT == kRW;
+
+// The second special-value pair of the weight mode.
+constexpr float kRazerWPair = 2.5f;
+
+// s_t = RN(A / (6 * largest block-scale value)): 6 * 448 for the E4M3 scale,
+// 6 * 30 for the weight mode's E3M3 scale.
+template <int FMT>
+__device__ __forceinline__ float tensor_scale_of(float amax)
+{
+    return __fdiv_rn(amax, FMT == kRW ? 180.0f : 2688.0f);
+}
 
 // Device error word of a translation unit (bits: kErrPipelineTimeout); each
 // unit that launches kernels reads and clears its own copy for the C ABI.
@@ -221,7 +237,8 @@ __device__ __forceinline__ void decode16(uint32_t w0, uint32_t w1, float* q)
 }
 
 // Per-tensor constants of the NVFP4 block-scale step, shared by a CTA: for
-// each of the 127 non-negative finite E4M3 bytes b, den[b] = RN(dec(b) * s_t),
+// each of the 127 non-negative finite E4M3 bytes b (the 64 E3M3 codes in the
+// weight mode), den[b] = RN(dec(b) * s_t),
 // rcp[b] = RN(1 / den[b]) (0 when den[b] = 0: a zero scale zeroes every code)
 // and den[b]^2 (exact in binary64).  The quotient t = RN(a / RN(6 s_t)) uses
 // inv6 = RN(1 / RN(6 s_t)) and one correction step (Markstein's theorem: with
@@ -240,6 +257,7 @@ struct NvScale {
     uint32_t tab;         // shared address of the CTA's NvTable
 };
 
+template <int FMT>
 __device__ __forceinline__ NvScale nv_scale_setup(float s_t, NvTable* tab)
 {
     NvScale c;
@@ -248,7 +266,9 @@ __device__ __forceinline__ NvScale nv_scale_setup(float s_t, NvTable* tab)
     c.exact_div = !(c.six_st >= 0x1p-64f && c.six_st <= 0x1p64f);
     c.inv6 = c.exact_div ? 0.0f : __frcp_rn(c.six_st);
     for (int b = threadIdx.x; b < 128; b += blockDim.x) {
-        const float d = b < 127 ? __fmul_rn(e4m3_to_f32((uint32_t)b), s_t) : 0.0f;
+        float d = 0.0f;
+        if (FMT == kRW) d = b < 64 ? __fmul_rn(e3m3_to_f32((uint32_t)b), s_t) : 0.0f;
+        else d = b < 127 ? __fmul_rn(e4m3_to_f32((uint32_t)b), s_t) : 0.0f;
         tab->dr[b] = make_float2(d, d != 0.0f ? __frcp_rn(d) : 0.0f);
         tab->den2[b] = (double)d * (double)d;
     }
@@ -257,7 +277,7 @@ __device__ __forceinline__ NvScale nv_scale_setup(float s_t, NvTable* tab)
     return c;
 }
 
-// {den, rcp} of scale byte sb (bit 7 clear).
+// {den, rcp} of the unsigned scale code sb.
 __device__ __forceinline__ float2 nv_den_rcp(const NvScale& c, uint32_t sb)
 {
     float2 v;
@@ -265,7 +285,7 @@ __device__ __forceinline__ float2 nv_den_rcp(const NvScale& c, uint32_t sb)
     return v;
 }
 
-// den^2 of scale byte sb (bit 7 clear).
+// den^2 of the unsigned scale code sb.
 __device__ __forceinline__ double nv_den2(const NvScale& c, uint32_t sb)
 {
     double v;
@@ -280,6 +300,36 @@ __device__ __forceinline__ float nv_block_ratio(const NvScale& c, float a)
     const float q = __fmul_rn(a, c.inv6);
     const float r = __fmaf_rn(-q, c.six_st, a);
     return __fmaf_rn(r, c.inv6, q);
+}
+
+// Unsigned block-scale code of a block with absmax a: E4M3, or E3M3 in the
+// weight mode, of t = RN(a / RN(6 s_t)), nearest even, saturating.
+template <int FMT>
+__device__ __forceinline__ uint32_t nv_scale_code(const NvScale& c, float a)
+{
+    const float t = nv_block_ratio(c, a);
+    return FMT == kRW ? e3m3_rn_sat(t) : e4m3_rn_satfinite(t);
+}
+
+// Decoded block scale of scale byte sb (its selector bits ignored).
+template <int FMT>
+__device__ __forceinline__ float nv_scale_value(uint32_t sb)
+{
+    if (FMT == kRW) return e3m3_to_f32(sb & 0x3Fu);
+    return e4m3_to_f32(FMT == kRZ ? (sb & 0x7Fu) : sb);
+}
+
+// The special value code 0b1000 stands for in a block with scale byte sb:
+// activation mode +5, or -5 with bit 7 set; weight mode, by bits 6..7,
+// +5, -5, +2.5, -2.5.
+template <int FMT>
+__device__ __forceinline__ float razer_special(uint32_t sb)
+{
+    if (FMT == kRW) {
+        const float m = (sb & 0x80u) ? kRazerWPair : 5.0f;
+        return (sb & 0x40u) ? -m : m;
+    }
+    return (sb & 0x80u) ? -5.0f : 5.0f;
 }
 
 // RaZeR remap of one block given cs[i] = sign(v_i) * gain_i, the signed gains
@@ -330,14 +380,99 @@ __device__ __forceinline__ void razer_tent(const float* v, uint32_t& w0, uint32_
     razer_apply(cs, sp[0].x + sp[0].y, w0, w1, sb);
 }
 
+// Weight-mode remap of one block (candidates +5, -5, +2.5, -2.5 = selectors
+// 0..3) given c5[i] = sign(v_i) * gain of remapping element i to
+// sign(v_i) * 5 and c2[i] likewise for 2.5, U5, U2 the sums of the gains and
+// S5, S2 the sums of the signed gains.  For either pair the better member's
+// gain is (U + |S|) / 2; these sums are exact (gains of 5 are multiples of
+// 2^-20 up to 1, of 2.5 multiples of 2^-22 up to 1/4), so the comparisons
+// are.  The pair 2.5 is taken only when its gain is strictly larger, and in
+// a pair the negative member only when its gain is strictly larger: ties go
+// to the lower selector.  Winners are flagged as in razer_apply, the gains of
+// the pair not taken multiplied by 0 (a candidate for one pair never is for
+// the other).  Returns the chosen gain.
+__device__ __forceinline__ float razer_w_apply(const float* c5, const float* c2, float U5, float S5, float U2,
+                                               float S2, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+{
+    const float t5 = U5 + fabsf(S5), t2 = U2 + fabsf(S2);
+    const bool p2 = t2 > t5;
+    const bool neg = (p2 ? S2 : S5) < 0.0f;
+    const float sk = neg ? -0x1p40f : 0x1p40f;
+    const float k5 = p2 ? 0.0f : sk, k2 = p2 ? sk : 0.0f;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float2 p = fma2_rn(make_float2(c2[i], c2[i + 1]), make_float2(k2, k2),
+                                 mul2_rn(make_float2(c5[i], c5[i + 1]), make_float2(k5, k5)));
+        x[i] = p.x;
+        x[i + 1] = p.y;
+    }
+    const uint32_t k0 = e2m1x8(x), k1 = e2m1x8(x + 8);
+    const uint32_t f0 = k0 & ~(k0 >> 3) & 0x11111111u;
+    const uint32_t f1 = k1 & ~(k1 >> 3) & 0x11111111u;
+    w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
+    w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
+    sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
+    return 0.5f * fmaxf(t5, t2);
+}
+
+// Gain of remapping |v| to 2.5: its regular value is 2 (|v| <= 2.5) or 3,
+// and (|v| - q)^2 - (|v| - 2.5)^2 = 1/4 - | |v| - 2.5 |, positive exactly on
+// (2.25, 2.75) and clamped to 0 elsewhere; |v| - 2.5 is exact there, so the
+// gain is a multiple of 2^-22.
+__device__ __forceinline__ float razer_gain_w2(float v)
+{
+    return __saturatef(0.25f - fabsf(fabsf(v) - kRazerWPair));
+}
+
+// Weight-mode selection from the scaled values alone (any magnitude).
+__device__ __forceinline__ void razer_w_tent(const float* v, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+{
+    float c5[16], c2[16];
+    float2 u5[8], s5[8], u2[8], s2[8];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float a0 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
+        const float a1 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i + 1]) - 5.0f), 1.0f));
+        const float b0 = razer_gain_w2(v[i]), b1 = razer_gain_w2(v[i + 1]);
+        c5[i] = copysignf(a0, v[i]);
+        c5[i + 1] = copysignf(a1, v[i + 1]);
+        c2[i] = copysignf(b0, v[i]);
+        c2[i + 1] = copysignf(b1, v[i + 1]);
+        u5[i / 2] = make_float2(a0, a1);
+        u2[i / 2] = make_float2(b0, b1);
+        s5[i / 2] = make_float2(c5[i], c5[i + 1]);
+        s2[i / 2] = make_float2(c2[i], c2[i + 1]);
+    }
+#pragma unroll
+    for (int k = 4; k > 0; k >>= 1)
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+            u5[i] = add2_rn(u5[i], u5[i + k]);
+            s5[i] = add2_rn(s5[i], s5[i + k]);
+            u2[i] = add2_rn(u2[i], u2[i + k]);
+            s2[i] = add2_rn(s2[i], s2[i + k]);
+        }
+    razer_w_apply(c5, c2, u5[0].x + u5[0].y, s5[0].x + s5[0].y, u2[0].x + u2[0].y, s2[0].x + s2[0].y, w0, w1, sb);
+}
+
+// Selection from the scaled values for either RaZeR mode.
+template <int FMT>
+__device__ __forceinline__ void razer_from_v(const float* v, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+{
+    if (FMT == kRW) razer_w_tent(v, w0, w1, sb);
+    else razer_tent(v, w0, w1, sb);
+}
+
 // One 16-element NVFP4 / RaZeR block of values y (rotated ones, on the rotated
 // path) with absmax a: two code words and the scale byte and, when XH, the
-// fp32 reconstruction xh = RN(q den) (RaZeR winners: RN(+-5 den)).
-template <bool RAZER, bool XH>
+// fp32 reconstruction xh = RN(q den) (RaZeR winners: RN(special * den)).
+template <int FMT, bool XH>
 __device__ __forceinline__ void encode_nv16(const float* y, float a, const NvScale& sc, uint32_t& c0, uint32_t& c1,
                                             uint32_t& sb_out, float* xh)
 {
-    uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
+    constexpr bool RAZER = kRazer<FMT>;
+    uint32_t sb = nv_scale_code<FMT>(sc, a);
     const float2 dr = nv_den_rcp(sc, sb);
     const float den = dr.x, r = dr.y;
     float v[16];
@@ -349,11 +484,11 @@ __device__ __forceinline__ void encode_nv16(const float* y, float a, const NvSca
     }
     uint32_t w0 = canonical_zero(e2m1x8(v));
     uint32_t w1 = canonical_zero(e2m1x8(v + 8));
-    if (RAZER) razer_tent(v, w0, w1, sb);
+    if (RAZER) razer_from_v<FMT>(v, w0, w1, sb);
     if (XH) {
         float q[16];
         decode16(w0, w1, q);
-        const float special = (sb & 0x80u) ? -5.0f : 5.0f;
+        const float special = razer_special<FMT>(sb);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
             float q0 = q[i], q1 = q[i + 1];
@@ -386,9 +521,10 @@ struct BlockOut {
 // y - RN(q den) taken in fp32 (zero when the element is reproduced) and
 // squared and summed in fp64.  Taken for the rare blocks the fast path below
 // does not cover.
-template <bool RAZER>
+template <int FMT>
 __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32_t sb, float den, float r)
 {
+    constexpr bool RAZER = kRazer<FMT>;
     uint32_t w[8];
     const uint4 c0 = lds128(a0), c1 = lds128(a1);
     w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
@@ -405,10 +541,10 @@ __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32
     o.w0 = canonical_zero(e2m1x8(v));
     o.w1 = canonical_zero(e2m1x8(v + 8));
     o.sb = sb;
-    if (RAZER) razer_tent(v, o.w0, o.w1, o.sb);
+    if (RAZER) razer_from_v<FMT>(v, o.w0, o.w1, o.sb);
     float q[16];
     decode16(o.w0, o.w1, q);
-    const float special = (o.sb & 0x80u) ? -5.0f : 5.0f;
+    const float special = razer_special<FMT>(o.sb);
     double s = 0.0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -431,7 +567,8 @@ __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32
 // total gain of the RaZeR winners (0 for NVFP4).  For a candidate (|v| in
 // (4.5, 5.5), q = +-4 or +-6) the gain 1 - 2||v| - 5| equals 2|e| - 1, and
 // sat(2|e| - 1) is 0 for every other element as long as |v| <= 6.5, so gains,
-// decision and G come from e with no further per-element work.  den v differs
+// decision and G come from e with no further per-element work (the weight
+// mode's gains of 2.5 come from v, see razer_gain_w2).  den v differs
 // from y by at most 2^-23 |y| (two roundings), the only departure from the
 // exact error besides fp32 rounding of the sum.
 //
@@ -440,14 +577,15 @@ __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32
 // far below the block absmax), a fast sum below 2^-30 (the block is reproduced
 // exactly or almost, and the exact sum keeps a zero error zero), or one that
 // is not finite (an infinite reciprocal).
-template <bool RAZER, bool SSE>
+template <int FMT, bool SSE>
 __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_t a1, const NvScale& sc,
                                          uint32_t& c0, uint32_t& c1, uint32_t& sb_out, double& sse)
 {
+    constexpr bool RAZER = kRazer<FMT>;
     const uint32_t mm = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
                                       bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
     const float a = bf16x2_hmax_abs(mm);
-    uint32_t sb = e4m3_rn_satfinite(nv_block_ratio(sc, a));
+    uint32_t sb = nv_scale_code<FMT>(sc, a);
     const float2 dr = nv_den_rcp(sc, sb);
     float v[16];
     {
@@ -462,7 +600,7 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
     }
     if (!SSE) {
         uint32_t w0 = canonical_zero(e2m1x8(v)), w1 = canonical_zero(e2m1x8(v + 8));
-        if (RAZER) razer_tent(v, w0, w1, sb);
+        if (RAZER) razer_from_v<FMT>(v, w0, w1, sb);
         c0 = w0;
         c1 = w1;
         sb_out = sb;
@@ -481,7 +619,35 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
     w0 = canonical_zero(w0);
     w1 = canonical_zero(w1);
     const uint32_t sb0 = sb;
-    if (RAZER) {
+    if (FMT == kRW) {
+        float c5[16], c2[16];
+        float2 u5[8], s5[8], u2[8], s2[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float g0 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i]), -1.0f));
+            const float g1 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i + 1]), -1.0f));
+            const float h0 = razer_gain_w2(v[i]), h1 = razer_gain_w2(v[i + 1]);
+            c5[i] = copysignf(g0, v[i]);
+            c5[i + 1] = copysignf(g1, v[i + 1]);
+            c2[i] = copysignf(h0, v[i]);
+            c2[i + 1] = copysignf(h1, v[i + 1]);
+            u5[i / 2] = make_float2(g0, g1);
+            u2[i / 2] = make_float2(h0, h1);
+            s5[i / 2] = make_float2(c5[i], c5[i + 1]);
+            s2[i / 2] = make_float2(c2[i], c2[i + 1]);
+        }
+#pragma unroll
+        for (int k = 4; k > 0; k >>= 1)
+#pragma unroll
+            for (int i = 0; i < k; ++i) {
+                u5[i] = add2_rn(u5[i], u5[i + k]);
+                s5[i] = add2_rn(s5[i], s5[i + k]);
+                u2[i] = add2_rn(u2[i], u2[i + k]);
+                s2[i] = add2_rn(s2[i], s2[i + k]);
+            }
+        sv -= razer_w_apply(c5, c2, u5[0].x + u5[0].y, s5[0].x + s5[0].y, u2[0].x + u2[0].y, s2[0].x + s2[0].y, w0,
+                            w1, sb);
+    } else if (RAZER) {
         float cs[16];
         float2 gp[8], sp[8];
 #pragma unroll
@@ -512,7 +678,7 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
         sb_out = sb;
         sse = (double)sv * nv_den2(sc, sb0);
     } else {
-        const BlockOut o = nv_block_exact<RAZER>(a0, a1, sb0, dr.x, dr.y);
+        const BlockOut o = nv_block_exact<FMT>(a0, a1, sb0, dr.x, dr.y);
         c0 = o.w0;
         c1 = o.w1;
         sb_out = o.sb;
@@ -561,11 +727,12 @@ __device__ __forceinline__ void encode_mx32(const float* y, float a, uint32_t* c
 // Decoders (dequantize and error)
 // ---------------------------------------------------------------------------
 
-template <bool RAZER>
+template <int FMT>
 __device__ __forceinline__ void decode_nv16(uint32_t w0, uint32_t w1, uint32_t sb, float s_t, float* xh)
 {
-    const float den = __fmul_rn(e4m3_to_f32(RAZER ? (sb & 0x7Fu) : sb), s_t);
-    const float special = (sb & 0x80u) ? -5.0f : 5.0f;
+    constexpr bool RAZER = kRazer<FMT>;
+    const float den = __fmul_rn(nv_scale_value<FMT>(sb), s_t);
+    const float special = razer_special<FMT>(sb);
     float q[16];
     decode16(w0, w1, q);
     if (RAZER) {
@@ -603,8 +770,8 @@ __device__ __forceinline__ void decode_unit(const uint32_t* cw, const uint32_t* 
     if (FMT == kMX) {
         decode_mx32(cw, sb[0], xh);
     } else {
-        decode_nv16<FMT == kRZ>(cw[0], cw[1], sb[0], s_t, xh);
-        decode_nv16<FMT == kRZ>(cw[2], cw[3], sb[1], s_t, xh + 16);
+        decode_nv16<FMT>(cw[0], cw[1], sb[0], s_t, xh);
+        decode_nv16<FMT>(cw[2], cw[3], sb[1], s_t, xh + 16);
     }
 }
 
@@ -772,7 +939,7 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                 w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
                 uint32_t sbh;
                 double e = 0.0;
-                nv_block<FMT == kRZ, SSE>(w, a0, a1, nsc, cw[2 * half], cw[2 * half + 1], sbh, e);
+                nv_block<FMT, SSE>(w, a0, a1, nsc, cw[2 * half], cw[2 * half + 1], sbh, e);
                 if (half == 0) sb0 = sbh;
                 else sb1 = sbh;
                 if (SSE) acc += e;
@@ -798,8 +965,8 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                     a0 = fmaxf(a0, fabsf(y[i]));
                     a1 = fmaxf(a1, fabsf(y[16 + i]));
                 }
-                encode_nv16<FMT == kRZ, SSE>(y, a0, nsc, cw[0], cw[1], sb0, xh);
-                encode_nv16<FMT == kRZ, SSE>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16);
+                encode_nv16<FMT, SSE>(y, a0, nsc, cw[0], cw[1], sb0, xh);
+                encode_nv16<FMT, SSE>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16);
             }
             if (SSE) {
                 // the original values again, from the tile still in shared memory

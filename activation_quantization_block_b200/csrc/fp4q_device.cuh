@@ -2,7 +2,8 @@
 //
 // Number formats follow "RaZeR: Pushing the Limits of NVFP4 Quantization with
 // Redundant Zero Remapping" (technical summary sect. 1: E2M1 elements
-// {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit, FP8-E4M3 block scale) and
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit, FP8-E4M3 block scale; sect.
+// 2.1 and 2.2: the 6-bit E3M3 block scale of its weight mode) and
 // "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization" (sect. 1:
 // 32-element blocks with a shared power-of-two scale).  Conversions use the
 // hardware cvt instructions of sm_100a: E2M1 and E4M3 encoding round to
@@ -203,6 +204,30 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte)
     uint16_t in = (uint16_t)(byte & 0xFFu);
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(in));
     return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+}
+
+// ---- E3M3 (block scale of the RaZeR weight mode) ---------------------------
+//
+// Unsigned; exponent field e (3 bits, bias 3) and mantissa m (3 bits):
+// (1 + m/8) 2^(e-3) for e > 0, m 2^-5 for e = 0; largest value 30 (0x3F).
+
+// Non-negative finite fp32 -> E3M3 code, nearest even, saturating at 30.  From
+// 0.25 (the smallest normal) up to 30, E3M3 and E4M3 have the same values and
+// the same 3-bit mantissa, so the E4M3 conversion of min(t, 30) is the E3M3
+// code with 4 added to the exponent field; below 0.25 the quantum is 2^-5
+// throughout and the code is RN_even(32 t), in [0, 8] (8 encodes 0.25).
+__device__ __forceinline__ uint32_t e3m3_rn_sat(float t)
+{
+    const uint32_t lo = (uint32_t)__float2int_rn(t * 32.0f);
+    const uint32_t hi = e4m3_rn_satfinite(fminf(t, 30.0f)) - 32u;
+    return t < 0.25f ? lo : hi;
+}
+
+// E3M3 code (6 bits) -> fp32, exact.
+__device__ __forceinline__ float e3m3_to_f32(uint32_t c)
+{
+    const uint32_t e = (c >> 3) & 7u, m = c & 7u;
+    return e == 0u ? (float)m * 0x1p-5f : __uint_as_float(((e + 124u) << 23) | (m << 20));
 }
 
 // ---- E8M0 -----------------------------------------------------------------

@@ -22,7 +22,8 @@
 //  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant Zero
 //   Remapping": sect. 1 (E2M1 set, E4M3 block scale from the block absmax,
 //   unused scale sign bit), sect. 2.2 (-0 code remapped to a special value
-//   chosen per block by minimum squared error; one bit -> the pair +-5).
+//   chosen per block by minimum squared error; one bit -> the pair +-5;
+//   weights: a 6-bit E3M3 block scale and two bits -> four special values).
 //  "TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization": sect. 1
 //   (32-element blocks, shared exponent, e2m1 codebook), sect. 2 (orthogonal
 //   intra-block rotation before quantization).
@@ -108,7 +109,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_cons
         for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT>(p, &xmap, a.tl, sc, j);
     pdl_wait();
 
-    // Tensor scale (NVFP4 formats): s_t = RN(A / (6 * 448)) from the absmax partials.
+    // Tensor scale (NVFP4 formats): s_t = RN(A / (6 * 448)), or RN(A / (6 * 30))
+    // in the weight mode, from the absmax partials.
     float s_t = 0.0f;
     if (FMT != kMX) {
         if (a.scale_given) {
@@ -117,13 +119,13 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_cons
             float m = 0.0f;
             for (int i = t; i < a.n_amax; i += kThreads) m = fmaxf(m, a.amax_partials[i]);
             m = block_max(m, shf);
-            s_t = __fdiv_rn(m, 2688.0f);
+            s_t = tensor_scale_of<FMT>(m);
             if (blockIdx.x == 0 && t == 0) *a.tensor_scale = s_t;
         }
     }
     pdl_trigger();
     __shared__ NvTable nvt;
-    const NvScale nsc = nv_scale_setup(s_t, &nvt);
+    const NvScale nsc = nv_scale_setup<FMT>(s_t, &nvt);
 
     double acc = 0.0;
     for (int64_t j = 0; j < sc.mine; ++j) {
@@ -361,6 +363,8 @@ cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int r
         case 3: return quantize_dispatch<kRZ, true>(map, a, sse, after_amax, grid_out, st);
         case 4: return quantize_dispatch<kMX, false>(map, a, sse, after_amax, grid_out, st);
         case 5: return quantize_dispatch<kMX, true>(map, a, sse, after_amax, grid_out, st);
+        case 6: return quantize_dispatch<kRW, false>(map, a, sse, after_amax, grid_out, st);
+        case 7: return quantize_dispatch<kRW, true>(map, a, sse, after_amax, grid_out, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -393,6 +397,8 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
         case 3: return dequantize_dispatch<kRZ, true>(map, a, st);
         case 4: return dequantize_dispatch<kMX, false>(map, a, st);
         case 5: return dequantize_dispatch<kMX, true>(map, a, st);
+        case 6: return dequantize_dispatch<kRW, false>(map, a, st);
+        case 7: return dequantize_dispatch<kRW, true>(map, a, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -426,6 +432,8 @@ cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t*
         case 3: return error_dispatch<kRZ, true>(map, a, grid_out, st);
         case 4: return error_dispatch<kMX, false>(map, a, grid_out, st);
         case 5: return error_dispatch<kMX, true>(map, a, grid_out, st);
+        case 6: return error_dispatch<kRW, false>(map, a, grid_out, st);
+        case 7: return error_dispatch<kRW, true>(map, a, grid_out, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -17,8 +17,8 @@ import torch
 
 from . import _build
 
-NVFP4, NVFP4_RAZER, MXFP4 = 0, 1, 2
-FORMATS = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4}
+NVFP4, NVFP4_RAZER, MXFP4, NVFP4_RAZER_W = 0, 1, 2, 3
+FORMATS = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4, "nvfp4_razer_w": NVFP4_RAZER_W}
 FLAG_TENSOR_SCALE_GIVEN = 0x1
 
 SUCCESS = 0

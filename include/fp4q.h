@@ -36,6 +36,19 @@
  *                    with e = clamp(floor(log2 amax_b) - 2, -127, 127);
  *                    element code = nearest E2M1 to x * 2^-e (exact scaling).
  *                    No tensor scale.
+ *  FP4Q_NVFP4_RAZER_W  RaZeR weight mode (RaZeR sect. 2.1, 2.2): 16-element
+ *                    blocks with a 6-bit unsigned E3M3 block scale (exponent
+ *                    bias 3, exponent field 0 subnormal = m * 2^-5, largest
+ *                    value 30) in bits 0..5 of the scale byte; bits 6..7 hold
+ *                    the selector of the special value code 0b1000 stands
+ *                    for: 0 -> +5, 1 -> -5, 2 -> +2.5, 3 -> -2.5 (the second
+ *                    pair fixed offline by an error search over multiples of
+ *                    0.5 on synthetic weights).  s_t = RN(amax / (6 * 30));
+ *                    block scale E3M3_RNE_sat(RN(amax_b / RN(6 s_t))); codes
+ *                    as NVFP4; per block the candidate with the largest
+ *                    squared-error gain is chosen (ties: the lower selector)
+ *                    and every element strictly closer to it than to its
+ *                    regular value becomes 0b1000.
  *
  * rotate = 1 applies, before quantization, the orthonormal 32-point
  * Walsh-Hadamard transform y = RN(RN(H32 x) * RN(1/sqrt 32)) to every aligned
@@ -49,7 +62,8 @@
  * Layouts (all dense, row-major, caller-allocated, 16-byte aligned):
  *  x, y      bf16 [rows][ld], ld >= cols, ld a multiple of 8 elements.
  *  codes     uint8 [rows][cols/2]; element 2k in the low nibble of byte k.
- *  scales    uint8 [rows][cols/16] (NVFP4, NVFP4_RAZER) or [rows][cols/32] (MXFP4).
+ *  scales    uint8 [rows][cols/16] (NVFP4, NVFP4_RAZER, NVFP4_RAZER_W) or
+ *            [rows][cols/32] (MXFP4).
  *  tensor_scale  one fp32 (NVFP4 formats; may be NULL for MXFP4).
  *  mse       one fp64: sum over all elements of (x - x^)^2 / (rows*cols),
  *            x^ the fp32 reconstruction (before any bf16 rounding) in the
@@ -81,7 +95,7 @@
 extern "C" {
 #endif
 
-#define FP4Q_ABI_VERSION 1
+#define FP4Q_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FP4Q_API __attribute__((visibility("default")))
@@ -92,7 +106,8 @@ extern "C" {
 typedef enum {
     FP4Q_NVFP4 = 0,
     FP4Q_NVFP4_RAZER = 1,
-    FP4Q_MXFP4 = 2
+    FP4Q_MXFP4 = 2,
+    FP4Q_NVFP4_RAZER_W = 3
 } fp4q_format_t;
 
 typedef enum {

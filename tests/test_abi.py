@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_status_strings_workspace():
-    assert fp4q.fp4q_abi_version() == 1
+    assert fp4q.fp4q_abi_version() == 2
     for code in range(7):
         assert fp4q.fp4q_status_string(code)
     assert fp4q.fp4q_status_string(99) == "unknown status"
@@ -51,8 +51,10 @@ def q(**kw):
 
 
 @pytest.mark.parametrize("kw,expect", [
-    (dict(fmt=3), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(fmt=4), "FP4Q_ERROR_INVALID_VALUE"),
     (dict(fmt=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(fmt=3, cols=40, ldx=40), "FP4Q_ERROR_SHAPE"),          # weight mode: blocks of 16
+    (dict(fmt=3, tensor_scale=None), "FP4Q_ERROR_INVALID_VALUE"),  # weight mode needs it
     (dict(rotate=2), "FP4Q_ERROR_INVALID_VALUE"),
     (dict(flags=2), "FP4Q_ERROR_INVALID_VALUE"),
     (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
@@ -86,6 +88,7 @@ def test_quantize_argument_rules_that_relax():
         pytest.skip("these calls would launch on a real device")
     assert q(fmt=2, tensor_scale=None) in ok_then_device
     assert q(flags=1, workspace=None, workspace_bytes=0) in ok_then_device
+    assert q(fmt=3, cols=48, ldx=48) in ok_then_device           # weight mode: 16-element blocks
 
 
 def _no_gpu() -> bool:

@@ -51,7 +51,7 @@ def _compare(got, want, xs):
         assert a == b or abs(a - b) <= 1e-12 * abs(b)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_batch_equals_per_tensor_calls(dev, fmt, rotate):
     xs = _mixed_tensors(dev, fmt, rotate)
@@ -62,7 +62,7 @@ def test_batch_equals_per_tensor_calls(dev, fmt, rotate):
     assert fp4q.fp4q_device_errors()[1] == 0
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "nvfp4_razer_w"])
 def test_batch_with_given_scales(dev, fmt):
     xs = _mixed_tensors(dev, fmt, False, seed=50)
     scales = [torch.tensor([s], dtype=torch.float32, device=dev) for s in np.geomspace(1e-6, 1e-2, len(xs))]

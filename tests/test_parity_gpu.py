@@ -20,7 +20,8 @@ from activation_quantization_block_b200 import fp4q, synthetic
 
 pytestmark = pytest.mark.gpu
 
-FMTS = ["nvfp4", "nvfp4_razer", "mxfp4"]
+FMTS = ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"]
+NV_FMTS = ["nvfp4", "nvfp4_razer", "nvfp4_razer_w"]
 
 
 @pytest.fixture(scope="module")
@@ -158,7 +159,7 @@ def check_dequant_rotated(orc, codes, scales, ts, rows, cols, fmt, dev):
 def test_weight_2048_nvfp4_and_razer(orc, dev):
     """2048 x 2048 LLM weight, N(0, 0.02^2) with 0.1 % outliers x20, seed 0."""
     x = synthetic.llm_weight(2048, 2048, seed=0, device="cpu").to(dev)
-    for fmt in ("nvfp4", "nvfp4_razer"):
+    for fmt in NV_FMTS:
         check_exact(orc, x, fmt)
 
 
@@ -173,7 +174,7 @@ def test_activation_t3_mxfp4(orc, dev, rotate):
         check_exact(orc, x, "mxfp4")
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
+@pytest.mark.parametrize("fmt", NV_FMTS)
 def test_nvfp4_rotated(orc, dev, fmt):
     x = synthetic.activation_t3(512, 1024, seed=5, device="cpu").to(dev)
     codes, scales, ts = check_rotated(orc, x, fmt)
@@ -216,7 +217,7 @@ def test_small_and_ragged_shapes(orc, dev, fmt, shape):
     check_exact(orc, x, fmt)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
+@pytest.mark.parametrize("fmt", NV_FMTS)
 @pytest.mark.parametrize("shape", [(1, 16), (3, 16), (5, 48), (9, 80), (1, 4112)])
 def test_half_unit_shapes(orc, dev, fmt, shape):
     """cols % 32 == 16: units straddle rows and the last unit is a single block."""
@@ -267,7 +268,7 @@ def test_extreme_magnitudes(orc, dev, fmt):
     check_exact(orc, _bf(mixed).to(dev), fmt)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
+@pytest.mark.parametrize("fmt", NV_FMTS)
 def test_tensor_scale_given(orc, dev, fmt):
     x = synthetic.llm_weight(64, 256, seed=10, device="cpu").to(dev)
     for ts in (1.0, 3.0e-5, 2.0 ** -12, 0.0):
@@ -312,6 +313,57 @@ def test_razer_both_signs_tie_breaks(orc, dev):
     check_exact(orc, _bf(np.array(rows)).to(dev), "nvfp4_razer")
 
 
+def test_razer_weight_worked_blocks_on_gpu(orc, dev):
+    """RaZeR weight mode: a block at the largest E3M3 scale holding 6, and 2.5 or
+    5 of either sign, is reproduced exactly with the selector of that value."""
+    d = 30 * 2.0 ** -6                       # den = 30 * s_t with s_t = 2^-6
+    for special, sel in ((5.0, 0), (-5.0, 1), (2.5, 2), (-2.5, 3)):
+        x = np.zeros((1, 16), np.float32)
+        x[0, 0], x[0, 1] = 6 * d, special * d
+        codes, scales, ts, mse = check_exact(orc, _bf(x).to(dev), "nvfp4_razer_w", tensor_scale=2.0 ** -6)
+        assert scales[0, 0] == (sel << 6) | 0x3F and (codes[0, 0] >> 4) == 8 and mse == 0.0
+
+
+def test_razer_weight_candidates_and_ties(orc, dev):
+    """Blocks with candidates of all four special values (gains of 5 and of 2.5
+    equal, larger or smaller; both signs; exact ties go to the lower selector)."""
+    rng = np.random.default_rng(21)
+    d = 2.0 ** -3                            # block max 6 d: E3M3 16 (0x38), den = 16 * 2^-7
+    rows = []
+    for _ in range(512):
+        v = rng.choice([0.0, 0.5, -1.0, 1.5, 3.0, -4.0], size=16)
+        v[0] = 6.0
+        pos = rng.permutation(np.arange(1, 16))
+        n5, n2 = rng.integers(0, 4, size=2)
+        m5 = rng.choice([4.625, 4.75, 4.875, 5.0, 5.125, 5.25, 5.375], size=n5)
+        m2 = rng.choice([2.3125, 2.375, 2.4375, 2.5, 2.5625, 2.625, 2.6875], size=n2)
+        v[pos[:n5]] = m5 * rng.choice([-1, 1], size=n5)
+        v[pos[n5:n5 + n2]] = m2 * rng.choice([-1, 1], size=n2)
+        rows.append(v * d)
+    x = _bf(np.array(rows)).to(dev)
+    codes, scales, _, _ = check_exact(orc, x, "nvfp4_razer_w", tensor_scale=2.0 ** -7)
+    assert np.all(scales & 0x3F == 0x38)
+    assert len(np.unique(scales >> 6)) == 4          # every selector occurs
+
+
+def test_razer_weight_small_block_scales(orc, dev):
+    """Blocks far below the tensor maximum: E3M3 subnormal scales (m * 2^-5),
+    the boundary to the smallest normal (0.25) and the rounding ties there."""
+    rng = np.random.default_rng(22)
+    rows = rng.standard_normal((64, 256)) * 0.02
+    rows[0, 0] = 30.0                                 # tensor maximum
+    # block absmaxes a_b = t * 6 s_t for t near k * 2^-5 and 0.25
+    s_t = np.float32(30.0) / np.float32(180.0)
+    ts = np.concatenate([np.arange(1, 10) * 2.0 ** -5, np.arange(1, 10) * 2.0 ** -5 + 2.0 ** -6,
+                         [0.2421875, 0.25, 0.2578125, 0.234375, 0.4 * 2.0 ** -5, 0.6 * 2.0 ** -5]])
+    for i, t in enumerate(ts):
+        r, b = 1 + i // 16, i % 16
+        blk = rng.standard_normal(16) * 0.1 * t * 6 * s_t
+        blk[rng.integers(16)] = t * 6 * s_t
+        rows[r, 16 * b:16 * b + 16] = blk
+    check_exact(orc, _bf(rows).to(dev), "nvfp4_razer_w")
+
+
 def test_empty_tensor(dev):
     x = torch.empty(0, 64, dtype=torch.bfloat16, device=dev)
     q = fp4q.quantize(x, "nvfp4_razer")
@@ -335,7 +387,7 @@ def _sampled_rows_check(orc, x: torch.Tensor, fmt, nrows=64, seed=0):
         amax = 0.0
         for r0 in range(0, rows, 4096):   # bounded host copies
             amax = max(amax, orc.tensor_amax(bits(x[r0:r0 + 4096])))
-        ts = orc.tensor_scale_from_amax(amax)
+        ts = orc.tensor_scale_from_amax(amax, fmt)
         assert q.tensor_scale.item() == np.float32(ts)
     rc, rs, _, _ = orc.quantize(xs, fmt, False, tensor_scale=ts, want_sse=False)
     idx = torch.from_numpy(pick).to(x.device)

@@ -27,7 +27,7 @@ def _outputs(x, fmt):
             torch.full((1,), -1.0, dtype=torch.float64, device=d))
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
 @pytest.mark.parametrize("rotate", [0, 1])
 def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(fmt, rotate):
     if not torch.cuda.is_available():
