@@ -40,6 +40,14 @@ WORKLOAD = ("llama3-8b weight set: 32 layers x {q 4096x4096, k 1024x4096, v 1024
             "NVFP4_RAZER, rotate 0, per-tensor computed scale, fused MSE")
 
 
+def set_format(fmt: str):
+    """Run the same workload in another NVFP4 format (the default is the headline's)."""
+    global FMT, WORKLOAD
+    if fmt != FMT:
+        WORKLOAD = WORKLOAD.replace(FMT.upper(), fmt.upper())
+        FMT = fmt
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -50,6 +58,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--fmt", choices=["nvfp4_razer", "nvfp4", "nvfp4_razer_w"], default=FMT,
+                   help="format of the run (all three read 4.5625 B/element with the computed tensor scale)")
     p.add_argument("--mode", choices=["batch", "per-call"], default="batch",
                    help="batch: fp4q_quantize_batch over 16 layers (112 tensors) per call; "
                         "per-call: one fp4q_quantize per tensor")
@@ -212,6 +222,7 @@ def run_reference(args):
 
 def main():
     args = parse()
+    set_format(args.fmt)
     if args.impl == "reference":
         return run_reference(args)
 
@@ -318,7 +329,7 @@ def main():
     avg_call_bytes = BYTES_PER_ELEMENT * statistics.mean(call_elements)
     peak, peak_kind = peaks()
     achieved = avg_call_bytes / (avg_call_ms / 1e3) / 1e9
-    dram_bpe = traffic_record("quantize_batch_nvfp4_razer_sse" if args.mode == "batch" else "quantize_nvfp4_razer_sse")
+    dram_bpe = traffic_record(f"quantize_batch_{FMT}_sse" if args.mode == "batch" else f"quantize_{FMT}_sse")
     roofline = {"bound": "hbm", "kernel": kernel_desc,
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_kind": f"{peak_kind} copy bandwidth",
