@@ -72,6 +72,12 @@ def lib() -> ctypes.CDLL:
         L.orc_dequantize.restype = i32
         L.orc_error.argtypes = [vp, i64, vp, vp, f32, i64, i64, i32, i32, vp, i32]
         L.orc_error.restype = i32
+        L.orc_mma_planes.argtypes = [i32]; L.orc_mma_planes.restype = i32
+        L.orc_mma_sf_bytes.argtypes = [i64, i64]; L.orc_mma_sf_bytes.restype = i64
+        L.orc_mma_sf_offset.argtypes = [i64, i64, i64]; L.orc_mma_sf_offset.restype = i64
+        L.orc_mma_scale_byte.argtypes = [i32, i32]; L.orc_mma_scale_byte.restype = i32
+        L.orc_mma_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp]; L.orc_mma_pack.restype = i32
+        L.orc_gemm.argtypes = [vp, vp, i64, i64, i64, vp, vp, i32]; L.orc_gemm.restype = i32
     return _lib
 
 
@@ -246,3 +252,49 @@ def error(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, tensor_scale: fl
     if rc != 0:
         raise ValueError("oracle rejected shape")
     return float(sse[0])
+
+
+# ---------------------------------------------------------------- tensor-core operand form, W4A4 product
+
+def mma_planes(fmt) -> int:
+    """Code planes of a format's tensor-core operand form (1 for NVFP4, 2 for RaZeR)."""
+    return lib().orc_mma_planes(_fmt(fmt))
+
+
+def mma_sf_bytes(rows: int, cols: int) -> int:
+    return lib().orc_mma_sf_bytes(int(rows), int(cols))
+
+
+def mma_sf_offset(r: int, kb: int, cols: int) -> int:
+    return lib().orc_mma_sf_offset(int(r), int(kb), int(cols))
+
+
+def mma_scale_byte(fmt, sbyte: int) -> int:
+    return lib().orc_mma_scale_byte(_fmt(fmt), int(sbyte))
+
+
+def mma_pack(codes: np.ndarray, scales: np.ndarray, fmt):
+    """Return ``(planes, sf)``: planes uint8 [rows][planes * cols/2], sf uint8 [mma_sf_bytes]."""
+    f = _fmt(fmt)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    np_ = mma_planes(f)
+    planes = np.empty((rows, np_ * cols // 2), dtype=np.uint8)
+    sf = np.empty(mma_sf_bytes(rows, cols), dtype=np.uint8)
+    if lib().orc_mma_pack(_ptr(codes), _ptr(scales), rows, cols, f, _ptr(planes), _ptr(sf)) != 0:
+        raise ValueError("oracle rejected format or shape")
+    return planes, sf
+
+
+def gemm(a: np.ndarray, w: np.ndarray, nthreads: int | None = None):
+    """Return ``(y, yabs)``: y = a w^T and yabs = |a| |w|^T in binary64 (a: M x K, w: N x K fp32)."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    (M, K), (N, K2) = a.shape, w.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    y = np.empty((M, N), dtype=np.float64)
+    yabs = np.empty((M, N), dtype=np.float64)
+    lib().orc_gemm(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(yabs), nthreads or default_threads())
+    return y, yabs

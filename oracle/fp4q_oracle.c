@@ -46,6 +46,22 @@
  *     s_t = RN(A / (6 * 30)); per block the special value with the largest
  *     squared-error gain wins, ties going to the lower selector; s2 is the
  *     second pair found by the offline search in oracle/razer_weight_pair.py.
+ *  R8 tensor-core operand form [RaZeR sect. 2.3: GEMMs on existing tensor
+ *     cores handle the remapped code with two passes]: a quantized matrix
+ *     becomes one code plane (NVFP4) or two (RaZeR, either mode) whose decoded
+ *     sum is the reconstruction.  Plane 0 keeps every code except 0b1000, which
+ *     becomes the special value's base b, the largest E2M1 magnitude below
+ *     |s|, with the sign of s; plane 1 is +0 except at those elements, where it
+ *     holds s - b (+-1 for +-5, +-0.5 for +-2.5).  Both planes use the block's
+ *     scale magnitude as an E4M3 byte with bit 7 clear (weight mode: the E3M3
+ *     value, which every E3M3 code has exactly in E4M3).  Plane p of row r
+ *     occupies bytes [p * cols/2, (p+1) * cols/2) of the row.  The scale
+ *     bytes are stored in 512-byte atoms, one per 128 rows x 4 blocks: rows
+ *     padded to a multiple of 128 and blocks to a multiple of 4 with zeros,
+ *     atom (r / 128, kb / 4) in row-major order, and inside it the byte
+ *     (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
+ *  R9 W4A4 product: Y = A^ W^T for A^ (M x K) and W^ (N x K) the fp32
+ *     reconstructions of two quantized matrices, summed in binary64.
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC
  * -pthread.  Floating point is IEEE binary32/binary64 with round-to-nearest
@@ -640,5 +656,113 @@ int orc_error(const uint16_t* x, int64_t ldx, const uint8_t* codes, const uint8_
     proto.x = x; proto.ldx = ldx; proto.cols = cols; proto.fmt = fmt; proto.rotate = rotate;
     proto.s_t = tensor_scale; proto.ccodes = codes; proto.cscales = scales;
     *sse = run_rows(error_worker, proto, rows, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tensor-core operand form (R8) and the W4A4 product (R9)                   */
+/* ------------------------------------------------------------------------ */
+
+int orc_mma_planes(int fmt) { return (fmt == ORC_NVFP4_RAZER || fmt == ORC_NVFP4_RAZER_W) ? 2 : 1; }
+
+int64_t orc_mma_sf_bytes(int64_t rows, int64_t cols)
+{
+    return ((rows + 127) / 128) * ((cols / 16 + 3) / 4) * 512;
+}
+
+int64_t orc_mma_sf_offset(int64_t r, int64_t kb, int64_t cols)
+{
+    const int64_t atoms_per_row_block = (cols / 16 + 3) / 4;
+    return ((r / 128) * atoms_per_row_block + kb / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4;
+}
+
+/* The block's scale magnitude as an E4M3 byte (bit 7 clear). */
+int orc_mma_scale_byte(int fmt, int sbyte)
+{
+    if (fmt == ORC_NVFP4_RAZER_W) return orc_e4m3_encode((float)orc_e3m3_value(sbyte & 0x3F));
+    if (fmt == ORC_NVFP4_RAZER) return sbyte & 0x7F;
+    return sbyte;
+}
+
+/* Base of a special value s: the largest E2M1 magnitude below |s|, signed as s. */
+static double special_base(double s)
+{
+    double b = 0.0;
+    for (int c = 0; c < 8; ++c) {
+        const double m = orc_e2m1_value(c);
+        if (m < fabs(s) && m > b) b = m;
+    }
+    return s < 0.0 ? -b : b;
+}
+
+/* Codes (dense, rows x cols/2) and scales (rows x cols/16) of an NVFP4-family
+ * matrix -> planes (rows x planes*cols/2) and scale atoms (orc_mma_sf_bytes). */
+int orc_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, int fmt,
+                 uint8_t* planes, uint8_t* sf)
+{
+    if (fmt == ORC_MXFP4 || rows < 0 || cols % 16) return -1;
+    const int np = orc_mma_planes(fmt);
+    const int64_t half = cols / 2, nb = cols / 16;
+    memset(sf, 0, (size_t)orc_mma_sf_bytes(rows, cols));
+    memset(planes, 0, (size_t)(rows * np * half));
+    for (int64_t r = 0; r < rows; ++r) {
+        uint8_t* prow = planes + r * np * half;
+        for (int64_t j = 0; j < cols; ++j) {
+            const int code = get_code(codes + r * half, j);
+            const int sbyte = scales[r * nb + j / 16];
+            int c0 = code, c1 = 0;
+            if (np == 2 && code == 8) {
+                const double s = special_value(fmt, sbyte);
+                const double b = special_base(s);
+                c0 = orc_e2m1_encode((float)b);
+                c1 = orc_e2m1_encode((float)(s - b));
+            }
+            set_code(prow, j, c0);
+            if (np == 2) set_code(prow + half, j, c1);
+        }
+        for (int64_t kb = 0; kb < nb; ++kb)
+            sf[orc_mma_sf_offset(r, kb, cols)] = (uint8_t)orc_mma_scale_byte(fmt, scales[r * nb + kb]);
+    }
+    return 0;
+}
+
+typedef struct {
+    const float *a, *w;
+    int64_t m0, m1, N, K;
+    double *y, *yabs;
+} gemm_job;
+
+static void* gemm_worker(void* p)
+{
+    gemm_job* j = (gemm_job*)p;
+    for (int64_t m = j->m0; m < j->m1; ++m)
+        for (int64_t n = 0; n < j->N; ++n) {
+            double s = 0.0, t = 0.0;
+            for (int64_t k = 0; k < j->K; ++k) {
+                const double prod = (double)j->a[m * j->K + k] * (double)j->w[n * j->K + k];
+                s += prod;
+                t += fabs(prod);
+            }
+            j->y[m * j->N + n] = s;
+            if (j->yabs) j->yabs[m * j->N + n] = t;
+        }
+    return NULL;
+}
+
+/* R9: y = a w^T (a: M x K, w: N x K, row-major fp32), and yabs = |a| |w|^T. */
+int orc_gemm(const float* a, const float* w, int64_t M, int64_t N, int64_t K, double* y, double* yabs,
+             int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0) return -1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > M) nthreads = M > 0 ? (int)M : 1;
+    gemm_job* jobs = (gemm_job*)calloc((size_t)nthreads, sizeof(gemm_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = (gemm_job){a, w, M * t / nthreads, M * (t + 1) / nthreads, N, K, y, yabs};
+        pthread_create(&th[t], NULL, gemm_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(jobs); free(th);
     return 0;
 }

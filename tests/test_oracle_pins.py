@@ -503,3 +503,107 @@ def test_weight_mode_second_pair_wins_a_reduced_search(orc):
         orc.set_razer_w_pair(keep)
     assert min(table, key=table.get) == keep == 2.5
     assert all(keep % 0.5 == 0 for keep in table)
+
+
+# ---------------------------------------------------------------- tensor-core operand form and W4A4 product
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "nvfp4_razer_w"])
+def test_mma_planes_sum_to_the_reconstruction(orc, fmt):
+    """Decoded with the brute-force E2M1 table, the planes' values add up exactly to
+    the element's value (special values included), and with the atom's scale and
+    the tensor scale, rounded as a reconstruction is, give the brute-force
+    dequantizer's value."""
+    from activation_quantization_block_b200 import synthetic
+    rows, cols = 40, 96
+    xb = synthetic.bf16_bits(synthetic.llm_weight(rows, cols, seed=41))
+    codes, scales, ts, _ = orc.quantize(xb, fmt, nthreads=2)
+    planes, sf = orc.mma_pack(codes, scales, fmt)
+    np_ = orc.mma_planes(fmt)
+    assert np_ == (1 if fmt == "nvfp4" else 2) and planes.shape == (rows, np_ * cols // 2)
+    ref = bf.dequantize_bruteforce(codes, scales, float(ts), fmt, False)
+    n_special = 0
+    for r in range(rows):
+        q0 = bf.unpack_codes(planes[r:r + 1, :cols // 2], cols)[0]
+        q1 = bf.unpack_codes(planes[r:r + 1, cols // 2:], cols)[0] if np_ == 2 else np.zeros(cols, int)
+        for j in range(cols):
+            byte = int(sf[orc.mma_sf_offset(r, j // 16, cols)])
+            assert byte < 0x7F                                   # an E4M3 magnitude, bit 7 clear
+            q = Fraction(bf.E2M1[q0[j]]) + Fraction(bf.E2M1[q1[j]])
+            den = np.float32(np.float32(bf.e4m3_from_bits(byte)) * np.float32(ts))
+            assert np.float32(np.float32(float(q)) * den) == ref[r][j]
+            orig = bf.unpack_codes(codes[r:r + 1], cols)[0][j]
+            if np_ == 2 and orig == 8:
+                sb = int(scales[r, j // 16])
+                s = ((-5.0 if sb & 0x80 else 5.0) if fmt == "nvfp4_razer"
+                     else (5.0, -5.0, 2.5, -2.5)[(sb >> 6) & 3])
+                assert q == Fraction(s)
+                n_special += 1
+            else:
+                assert q == Fraction(bf.E2M1[orig]) and q1[j] == 0
+    if fmt != "nvfp4":
+        assert n_special > 0
+
+
+def test_mma_plane_split_of_each_special_value(orc):
+    """The split of every special value: base = the largest E2M1 magnitude below it."""
+    for fmt, sbyte, s in (("nvfp4_razer", 0x38, 5.0), ("nvfp4_razer", 0xB8, -5.0),
+                          ("nvfp4_razer_w", 0x00 | 0x20, 5.0), ("nvfp4_razer_w", 0x40 | 0x20, -5.0),
+                          ("nvfp4_razer_w", 0x80 | 0x20, 2.5), ("nvfp4_razer_w", 0xC0 | 0x20, -2.5)):
+        codes = np.full((1, 8), 0x08, np.uint8)                 # element 0 special, element 1 zero
+        scales = np.full((1, 1), sbyte, np.uint8)
+        planes, _ = orc.mma_pack(codes, scales, fmt)
+        b = math.copysign(4.0 if abs(s) == 5.0 else 2.0, s)
+        assert bf.E2M1[planes[0, 0] & 15] == b and bf.E2M1[planes[0, 8] & 15] == s - b
+        assert bf.E2M1[planes[0, 0] >> 4] == 0 and bf.E2M1[planes[0, 8] >> 4] == 0
+
+
+def test_mma_scale_bytes_are_exact_e4m3(orc):
+    """Every E3M3 value is an E4M3 value; activation-mode scales lose only bit 7."""
+    for c in range(64):
+        b = orc.mma_scale_byte("nvfp4_razer_w", c | 0xC0)
+        assert float(np.array([b], np.uint8).view(ml_dtypes.float8_e4m3fn)[0]) == bf.E3M3[c]
+    for b in range(0x7F):
+        assert orc.mma_scale_byte("nvfp4_razer", b | 0x80) == b == orc.mma_scale_byte("nvfp4", b)
+
+
+def test_mma_scale_atoms_match_a_reshape(orc):
+    """The atom order restated as numpy axes: [row block][block group][row % 32]
+    [(row % 128) / 32][block % 4]; padding is zero."""
+    rows, cols = 300, 16 * 37
+    nb = cols // 16
+    rng = np.random.default_rng(5)
+    scales = rng.integers(1, 0x7F, size=(rows, nb), dtype=np.uint8)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    _, sf = orc.mma_pack(codes, scales, "nvfp4")
+    rb, kb4 = -(-rows // 128), -(-nb // 4)
+    pad = np.zeros((rb * 128, kb4 * 4), np.uint8)
+    pad[:rows, :nb] = scales
+    want = pad.reshape(rb, 4, 32, kb4, 4).transpose(0, 3, 2, 1, 4).ravel()
+    assert sf.size == orc.mma_sf_bytes(rows, cols) == rb * kb4 * 512
+    assert np.array_equal(sf, want)
+
+
+def test_gemm_oracle_against_numpy_and_exact_integers(orc):
+    rng = np.random.default_rng(6)
+    a = rng.standard_normal((37, 200)).astype(np.float32)
+    w = rng.standard_normal((23, 200)).astype(np.float32)
+    y, yabs = orc.gemm(a, w, nthreads=3)
+    ref = a.astype(np.float64) @ w.astype(np.float64).T
+    assert np.all(np.abs(y - ref) <= 1e-12 * (np.abs(a).astype(np.float64) @ np.abs(w).astype(np.float64).T))
+    assert np.allclose(yabs, np.abs(a).astype(np.float64) @ np.abs(w).astype(np.float64).T, rtol=1e-12)
+    ai = rng.integers(-6, 7, size=(5, 64)).astype(np.float32)
+    wi = rng.integers(-6, 7, size=(7, 64)).astype(np.float32)
+    yi, _ = orc.gemm(ai, wi)
+    assert np.array_equal(yi, ai.astype(np.int64) @ wi.astype(np.int64).T)
+
+
+def test_gemm_of_one_hot_rows_returns_weight_columns(orc):
+    """A one-hot activation row picks one column of the weight reconstruction."""
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.llm_weight(24, 128, seed=43))
+    codes, scales, ts, _ = orc.quantize(xb, "nvfp4_razer_w", nthreads=2)
+    w, _ = orc.dequantize(codes, scales, ts, "nvfp4_razer_w")
+    a = np.zeros((128, 128), np.float32)
+    a[np.arange(128), np.arange(128)] = 1.0
+    y, _ = orc.gemm(a, w)
+    assert np.array_equal(y, w.T.astype(np.float64))
