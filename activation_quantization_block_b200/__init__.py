@@ -10,4 +10,5 @@ from .fp4q import (  # noqa: F401
     error,
     fp4q_abi_version, fp4q_dequantize, fp4q_error, fp4q_quantize, fp4q_status_string, fp4q_workspace_size,
     lib, library_path, quantize, quantize_batch, fp4q_quantize_batch, fp4q_batch_workspace_size,
+    MmaOperand, mma_operand, gemm, fp4q_mma_planes, fp4q_mma_sf_bytes, fp4q_mma_pack, fp4q_gemm,
 )

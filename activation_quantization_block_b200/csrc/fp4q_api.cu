@@ -205,13 +205,65 @@ fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
     if (bits == nullptr) return FP4Q_ERROR_INVALID_VALUE;
     fp4q_status_t s = check_device();
     if (s != FP4Q_SUCCESS) return s;
-    unsigned int v = 0, w = 0;
-    if (read_device_errors(&v, clear != 0) != cudaSuccess || read_batch_device_errors(&w, clear != 0) != cudaSuccess) {
+    unsigned int v = 0, w = 0, u = 0;
+    if (read_device_errors(&v, clear != 0) != cudaSuccess || read_batch_device_errors(&w, clear != 0) != cudaSuccess ||
+        read_gemm_device_errors(&u, clear != 0) != cudaSuccess) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }
-    *bits = v | w;
+    *bits = v | w | u;
     return FP4Q_SUCCESS;
+}
+
+int fp4q_mma_planes(fp4q_format_t fmt)
+{
+    if (fmt == FP4Q_NVFP4) return 1;
+    if (fmt == FP4Q_NVFP4_RAZER || fmt == FP4Q_NVFP4_RAZER_W) return 2;
+    return 0;
+}
+
+size_t fp4q_mma_sf_bytes(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0 || rows > ((int64_t)1 << 40) || cols > ((int64_t)1 << 40)) return 0;
+    return (size_t)mma_sf_bytes(rows, cols);
+}
+
+fp4q_status_t fp4q_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                            fp4q_format_t fmt, uint8_t* planes, uint8_t* sf, fp4q_stream_t stream)
+{
+    if (fp4q_mma_planes(fmt) == 0 || rows < 0 || cols < 0) return FP4Q_ERROR_INVALID_VALUE;
+    if (cols % 16 != 0 || rows > ((int64_t)1 << 40) || cols > ((int64_t)1 << 40)) return FP4Q_ERROR_SHAPE;
+    if (rows * cols == 0) return FP4Q_SUCCESS;
+    if (codes == nullptr || scales == nullptr || planes == nullptr || sf == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(planes, 16) || !aligned(sf, 16))
+        return FP4Q_ERROR_MISALIGNED;
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_mma_pack(codes, scales, rows, cols, fmt, planes, sf,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status_t fp4q_gemm(const uint8_t* a_planes, const uint8_t* a_sf, int a_np, const float* a_scale,
+                        const uint8_t* w_planes, const uint8_t* w_sf, int w_np, const float* w_scale,
+                        int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, fp4q_stream_t stream)
+{
+    if ((a_np != 1 && a_np != 2) || (w_np != 1 && w_np != 2)) return FP4Q_ERROR_INVALID_VALUE;
+    if (M < 0 || N < 0 || K < 0) return FP4Q_ERROR_INVALID_VALUE;
+    if (K == 0 || K % 256 != 0 || N % 8 != 0 || ldy < N || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) ||
+        K >= ((int64_t)1 << 31) || ldy >= ((int64_t)1 << 31))
+        return FP4Q_ERROR_SHAPE;
+    if (ldy % 8 != 0) return FP4Q_ERROR_MISALIGNED;
+    if (M == 0 || N == 0) return FP4Q_SUCCESS;
+    if (a_planes == nullptr || a_sf == nullptr || a_scale == nullptr || w_planes == nullptr || w_sf == nullptr ||
+        w_scale == nullptr || y == nullptr)
+        return FP4Q_ERROR_INVALID_VALUE;
+    if (!aligned(a_planes, 16) || !aligned(a_sf, 16) || !aligned(w_planes, 16) || !aligned(w_sf, 16) ||
+        !aligned(y, 16) || !aligned(a_scale, 4) || !aligned(w_scale, 4))
+        return FP4Q_ERROR_MISALIGNED;
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_gemm_w4a4(a_planes, a_sf, a_np, a_scale, w_planes, w_sf, w_np, w_scale, M, N, K,
+                                      static_cast<uint16_t*>(y), ldy, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t fp4q_batch_workspace_size(int count, const fp4q_tensor_desc_t* tensors, fp4q_format_t fmt, int rotate)

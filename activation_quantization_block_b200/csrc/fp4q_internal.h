@@ -60,6 +60,15 @@ cudaError_t launch_sse_finalize(const double* partials, int n, double count, dou
 cudaError_t read_device_errors(unsigned int* bits, bool clear);
 cudaError_t read_batch_device_errors(unsigned int* bits, bool clear);
 
+// Tensor-core operand form and the W4A4 product (fp4q_gemm.cu).
+int64_t mma_sf_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, int fmt,
+                            uint8_t* planes, uint8_t* sf, cudaStream_t st);
+cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a_np, const float* a_scale,
+                             const uint8_t* w_planes, const uint8_t* w_sf, int w_np, const float* w_scale, int64_t M,
+                             int64_t N, int64_t K, uint16_t* y, int64_t ldy, cudaStream_t st);
+cudaError_t read_gemm_device_errors(unsigned int* bits, bool clear);
+
 // Tile count of a bf16 matrix's view (see make_view): 16 KB tiles.
 int64_t view_tiles(const Geometry& g);
 

@@ -30,7 +30,8 @@ STATUS_NAMES = {
 # Names the C header declares; the tests check that the library exports each one.
 ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc",
-               "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch")
+               "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch",
+               "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm")
 
 
 class TensorDesc(ctypes.Structure):
@@ -79,6 +80,14 @@ def lib() -> ctypes.CDLL:
         L.fp4q_batch_workspace_size.restype = sz
         L.fp4q_quantize_batch.argtypes = [i32, ctypes.POINTER(TensorDesc), i32, i32, u32, vp, sz, vp]
         L.fp4q_quantize_batch.restype = i32
+        L.fp4q_mma_planes.argtypes = [i32]
+        L.fp4q_mma_planes.restype = i32
+        L.fp4q_mma_sf_bytes.argtypes = [i64, i64]
+        L.fp4q_mma_sf_bytes.restype = sz
+        L.fp4q_mma_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp]
+        L.fp4q_mma_pack.restype = i32
+        L.fp4q_gemm.argtypes = [vp, vp, i32, vp, vp, vp, i32, vp, i64, i64, i64, vp, i64, vp]
+        L.fp4q_gemm.restype = i32
         _lib = L
     return _lib
 
@@ -166,6 +175,24 @@ def fp4q_batch_workspace_size(count, descs, fmt, rotate) -> int:
 def fp4q_quantize_batch(count, descs, fmt, rotate, flags, workspace, workspace_bytes, stream=None) -> int:
     return lib().fp4q_quantize_batch(count, _descs(descs), _fmt(fmt), int(rotate), flags, _ptr(workspace),
                                      workspace_bytes, _stream(stream))
+
+
+def fp4q_mma_planes(fmt) -> int:
+    return lib().fp4q_mma_planes(_fmt(fmt))
+
+
+def fp4q_mma_sf_bytes(rows: int, cols: int) -> int:
+    return lib().fp4q_mma_sf_bytes(rows, cols)
+
+
+def fp4q_mma_pack(codes, scales, rows, cols, fmt, planes, sf, stream=None) -> int:
+    return lib().fp4q_mma_pack(_ptr(codes), _ptr(scales), rows, cols, _fmt(fmt), _ptr(planes), _ptr(sf),
+                               _stream(stream))
+
+
+def fp4q_gemm(a_planes, a_sf, a_np, a_scale, w_planes, w_sf, w_np, w_scale, M, N, K, y, ldy, stream=None) -> int:
+    return lib().fp4q_gemm(_ptr(a_planes), _ptr(a_sf), a_np, _ptr(a_scale), _ptr(w_planes), _ptr(w_sf), w_np,
+                           _ptr(w_scale), M, N, K, _ptr(y), ldy, _stream(stream))
 
 
 def tensor_desc(x, q: "Quantized") -> TensorDesc:
@@ -292,3 +319,35 @@ def error(x: torch.Tensor, q: Quantized, fmt="nvfp4_razer", rotate: bool = False
                     ws.numel(), stream)
     _check(st, "fp4q_error")
     return mse
+
+
+class MmaOperand(NamedTuple):
+    planes: torch.Tensor         # uint8 [rows, planes * cols/2]
+    sf: torch.Tensor             # uint8 [fp4q_mma_sf_bytes(rows, cols)]
+    tensor_scale: torch.Tensor   # float32 [1]
+    nplanes: int
+
+
+def mma_operand(q: Quantized, fmt, stream=None) -> MmaOperand:
+    """Tensor-core operand form of a quantized NVFP4-family matrix."""
+    rows, cols = q.codes.shape[0], q.codes.shape[1] * 2
+    npl = fp4q_mma_planes(fmt)
+    if npl == 0:
+        raise Fp4qError(1, "no operand form for this format")
+    planes = torch.empty(rows, npl * cols // 2, dtype=torch.uint8, device=q.codes.device)
+    sf = torch.empty(max(1, fp4q_mma_sf_bytes(rows, cols)), dtype=torch.uint8, device=q.codes.device)
+    _check(fp4q_mma_pack(q.codes, q.scales, rows, cols, fmt, planes, sf, stream), "fp4q_mma_pack")
+    return MmaOperand(planes, sf, q.tensor_scale, npl)
+
+
+def gemm(a: MmaOperand, w: MmaOperand, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16 y = A^ W^T of two operands in tensor-core form (A: M x K, W: N x K)."""
+    M, N = a.planes.shape[0], w.planes.shape[0]
+    K = a.planes.shape[1] * 2 // a.nplanes
+    if w.planes.shape[1] * 2 // w.nplanes != K:
+        raise ValueError("inner dimensions differ")
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=a.planes.device)
+    ldy = y.stride(0) if M > 1 else N
+    _check(fp4q_gemm(a.planes, a.sf, a.nplanes, a.tensor_scale, w.planes, w.sf, w.nplanes, w.tensor_scale, M, N, K,
+                     y, ldy, stream), "fp4q_gemm")
+    return y

@@ -246,6 +246,57 @@ FP4Q_API fp4q_status_t fp4q_quantize_noalloc(const void* x, int64_t rows, int64_
                                              uint8_t* codes, uint8_t* scales, float* tensor_scale,
                                              double* mse, fp4q_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Tensor-core operand form and the W4A4 product ("RaZeR", sect. 2.3: GEMMs on
+ * existing tensor cores handle the remapped code in two passes).
+ *
+ * The operand form of a quantized NVFP4-family matrix (rows x cols, codes and
+ * scales as fp4q_quantize writes them) is what the sm_100a block-scaled tensor
+ * cores read:
+ *  planes  uint8 [rows][P * cols/2], P = fp4q_mma_planes(fmt): P code planes
+ *          per row, each cols/2 bytes in the codes layout.  NVFP4: the codes.
+ *          RaZeR (both modes): plane 0 holds every code except 0b1000, which
+ *          becomes the special value's base b -- the largest E2M1 magnitude
+ *          below |s|, with the sign of s (+-4 for +-5, +-2 for +-2.5) -- and
+ *          plane 1 holds s - b there (+-1, +-0.5) and +0 elsewhere, so the
+ *          decoded planes add up to the reconstruction.
+ *  sf      uint8 [fp4q_mma_sf_bytes(rows, cols)]: each block's scale
+ *          magnitude as an E4M3 byte, bit 7 clear (weight mode: its E3M3 value,
+ *          exact in E4M3), in 512-byte atoms of 128 rows x 4 blocks.  Atom
+ *          (r / 128, kb / 4), row-major over ceil(rows/128) x ceil(cols/64)
+ *          atoms, holds block kb of row r at byte
+ *          (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4; padding is 0.
+ * ------------------------------------------------------------------------ */
+
+/* Code planes of a format's operand form: 1 (NVFP4), 2 (NVFP4_RAZER,
+ * NVFP4_RAZER_W), 0 (MXFP4 or an invalid format: no operand form). */
+FP4Q_API int fp4q_mma_planes(fp4q_format_t fmt);
+
+/* Bytes of the scale atoms of a rows x cols operand (0 for negative sizes). */
+FP4Q_API size_t fp4q_mma_sf_bytes(int64_t rows, int64_t cols);
+
+/* Write the operand form of (codes, scales).  codes, scales, planes and sf are
+ * device pointers, 16-byte aligned; cols a multiple of 16.  Enqueues one
+ * kernel on `stream`.  FP4Q_ERROR_INVALID_VALUE for MXFP4, a bad format, a
+ * null pointer or a negative size. */
+FP4Q_API fp4q_status_t fp4q_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                     fp4q_format_t fmt, uint8_t* planes, uint8_t* sf, fp4q_stream_t stream);
+
+/* y = s_a * s_w * (A^ W^T) as bf16 (round to nearest even), A^ (M x K) and W^
+ * (N x K) the reconstructions of two quantized matrices given in operand form:
+ * a_planes / a_sf with a_np planes and tensor scale *a_scale, w_planes / w_sf
+ * with w_np planes and *w_scale (device fp32 scalars).  The tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, 16-element E4M3 scales, fp32 accumulation)
+ * run the a_np * w_np plane products as one accumulation of a_np * w_np * K
+ * elements.  y is row-major [M][ldy] bf16.  Shapes: K > 0 a multiple of 256,
+ * N a multiple of 8, ldy >= N a multiple of 8, a_np and w_np in {1, 2};
+ * M, N, a_np * K / 2 and w_np * K / 2 below 2^31.  Pointers 16-byte aligned
+ * (the scales 4).  M = 0 or N = 0 enqueues nothing.  The result equals the
+ * exact product up to fp32 accumulation and the final bf16 rounding. */
+FP4Q_API fp4q_status_t fp4q_gemm(const uint8_t* a_planes, const uint8_t* a_sf, int a_np, const float* a_scale,
+                                 const uint8_t* w_planes, const uint8_t* w_sf, int w_np, const float* w_scale,
+                                 int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, fp4q_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -175,3 +175,48 @@ def test_batch_rejects_bad_arguments(descs, kw, expect):
 
 def test_batch_of_nothing_is_a_no_op():
     assert fp4q.fp4q_quantize_batch(0, [], 0, 0, 0, None, 0, 0) == ST["FP4Q_SUCCESS"]
+
+
+def test_mma_planes_and_sf_bytes():
+    assert [fp4q.fp4q_mma_planes(f) for f in (0, 1, 2, 3, 7)] == [1, 2, 0, 2, 0]
+    assert fp4q.fp4q_mma_sf_bytes(300, 4096) == 3 * 64 * 512
+    assert fp4q.fp4q_mma_sf_bytes(1, 16) == 512 and fp4q.fp4q_mma_sf_bytes(-1, 16) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(fmt=2), "FP4Q_ERROR_INVALID_VALUE"),                 # MXFP4 has no operand form
+    (dict(fmt=9), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(cols=40), "FP4Q_ERROR_SHAPE"),
+    (dict(planes=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(sf=A + 4), "FP4Q_ERROR_MISALIGNED"),
+])
+def test_mma_pack_rejects_bad_arguments(kw, expect):
+    args = dict(codes=A, scales=A, rows=4, cols=64, fmt=1, planes=A, sf=A, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_mma_pack(**args) == ST[expect]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(a_np=3), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(w_np=0), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(M=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(K=128), "FP4Q_ERROR_SHAPE"),                         # K a multiple of 256
+    (dict(K=0), "FP4Q_ERROR_SHAPE"),
+    (dict(N=12, ldy=16), "FP4Q_ERROR_SHAPE"),                  # N a multiple of 8
+    (dict(ldy=8), "FP4Q_ERROR_SHAPE"),                         # ldy >= N
+    (dict(ldy=68), "FP4Q_ERROR_MISALIGNED"),
+    (dict(y=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(w_scale=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(a_planes=A + 8), "FP4Q_ERROR_MISALIGNED"),
+    (dict(a_scale=A + 2), "FP4Q_ERROR_MISALIGNED"),
+])
+def test_gemm_rejects_bad_arguments(kw, expect):
+    args = dict(a_planes=A, a_sf=A, a_np=2, a_scale=A, w_planes=A, w_sf=A, w_np=1, w_scale=A, M=4, N=64, K=256,
+                y=A, ldy=64, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_gemm(**args) == ST[expect]
+
+
+def test_gemm_of_nothing_is_a_no_op():
+    assert fp4q.fp4q_gemm(A, A, 1, A, A, A, 1, A, 0, 64, 256, A, 64, 0) == ST["FP4Q_SUCCESS"]
