@@ -2,6 +2,8 @@
 
     python -m activation_quantization_block_b200.kernel_bench --op quantize --fmt nvfp4_razer \\
         --rows 14336 --cols 4096 [--rotate] [--no-mse] [--scale-given] [--iters 20]
+    python -m activation_quantization_block_b200.kernel_bench --op gemm --a-fmt nvfp4_razer \\
+        --w-fmt nvfp4_razer_w --M 8192 --N 8192 --K 8192
 
 Each iteration is one C-ABI call on the current stream, timed with CUDA events;
 between iterations a 512 MB buffer is overwritten so that no input stays in
@@ -10,11 +12,18 @@ per call, elements/s and the call's algorithmic bytes per second
 (quantize: 2 B read + codes and scales written, plus 2 B for the absmax read
 when the tensor scale is computed; dequantize: codes and scales read + 2 B
 written; error: 2 B + codes and scales read).
+
+--op gemm times fp4q_gemm on the operand forms of a seeded activation-like A
+(M x K, --a-fmt) and LLM-weight W (N x K, --w-fmt) and reports TFLOP/s: useful
+(2 M N K) and on the tensor cores (times the plane passes), and their fraction
+of the dense FP4 peak, taken as the measured bf16 peak of MEASURED_PEAKS.json
+times 4 (the nominal FP4 / bf16 ratio, 9 / 2.25 PFLOP/s).
 """
 from __future__ import annotations
 
 import argparse
 import json
+import os
 import statistics
 
 import torch
@@ -24,7 +33,7 @@ from . import fp4q, synthetic
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["quantize", "dequantize", "error"], default="quantize")
+    p.add_argument("--op", choices=["quantize", "dequantize", "error", "gemm"], default="quantize")
     p.add_argument("--fmt", choices=list(fp4q.FORMATS), default="nvfp4_razer")
     p.add_argument("--rows", type=int, default=14336)
     p.add_argument("--cols", type=int, default=4096)
@@ -36,7 +45,14 @@ def main(argv=None):
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--no-flush", action="store_true")
+    p.add_argument("--a-fmt", choices=["nvfp4", "nvfp4_razer", "nvfp4_razer_w"], default="nvfp4_razer")
+    p.add_argument("--w-fmt", choices=["nvfp4", "nvfp4_razer", "nvfp4_razer_w"], default="nvfp4_razer_w")
+    p.add_argument("--M", type=int, default=8192)
+    p.add_argument("--N", type=int, default=8192)
+    p.add_argument("--K", type=int, default=8192)
     a = p.parse_args(argv)
+    if a.op == "gemm":
+        return gemm_main(a)
 
     dev = torch.device("cuda", torch.cuda.current_device())
     gen = {"weight": synthetic.llm_weight, "activation": synthetic.activation_t3,
@@ -91,6 +107,51 @@ def main(argv=None):
         "ms_median": med, "ms_min": best, "elements_per_s": n / (med / 1e3),
         "algorithmic_bytes": nbytes, "gbs_median": nbytes / (med / 1e3) / 1e9, "gbs_best": nbytes / (best / 1e3) / 1e9,
     }), flush=True)
+
+
+def fp4_peak_tflops():
+    """Dense FP4 peak: measured bf16 burst peak x 4, else the pool's fallback bf16 figure x 4."""
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 4"
+    except (OSError, ValueError, KeyError):
+        return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
+def gemm_main(a):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    xa = synthetic.activation_t3(a.M, a.K, seed=a.seed, device=dev)
+    xw = synthetic.llm_weight(a.N, a.K, seed=a.seed + 1, device=dev)
+    oa = fp4q.mma_operand(fp4q.quantize(xa, a.a_fmt, want_mse=False), a.a_fmt)
+    ow = fp4q.mma_operand(fp4q.quantize(xw, a.w_fmt, want_mse=False), a.w_fmt)
+    del xa, xw
+    y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
+    flush = None if a.no_flush else torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    for _ in range(a.warmup):
+        fp4q.gemm(oa, ow, out=y)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(a.iters):
+        if flush is not None:
+            flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fp4q.gemm(oa, ow, out=y)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    med = statistics.median(times)
+    passes = oa.nplanes * ow.nplanes
+    useful = 2.0 * a.M * a.N * a.K / (med / 1e3) / 1e12
+    peak, kind = fp4_peak_tflops()
+    print(json.dumps({
+        "op": "gemm", "a_fmt": a.a_fmt, "w_fmt": a.w_fmt, "M": a.M, "N": a.N, "K": a.K, "passes": passes,
+        "l2_flushed": flush is not None, "ms_median": med, "ms_min": min(times),
+        "useful_tflops": useful, "tensor_tflops": useful * passes, "fp4_peak_tflops": peak, "peak_kind": kind,
+        "tensor_frac": useful * passes / peak,
+    }), flush=True)
+    return 0
 
 
 if __name__ == "__main__":
