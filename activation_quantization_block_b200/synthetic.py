@@ -90,11 +90,12 @@ def mlp_row_scaled(rows: int, cols: int, seed: int, device="cpu", std: float = 0
 def random_packed(rows: int, cols: int, fmt: str, seed: int, device="cpu"):
     """Random valid packed tensor: ``(codes u8 [rows, cols/2], scales u8 [rows, cols/B], tensor_scale f32 [1])``.
 
-    ``fmt`` is "nvfp4", "nvfp4_razer", "mxfp4" or "nvfp4_razer_w".
+    ``fmt`` is "nvfp4", "nvfp4_razer", "mxfp4" (or "mxfp4_ceil", the same stored format) or
+    "nvfp4_razer_w".
     """
     g = _gen(seed, device)
     codes = torch.randint(0, 256, (rows, cols // 2), generator=g, device=device, dtype=torch.int32)
-    if fmt == "mxfp4":
+    if fmt in ("mxfp4", "mxfp4_ceil"):
         scales = torch.randint(127 - 20, 127 + 21, (rows, cols // 32), generator=g, device=device,
                                dtype=torch.int32)
     elif fmt == "nvfp4_razer_w":

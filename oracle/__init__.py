@@ -20,8 +20,11 @@ import subprocess
 
 import numpy as np
 
-NVFP4, NVFP4_RAZER, MXFP4, NVFP4_RAZER_W = 0, 1, 2, 3
-FORMAT_NAMES = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4, "nvfp4_razer_w": NVFP4_RAZER_W}
+NVFP4, NVFP4_RAZER, MXFP4, NVFP4_RAZER_W, MXFP4_CEIL = 0, 1, 2, 3, 4
+# "mxfp4_ceil": MXFP4 whose block exponent maps the block maximum onto 6 without clipping
+# (the encoder's choice only: stored and decoded exactly as MXFP4)
+FORMAT_NAMES = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4, "nvfp4_razer_w": NVFP4_RAZER_W,
+                "mxfp4_ceil": MXFP4_CEIL}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4q_oracle.c")
@@ -61,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.orc_tensor_scale_from_amax_w.argtypes = [f32]; L.orc_tensor_scale_from_amax_w.restype = f32
         L.orc_e8m0_value.argtypes = [i32]; L.orc_e8m0_value.restype = f64
         L.orc_mx_exponent.argtypes = [f32]; L.orc_mx_exponent.restype = i32
+        L.orc_mx_exponent_ceil.argtypes = [f32]; L.orc_mx_exponent_ceil.restype = i32
         L.orc_hadamard_entry.argtypes = [i32, i32]; L.orc_hadamard_entry.restype = i32
         L.orc_wht_constant.argtypes = []; L.orc_wht_constant.restype = f32
         L.orc_wht32.argtypes = [vp, vp]; L.orc_wht32.restype = None
@@ -93,7 +97,7 @@ def _fmt(fmt) -> int:
 
 
 def block_size(fmt) -> int:
-    return 32 if _fmt(fmt) == MXFP4 else 16
+    return 32 if _fmt(fmt) in (MXFP4, MXFP4_CEIL) else 16
 
 
 def _ptr(a: np.ndarray) -> int:
@@ -142,6 +146,11 @@ def e8m0_value(byte: int) -> float:
 
 def mx_exponent(a: float) -> int:
     return lib().orc_mx_exponent(float(a))
+
+
+def mx_exponent_ceil(a: float) -> int:
+    """Smallest e with a <= 6 * 2^e, clamped to [-127, 127] (the no-clipping block exponent)."""
+    return lib().orc_mx_exponent_ceil(float(a))
 
 
 def hadamard_entry(i: int, j: int) -> int:

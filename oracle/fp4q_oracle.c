@@ -62,6 +62,9 @@
  *     (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
  *  R9 W4A4 product: Y = A^ W^T for A^ (M x K) and W^ (N x K) the fp32
  *     reconstructions of two quantized matrices, summed in binary64.
+ *  R10 MXFP4 exponent without clipping [TORQ sect. 2, S-step: the block
+ *     scale maps the block maximum onto the largest code]: e is the smallest
+ *     integer with a <= 6 * 2^e, clamped to [-127, 127]; nothing saturates.
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC
  * -pthread.  Floating point is IEEE binary32/binary64 with round-to-nearest
@@ -77,6 +80,8 @@
 #define ORC_NVFP4_RAZER 1
 #define ORC_MXFP4 2
 #define ORC_NVFP4_RAZER_W 3
+#define ORC_MXFP4_CEIL 4      /* MXFP4 with the R10 exponent; stored and decoded as MXFP4 */
+#define IS_MX(f) ((f) == ORC_MXFP4 || (f) == ORC_MXFP4_CEIL)
 
 /* The second special-value pair of the RaZeR weight mode (R7): the winner of
  * the offline search over multiples of 0.5 (oracle/razer_weight_pair.py).
@@ -245,6 +250,19 @@ int orc_mx_exponent(float a)
     return e;
 }
 
+/* R10: the smallest e with a <= 6 * 2^e (a > 0), by search upward from an
+ * exponent known to be too small; 6 * 2^e is exact in binary64. */
+int orc_mx_exponent_ceil(float a)
+{
+    int k;
+    (void)frexp((double)a, &k);    /* a < 2^k */
+    int e = k - 4;                 /* 6 * 2^(k-4) < 2^k / 2: too small */
+    while ((double)a > 6.0 * ldexp(1.0, e)) ++e;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
 /* ------------------------------------------------------------------------ */
 /* 32-point Walsh-Hadamard rotation  [TORQ sect. 2: an orthogonal rotation     */
 /* inside each block; R5 fixes it to the Sylvester Hadamard matrix / sqrt 32]  */
@@ -288,7 +306,7 @@ static void load_row(const uint16_t* x, int64_t cols, int rotate, float* y)
         }
 }
 
-static int block_size(int fmt) { return fmt == ORC_MXFP4 ? 32 : 16; }
+static int block_size(int fmt) { return IS_MX(fmt) ? 32 : 16; }
 
 /* ------------------------------------------------------------------------ */
 /* Tensor absmax (NVFP4 first level, R2)                                      */
@@ -444,13 +462,13 @@ static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
         float v[32];
         int q[32];
         int sbyte;
-        if (fmt == ORC_MXFP4) {
+        if (IS_MX(fmt)) {
             /* TORQ sect. 1 / R3 */
             if (a == 0.0f) {
                 sbyte = 0;
                 for (int i = 0; i < B; ++i) q[i] = 0;
             } else {
-                int e = orc_mx_exponent(a);
+                int e = fmt == ORC_MXFP4_CEIL ? orc_mx_exponent_ceil(a) : orc_mx_exponent(a);
                 sbyte = e + 127;
                 float r = (float)ldexp(1.0, -e);    /* exact power of two */
                 for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
@@ -490,10 +508,10 @@ static void dequant_row(const uint8_t* row_codes, const uint8_t* row_scales, int
     const int B = block_size(fmt);
     for (int64_t b0 = 0; b0 < cols; b0 += B) {
         int sbyte = row_scales[b0 / B];
-        float den = (fmt == ORC_MXFP4) ? 0.0f : nv_den(fmt, sbyte, s_t);
+        float den = IS_MX(fmt) ? 0.0f : nv_den(fmt, sbyte, s_t);
         for (int i = 0; i < B; ++i) {
             int code = get_code(row_codes, b0 + i);
-            out[b0 + i] = (fmt == ORC_MXFP4) ? mx_decode(code, sbyte)
+            out[b0 + i] = IS_MX(fmt) ? mx_decode(code, sbyte)
                                              : nv_decode(fmt, code, sbyte, den);
         }
     }
@@ -577,7 +595,7 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
     const int B = block_size(fmt);
     if (rows < 0 || cols % B || (rotate && cols % 32) || ldx < cols) return -1;
     float s_t = 0.0f;
-    if (fmt != ORC_MXFP4) {
+    if (!IS_MX(fmt)) {
         if (scale_given) s_t = *tensor_scale;
         else {
             s_t = tensor_scale_for(fmt, orc_tensor_amax(x, rows, cols, ldx, rotate, nthreads));
@@ -700,7 +718,7 @@ static double special_base(double s)
 int orc_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, int fmt,
                  uint8_t* planes, uint8_t* sf)
 {
-    if (fmt == ORC_MXFP4 || rows < 0 || cols % 16) return -1;
+    if (IS_MX(fmt) || rows < 0 || cols % 16) return -1;
     const int np = orc_mma_planes(fmt);
     const int64_t half = cols / 2, nb = cols / 16;
     memset(sf, 0, (size_t)orc_mma_sf_bytes(rows, cols));

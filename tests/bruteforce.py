@@ -172,22 +172,26 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool, pair2: float 
                 for i in range(32):
                     s = sum((H[i, j] * seg[j] for j in range(32)), Fraction(0))
                     y[r, g + i] = np.float32(rn_f32(s) * c)
-    B = 32 if fmt == "mxfp4" else 16
+    mx = fmt in ("mxfp4", "mxfp4_ceil")
+    B = 32 if mx else 16
     codes = np.zeros((rows, cols), dtype=np.int64)
     scales = np.zeros((rows, cols // B), dtype=np.int64)
     ts = np.float32(0)
     wmode = fmt == "nvfp4_razer_w"
-    if fmt != "mxfp4":
+    if not mx:
         A = np.float32(np.max(np.abs(y))) if y.size else np.float32(0)
         ts = np.float32(A / np.float32(180 if wmode else 2688))
     for r in range(rows):
         for b in range(cols // B):
             blk = y[r, b * B:(b + 1) * B]
             a = np.float32(np.max(np.abs(blk)))
-            if fmt == "mxfp4":
+            if mx:
                 if a == 0:
                     continue
-                e = max(-127, min(127, floor_log2(float(a)) - 2))
+                if fmt == "mxfp4_ceil":   # the smallest exponent whose 6 * 2^e holds the block maximum
+                    e = min(k for k in range(-127, 128) if Fraction(float(a)) <= 6 * Fraction(2) ** k)
+                else:
+                    e = max(-127, min(127, floor_log2(float(a)) - 2))
                 scales[r, b] = e + 127
                 v = [np.float32(val * np.float32(2.0 ** -e)) for val in blk]
             else:
@@ -217,13 +221,14 @@ def dequantize_bruteforce(codes: np.ndarray, scales: np.ndarray, ts: float, fmt:
     """fp32 reconstruction from the bit-field definitions (exact rationals for rotation)."""
     rows, cols = codes.shape[0], codes.shape[1] * 2
     nib = unpack_codes(codes, cols)
-    B = 32 if fmt == "mxfp4" else 16
+    mx = fmt in ("mxfp4", "mxfp4_ceil")
+    B = 32 if mx else 16
     out = np.zeros((rows, cols), dtype=np.float32)
     for r in range(rows):
         for j in range(cols):
             sb = int(scales[r, j // B])
             code = int(nib[r, j])
-            if fmt == "mxfp4":
+            if mx:
                 out[r, j] = np.float32(E2M1[code] * 2.0 ** (sb - 127))
             else:
                 if fmt == "nvfp4_razer_w":

@@ -243,7 +243,7 @@ def _tiny_inputs():
     return [a.astype(ml_dtypes.bfloat16).view(np.uint16) for a in out]
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w", "mxfp4_ceil"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_quantize_equals_bruteforce(orc, fmt, rotate):
     for xb in _tiny_inputs():
@@ -258,7 +258,7 @@ def test_quantize_equals_bruteforce(orc, fmt, rotate):
         assert abs(sse - float(exact)) <= 1e-12 * max(1.0, float(exact))
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w", "mxfp4_ceil"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_dequantize_equals_bruteforce(orc, fmt, rotate):
     import torch
@@ -607,3 +607,51 @@ def test_gemm_of_one_hot_rows_returns_weight_columns(orc):
     a[np.arange(128), np.arange(128)] = 1.0
     y, _ = orc.gemm(a, w)
     assert np.array_equal(y, w.T.astype(np.float64))
+
+
+# ---------------------------------------------------------------- MXFP4 exponent without clipping
+
+def _mx_ceil_points():
+    pts = []
+    for k in list(range(-149, -120)) + list(range(-20, 21)) + list(range(120, 128)):
+        for m in (1.0, 1.25, 1.5, 1.75, 1.9990234375):
+            v = np.float32(m * 2.0 ** k)
+            if v > 0 and np.isfinite(v):
+                pts += [v, np.nextafter(v, np.float32(0)), np.nextafter(v, np.float32(np.inf))]
+    for e in range(-126, 126):          # 6 * 2^e and its neighbours
+        v = np.float32(6.0 * 2.0 ** e)
+        pts += [v, np.nextafter(v, np.float32(0)), np.nextafter(v, np.float32(np.inf))]
+    return [p for p in pts if p > 0 and np.isfinite(p)]
+
+
+def test_mx_exponent_ceil_equals_exhaustive_minimum(orc):
+    """e = min{e in [-127, 127] : a <= 6 * 2^e}, by enumeration with exact rationals."""
+    for a in _mx_ceil_points():
+        fa = Fraction(float(a))
+        want = min((k for k in range(-127, 128) if fa <= 6 * Fraction(2) ** k), default=127)
+        assert orc.mx_exponent_ceil(float(a)) == want, a
+
+
+def test_mx_exponent_ceil_closed_forms(orc):
+    assert orc.mx_exponent_ceil(6.0) == 0 and orc.mx_exponent_ceil(3.0) == -1 and orc.mx_exponent_ceil(4.0) == 0
+    assert orc.mx_exponent_ceil(float(np.nextafter(np.float32(6), np.float32(7)))) == 1
+    # differs from the floor rule exactly when the block maximum's mantissa exceeds 1.5
+    for k in range(-30, 30):
+        for m, up in ((1.0, 0), (1.5, 0), (1.5000001, 1), (1.75, 1), (1.99, 1)):
+            a = float(np.float32(m * 2.0 ** k))
+            assert orc.mx_exponent_ceil(a) - orc.mx_exponent(a) == up
+
+
+def test_mxfp4_ceil_never_saturates_and_decodes_as_mxfp4(orc):
+    from activation_quantization_block_b200 import synthetic
+    xb = synthetic.bf16_bits(synthetic.activation_t3(64, 512, seed=44))
+    x = bf.bits_to_f32(xb).astype(np.float64)
+    c, s, _, sse_c = orc.quantize(xb, "mxfp4_ceil", nthreads=2)
+    _, _, _, sse_f = orc.quantize(xb, "mxfp4", nthreads=2)
+    y_c, _ = orc.dequantize(c, s, 0.0, "mxfp4_ceil")
+    y_m, _ = orc.dequantize(c, s, 0.0, "mxfp4")
+    assert np.array_equal(y_c, y_m)                     # the same stored format
+    blocks = np.abs(x).reshape(64, 16, 32).max(-1)
+    scale = 2.0 ** (s.astype(np.float64) - 127)
+    assert np.all(blocks <= 6 * scale)                  # the block maximum fits: no element saturates
+    assert sse_c != sse_f
