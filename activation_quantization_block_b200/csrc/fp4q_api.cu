@@ -70,6 +70,13 @@ fp4q_status_t check_matrix(const void* p, int64_t cols, int64_t ld)
 
 fp4q_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_SUCCESS : FP4Q_ERROR_CUDA; }
 
+// Known flags only; the MX exponent flag only with MXFP4.
+bool valid_flags(uint32_t flags, int fmt)
+{
+    if (flags & ~(FP4Q_FLAG_TENSOR_SCALE_GIVEN | FP4Q_FLAG_MX_CEIL_SCALE)) return false;
+    return !(flags & FP4Q_FLAG_MX_CEIL_SCALE) || fmt == FP4Q_MXFP4;
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,7 +110,7 @@ fp4q_status_t fp4q_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
 {
     fp4q_status_t s = check_shape(rows, cols, fmt, rotate);
     if (s != FP4Q_SUCCESS) return s;
-    if (flags & ~FP4Q_FLAG_TENSOR_SCALE_GIVEN) return FP4Q_ERROR_INVALID_VALUE;
+    if (!valid_flags(flags, fmt)) return FP4Q_ERROR_INVALID_VALUE;
     const bool nv = fmt != FP4Q_MXFP4;
     const bool given = (flags & FP4Q_FLAG_TENSOR_SCALE_GIVEN) != 0;
     if (nv && tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
@@ -138,7 +145,8 @@ fp4q_status_t fp4q_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
         if ((s = from_cuda(launch_amax(xp, g, rotate, amax_part, &n_amax, st))) != FP4Q_SUCCESS) return s;
     }
     int n_sse = 0;
-    s = from_cuda(launch_quantize(xp, g, fmt, rotate, mse != nullptr, given ? 1 : 0, codes, scales,
+    s = from_cuda(launch_quantize(xp, g, fmt, rotate, mse != nullptr, given ? 1 : 0,
+                                  (flags & FP4Q_FLAG_MX_CEIL_SCALE) ? 1 : 0, codes, scales,
                                   tensor_scale, amax_part, n_amax, sse_part, &n_sse, st));
     if (s != FP4Q_SUCCESS) return s;
     if (mse) s = from_cuda(launch_sse_finalize(sse_part, n_sse, (double)n, mse, st));
@@ -276,7 +284,7 @@ fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* tensors, 
                                   uint32_t flags, void* workspace, size_t workspace_bytes, fp4q_stream_t stream)
 {
     if (count < 0 || (count > 0 && tensors == nullptr)) return FP4Q_ERROR_INVALID_VALUE;
-    if (flags & ~FP4Q_FLAG_TENSOR_SCALE_GIVEN) return FP4Q_ERROR_INVALID_VALUE;
+    if (!valid_flags(flags, fmt)) return FP4Q_ERROR_INVALID_VALUE;
     const bool nv = fmt != FP4Q_MXFP4;
     const bool given = (flags & FP4Q_FLAG_TENSOR_SCALE_GIVEN) != 0;
     fp4q_status_t s;
@@ -311,7 +319,8 @@ fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* tensors, 
         work.push_back(BatchTensor{t.x, t.rows, t.cols, t.ldx, t.codes, t.scales, t.tensor_scale, t.mse});
     }
     if (!work.empty() &&
-        launch_quantize_batch(work.data(), (int)work.size(), fmt, rotate, given ? 1 : 0, workspace, st) != cudaSuccess) {
+        launch_quantize_batch(work.data(), (int)work.size(), fmt, rotate, given ? 1 : 0,
+                              (flags & FP4Q_FLAG_MX_CEIL_SCALE) ? 1 : 0, workspace, st) != cudaSuccess) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }

@@ -53,6 +53,7 @@ struct ChainArgs {
     double fin_count;
     int32_t n_sse_in;
     int32_t has_fin;
+    int32_t mx_ceil;
 };
 
 template <int FMT, bool ROT, bool SSE>
@@ -152,8 +153,10 @@ __global__ void __launch_bounds__(kThreads, 3)
         const int64_t tile = slot_tile[s];
         const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
         if (is_q) {
-            if (a.q_flat) acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc);
-            else acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc);
+            if (a.q_flat)
+                acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0);
+            else
+                acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0);
         } else {
             m = fmaxf(m, amax_tile<ROT>(tp));
         }
@@ -225,8 +228,8 @@ struct View {
 
 size_t batch_workspace_bytes() { return (size_t)kRing * kMaxPartials * (sizeof(float) + sizeof(double)); }
 
-cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, void* workspace,
-                                  cudaStream_t st)
+cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, int mx_ceil,
+                                  void* workspace, cudaStream_t st)
 {
     if (n <= 0) return cudaSuccess;
     const bool computed = fmt != kMX && !scale_given;
@@ -246,6 +249,7 @@ cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rot
     std::vector<int> grids((size_t)n + 2, 0);    // CTAs (= partials written) of kernel j
     for (int64_t j = 0; j < n + lag + 1; ++j) {
         ChainArgs a = {};
+        a.mx_ceil = mx_ceil;
         const int64_t kq = j - lag;              // tensor quantized by kernel j
         const int64_t ka = computed ? j : -1;    // tensor whose absmax pass kernel j runs
         const int64_t kf = j - lag - 1;          // tensor whose MSE kernel j finalises

@@ -686,15 +686,21 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
     }
 }
 
-// One 32-element MXFP4 block.
+// One 32-element MXFP4 block.  The exponent is floor(log2 a) - 2 (values in
+// [6, 8) 2^e saturate to 6) or, with ceil, the smallest e with a <= 6 * 2^e:
+// one more when a's significand exceeds 1.5 ("TORQ: Two-Level Orthogonal
+// Rotation for MXFP4 Quantization", sect. 2, S-step: the block maximum onto
+// the largest code), at most 125 so that 6 * 2^e stays finite in fp32.
 template <bool XH>
-__device__ __forceinline__ void encode_mx32(const float* y, float a, uint32_t* cw, uint32_t& sb_out, float* xh)
+__device__ __forceinline__ void encode_mx32(const float* y, float a, bool ceil, uint32_t* cw, uint32_t& sb_out,
+                                            float* xh)
 {
     int e = -127;
     float r = 0.0f;
     uint32_t sb = 0;
     if (a > 0.0f) {
         e = floor_log2_f32(a) - 2;          // 2 = exponent of the largest E2M1 value
+        if (ceil) e = min(e + significand_above_1p5(a), 125);
         e = e < -127 ? -127 : (e > 127 ? 127 : e);
         sb = (uint32_t)(e + 127);
         r = exp2i(-e);
@@ -917,7 +923,7 @@ __device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint3
 // Returns the unit's squared error when SSE.
 template <int FMT, bool ROT, bool SSE, bool FLAT>
 __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, int64_t k, uint8_t* codes,
-                                                uint8_t* scales, const NvScale& nsc)
+                                                uint8_t* scales, const NvScale& nsc, bool mx_ceil = false)
 {
     const int t = threadIdx.x;
     const bool a16 = FLAT || (tl.cols % 32) == 0;
@@ -957,7 +963,7 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                 float am = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(y[i]));
-                encode_mx32<SSE>(y, am, cw, sb0, xh);
+                encode_mx32<SSE>(y, am, mx_ceil, cw, sb0, xh);
             } else {
                 float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll

@@ -241,6 +241,15 @@ __device__ __forceinline__ int floor_log2_f32(float a)
     return (31 - __clz((int)u)) - 149;
 }
 
+// 1 when the significand of a finite a > 0 exceeds 1.5 (a > 1.5 * 2^floor(log2 a)).
+__device__ __forceinline__ int significand_above_1p5(float a)
+{
+    const uint32_t u = __float_as_uint(a);
+    if ((u >> 23) & 0xFFu) return (u & 0x7FFFFFu) > 0x400000u ? 1 : 0;
+    const int b = 31 - __clz((int)u);                    // subnormal: leading bit of u
+    return b > 0 && (u & ((1u << b) - 1u)) > (1u << (b - 1)) ? 1 : 0;
+}
+
 // 2^k for k in [-127, 127] as fp32 (2^-127 is subnormal).
 __device__ __forceinline__ float exp2i(int k)
 {

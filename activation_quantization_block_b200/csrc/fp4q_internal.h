@@ -41,7 +41,7 @@ cudaError_t launch_amax(const uint16_t* x, const Geometry& g, int rotate, float*
                         int* grid_out, cudaStream_t st);
 
 cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int rotate, int want_sse,
-                            int scale_given, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                            int scale_given, int mx_ceil, uint8_t* codes, uint8_t* scales, float* tensor_scale,
                             const float* amax_partials, int n_amax, double* sse_partials,
                             int* grid_out, cudaStream_t st);
 
@@ -87,7 +87,8 @@ size_t batch_workspace_bytes();
 
 // Quantize n non-empty tensors as a chain of persistent kernels, one per tensor
 // (absmax pass of tensor j interleaved with the quantize pass of tensor j-1).
-cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, void* workspace,
+cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, int mx_ceil,
+                                  void* workspace,
                                   cudaStream_t st);
 
 }  // namespace fp4q

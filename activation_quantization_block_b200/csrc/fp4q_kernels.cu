@@ -90,6 +90,7 @@ struct QuantArgs {
     int n_amax;
     int scale_given;
     int reverse;
+    int mx_ceil;
     double* sse_partials;
 };
 
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_cons
             break;
         }
         const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
-        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc);
+        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc, a.mx_ceil != 0);
         pipe_release(p, j);
         if (t == 0 && j + kStages < sc.mine) {
             if (!pipe_stage_free(p, j)) {
@@ -338,7 +339,7 @@ static cudaError_t quantize_dispatch(const CUtensorMap& map, const QuantArgs& a,
 }
 
 cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int rotate, int want_sse,
-                            int scale_given, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                            int scale_given, int mx_ceil, uint8_t* codes, uint8_t* scales, float* tensor_scale,
                             const float* amax_partials, int n_amax, double* sse_partials, int* grid_out,
                             cudaStream_t st)
 {
@@ -351,6 +352,7 @@ cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int r
     a.amax_partials = amax_partials;
     a.n_amax = n_amax;
     a.scale_given = scale_given;
+    a.mx_ceil = mx_ceil;
     // after an absmax pass: start where that pass ended (its last tiles are in L2)
     const bool after_amax = fmt != kMX && !scale_given;
     a.reverse = after_amax ? 1 : 0;

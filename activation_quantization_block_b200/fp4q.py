@@ -20,6 +20,7 @@ from . import _build
 NVFP4, NVFP4_RAZER, MXFP4, NVFP4_RAZER_W = 0, 1, 2, 3
 FORMATS = {"nvfp4": NVFP4, "nvfp4_razer": NVFP4_RAZER, "mxfp4": MXFP4, "nvfp4_razer_w": NVFP4_RAZER_W}
 FLAG_TENSOR_SCALE_GIVEN = 0x1
+FLAG_MX_CEIL_SCALE = 0x2
 
 SUCCESS = 0
 STATUS_NAMES = {
@@ -246,8 +247,10 @@ def _rows_cols_ld(x: torch.Tensor):
 
 def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_scale: torch.Tensor | None = None,
              want_mse: bool = True, out: Quantized | None = None, workspace: torch.Tensor | None = None,
-             stream=None) -> Quantized:
-    """Quantize a bf16 CUDA matrix; returns codes, scales, tensor scale and (optionally) the MSE."""
+             stream=None, mx_ceil: bool = False) -> Quantized:
+    """Quantize a bf16 CUDA matrix; returns codes, scales, tensor scale and (optionally) the MSE.
+
+    mx_ceil (MXFP4): block exponent without clipping (FP4Q_FLAG_MX_CEIL_SCALE)."""
     if x.dtype != torch.bfloat16 or not x.is_cuda:
         raise TypeError("x must be a bf16 CUDA tensor")
     rows, cols, ld = _rows_cols_ld(x)
@@ -264,7 +267,7 @@ def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_sc
         if tensor_scale is not None:
             ts = tensor_scale
     ws = workspace if workspace is not None else workspace_for(dev, stream)
-    flags = FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0
+    flags = (FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
     st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize")
     return Quantized(codes, scales, ts, mse)
@@ -280,7 +283,8 @@ def empty_like_quantized(x: torch.Tensor, fmt, want_mse: bool = True) -> Quantiz
 
 
 def quantize_batch(xs, fmt="nvfp4_razer", rotate: bool = False, outs=None, scale_given: bool = False,
-                   want_mse: bool = True, workspace: torch.Tensor | None = None, stream=None) -> list:
+                   want_mse: bool = True, workspace: torch.Tensor | None = None, stream=None,
+                   mx_ceil: bool = False) -> list:
     """Quantize a list of bf16 CUDA matrices with one fp4q_quantize_batch call.
 
     With scale_given, each out's tensor_scale holds the input scale."""
@@ -292,7 +296,7 @@ def quantize_batch(xs, fmt="nvfp4_razer", rotate: bool = False, outs=None, scale
     descs = _descs([tensor_desc(x, q) for x, q in zip(xs, outs)])
     need = fp4q_batch_workspace_size(len(xs), descs, fmt, rotate)
     ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
-    flags = FLAG_TENSOR_SCALE_GIVEN if scale_given else 0
+    flags = (FLAG_TENSOR_SCALE_GIVEN if scale_given else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
     st = fp4q_quantize_batch(len(xs), descs, fmt, rotate, flags, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize_batch")
     return outs

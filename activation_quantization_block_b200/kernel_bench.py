@@ -40,6 +40,7 @@ def main(argv=None):
     p.add_argument("--rotate", action="store_true")
     p.add_argument("--no-mse", action="store_true")
     p.add_argument("--scale-given", action="store_true")
+    p.add_argument("--mx-ceil", action="store_true", help="MXFP4 block exponent without clipping")
     p.add_argument("--data", choices=["weight", "activation", "mlp"], default="weight")
     p.add_argument("--seed", type=int, default=2)
     p.add_argument("--iters", type=int, default=20)
@@ -67,7 +68,7 @@ def main(argv=None):
     flush = None if a.no_flush else torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
     packed = n // 2 + n // B
     if a.op == "quantize":
-        flags = fp4q.FLAG_TENSOR_SCALE_GIVEN if a.scale_given else 0
+        flags = (fp4q.FLAG_TENSOR_SCALE_GIVEN if a.scale_given else 0) | (fp4q.FLAG_MX_CEIL_SCALE if a.mx_ceil else 0)
         nbytes = 2 * n + packed + (0 if a.scale_given or a.fmt == "mxfp4" else 2 * n)
 
         def call():
@@ -103,6 +104,7 @@ def main(argv=None):
     med, best = statistics.median(times), min(times)
     print(json.dumps({
         "op": a.op, "fmt": a.fmt, "rotate": a.rotate, "mse": not a.no_mse, "scale_given": a.scale_given,
+        "mx_ceil": a.mx_ceil,
         "rows": a.rows, "cols": a.cols, "data": a.data, "l2_flushed": flush is not None,
         "ms_median": med, "ms_min": best, "elements_per_s": n / (med / 1e3),
         "algorithmic_bytes": nbytes, "gbs_median": nbytes / (med / 1e3) / 1e9, "gbs_best": nbytes / (best / 1e3) / 1e9,

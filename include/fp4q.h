@@ -120,8 +120,17 @@ typedef enum {
     FP4Q_ERROR_CUDA = 6               /* a CUDA runtime call or kernel launch failed */
 } fp4q_status_t;
 
-/* NVFP4 formats: *tensor_scale is an input; the tensor-absmax pass is skipped. */
+/* NVFP4 formats: *tensor_scale is an input; the tensor-absmax pass is skipped.
+ * With *tensor_scale = 1 this is single-level NVFP4: the E4M3 block scale alone
+ * carries the block's range (values whose block maximum / 6 falls below the
+ * E4M3 normal range take subnormal scales). */
 #define FP4Q_FLAG_TENSOR_SCALE_GIVEN 0x1u
+/* MXFP4 only: the block exponent is the smallest e with amax_b <= 6 * 2^e (the
+ * block maximum maps onto the largest code without clipping; "TORQ" sect. 2,
+ * S-step) instead of floor(log2 amax_b) - 2, at most 125 so that no
+ * reconstruction overflows fp32.  It differs exactly when amax_b's significand
+ * exceeds 1.5.  Stored and decoded as MXFP4. */
+#define FP4Q_FLAG_MX_CEIL_SCALE 0x2u
 
 /* The stream type is CUDA's cudaStream_t (a CUstream_st*); NULL is the legacy default stream. */
 typedef struct CUstream_st* fp4q_stream_t;

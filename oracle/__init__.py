@@ -149,7 +149,7 @@ def mx_exponent(a: float) -> int:
 
 
 def mx_exponent_ceil(a: float) -> int:
-    """Smallest e with a <= 6 * 2^e, clamped to [-127, 127] (the no-clipping block exponent)."""
+    """Smallest e with a <= 6 * 2^e, clamped to [-127, 125] (the no-clipping block exponent)."""
     return lib().orc_mx_exponent_ceil(float(a))
 
 

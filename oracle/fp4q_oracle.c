@@ -64,7 +64,9 @@
  *     reconstructions of two quantized matrices, summed in binary64.
  *  R10 MXFP4 exponent without clipping [TORQ sect. 2, S-step: the block
  *     scale maps the block maximum onto the largest code]: e is the smallest
- *     integer with a <= 6 * 2^e, clamped to [-127, 127]; nothing saturates.
+ *     integer with a <= 6 * 2^e, clamped to [-127, 125] so that every
+ *     reconstruction (at most 6 * 2^e) stays finite in binary32; below the
+ *     clamp nothing saturates.
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC
  * -pthread.  Floating point is IEEE binary32/binary64 with round-to-nearest
@@ -259,7 +261,7 @@ int orc_mx_exponent_ceil(float a)
     int e = k - 4;                 /* 6 * 2^(k-4) < 2^k / 2: too small */
     while ((double)a > 6.0 * ldexp(1.0, e)) ++e;
     if (e < -127) e = -127;
-    if (e > 127) e = 127;
+    if (e > 125) e = 125;
     return e;
 }
 

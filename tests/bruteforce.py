@@ -189,7 +189,8 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool, pair2: float 
                 if a == 0:
                     continue
                 if fmt == "mxfp4_ceil":   # the smallest exponent whose 6 * 2^e holds the block maximum
-                    e = min(k for k in range(-127, 128) if Fraction(float(a)) <= 6 * Fraction(2) ** k)
+                    e = min((k for k in range(-127, 126) if Fraction(float(a)) <= 6 * Fraction(2) ** k),
+                            default=125)
                 else:
                     e = max(-127, min(127, floor_log2(float(a)) - 2))
                 scales[r, b] = e + 127

@@ -56,7 +56,8 @@ def q(**kw):
     (dict(fmt=3, cols=40, ldx=40), "FP4Q_ERROR_SHAPE"),          # weight mode: blocks of 16
     (dict(fmt=3, tensor_scale=None), "FP4Q_ERROR_INVALID_VALUE"),  # weight mode needs it
     (dict(rotate=2), "FP4Q_ERROR_INVALID_VALUE"),
-    (dict(flags=2), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(flags=2), "FP4Q_ERROR_INVALID_VALUE"),                # the MX exponent flag needs MXFP4
+    (dict(flags=4), "FP4Q_ERROR_INVALID_VALUE"),
     (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
     (dict(cols=40, ldx=40), "FP4Q_ERROR_SHAPE"),                 # not a multiple of 16
     (dict(fmt=2, cols=48, ldx=48), "FP4Q_ERROR_SHAPE"),          # MXFP4 needs 32
@@ -89,6 +90,7 @@ def test_quantize_argument_rules_that_relax():
     assert q(fmt=2, tensor_scale=None) in ok_then_device
     assert q(flags=1, workspace=None, workspace_bytes=0) in ok_then_device
     assert q(fmt=3, cols=48, ldx=48) in ok_then_device           # weight mode: 16-element blocks
+    assert q(fmt=2, flags=2, tensor_scale=None) in ok_then_device  # MXFP4 with the ceil exponent
 
 
 def _no_gpu() -> bool:

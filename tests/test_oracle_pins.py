@@ -625,16 +625,17 @@ def _mx_ceil_points():
 
 
 def test_mx_exponent_ceil_equals_exhaustive_minimum(orc):
-    """e = min{e in [-127, 127] : a <= 6 * 2^e}, by enumeration with exact rationals."""
+    """e = min{e in [-127, 125] : a <= 6 * 2^e} (125 if none), by enumeration with exact rationals."""
     for a in _mx_ceil_points():
         fa = Fraction(float(a))
-        want = min((k for k in range(-127, 128) if fa <= 6 * Fraction(2) ** k), default=127)
+        want = min((k for k in range(-127, 126) if fa <= 6 * Fraction(2) ** k), default=125)
         assert orc.mx_exponent_ceil(float(a)) == want, a
 
 
 def test_mx_exponent_ceil_closed_forms(orc):
     assert orc.mx_exponent_ceil(6.0) == 0 and orc.mx_exponent_ceil(3.0) == -1 and orc.mx_exponent_ceil(4.0) == 0
     assert orc.mx_exponent_ceil(float(np.nextafter(np.float32(6), np.float32(7)))) == 1
+    assert orc.mx_exponent_ceil(3.3895313892515355e38) == 125       # the clamp: 4 * 2^126 would overflow
     # differs from the floor rule exactly when the block maximum's mantissa exceeds 1.5
     for k in range(-30, 30):
         for m, up in ((1.0, 0), (1.5, 0), (1.5000001, 1), (1.75, 1), (1.99, 1)):

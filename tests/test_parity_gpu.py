@@ -35,7 +35,7 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return synthetic.bf16_bits(t)
 
 
-def run_gpu(x: torch.Tensor, fmt, rotate, tensor_scale=None, want_mse=True, guard=64):
+def run_gpu(x: torch.Tensor, fmt, rotate, tensor_scale=None, want_mse=True, guard=64, extra_flags=0):
     """Quantize through the C ABI into guarded buffers; check the guards; return numpy results."""
     rows, cols = x.shape
     B = fp4q.block_size(fmt)
@@ -50,7 +50,7 @@ def run_gpu(x: torch.Tensor, fmt, rotate, tensor_scale=None, want_mse=True, guar
     mse = torch.full((1,), -1.0, dtype=torch.float64, device=dev) if want_mse else None
     ws = torch.empty(fp4q.fp4q_workspace_size(rows, cols, fmt, rotate), dtype=torch.uint8, device=dev)
     ld = x.stride(0) if rows > 1 else cols
-    flags = fp4q.FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0
+    flags = (fp4q.FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0) | extra_flags
     st = fp4q.fp4q_quantize(x, rows, cols, ld, fmt, rotate, flags, codes, scales, ts, mse, ws, ws.numel())
     assert st == 0, fp4q.fp4q_status_string(st)
     torch.cuda.synchronize()
@@ -413,3 +413,103 @@ def test_llama3_70b_mlp_sampled(orc, dev, fmt):
     name, r, c = synthetic.LLAMA3_70B_MLP[2]
     x = synthetic.mlp_row_scaled(r, c, seed=3, device=dev)
     _sampled_rows_check(orc, x, fmt, nrows=16)
+
+
+# ------------------------------------------------------------------ MXFP4 exponent without clipping
+
+def check_mx_ceil(orc, x: torch.Tensor, rotate=False):
+    """GPU MXFP4 with FP4Q_FLAG_MX_CEIL_SCALE against the oracle's "mxfp4_ceil"."""
+    xb = bits(x)
+    n = x.numel()
+    codes, scales, _, mse = run_gpu(x, "mxfp4", rotate, extra_flags=fp4q.FLAG_MX_CEIL_SCALE)
+    rc, rs, _, rsse = orc.quantize(xb, "mxfp4_ceil", rotate)
+    if not rotate:
+        assert np.array_equal(scales, rs) and np.array_equal(codes, rc)
+        assert rel(mse, rsse / n) <= 1e-5 or (mse == 0.0 and rsse == 0.0)
+        y = run_dequant(codes, scales, 0.0, x.shape[0], x.shape[1], "mxfp4", False, x.device)
+        _, ry = orc.dequantize(rc, rs, 0.0, "mxfp4_ceil", False)
+        assert np.array_equal(y, ry)
+    else:
+        assert rel(mse, rsse / n) <= 1e-3
+        nib = np.stack([codes & 15, codes >> 4], -1).reshape(x.shape)
+        rnib = np.stack([rc & 15, rc >> 4], -1).reshape(x.shape)
+        bad = (nib != rnib) | np.repeat(scales != rs, 32, axis=1)
+        assert bad.mean() <= 1e-4
+    return codes, scales, mse
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_mxfp4_ceil_activation_t3(orc, dev, rotate):
+    x = synthetic.activation_t3(2048, 4096, seed=31, device="cpu").to(dev)
+    _, scales, mse_c = check_mx_ceil(orc, x, rotate)
+    _, scales_f, _, _ = run_gpu(x, "mxfp4", rotate)
+    assert np.all(scales >= scales_f) and np.any(scales > scales_f)
+
+
+@pytest.mark.parametrize("shape", [(1, 32), (7, 160), (33, 224), (1, 4096 + 32)])
+def test_mxfp4_ceil_small_shapes_and_extremes(orc, dev, shape):
+    check_mx_ceil(orc, synthetic.llm_weight(*shape, seed=sum(shape), device="cpu").to(dev))
+    rng = np.random.default_rng(9)
+    big = rng.standard_normal((4, 64)) * 1e37
+    big[1, 3] = 3.3895313892515355e38
+    check_mx_ceil(orc, _bf(big).to(dev))
+    sub = rng.integers(1, 128, size=(4, 64)) * 2.0 ** -133 * rng.choice([-1, 1], size=(4, 64))
+    check_mx_ceil(orc, _bf(sub).to(dev))
+    m = np.array([1.0, 1.5, 1.5078125, 1.75, 1.9921875])           # significands around 1.5
+    blocks = np.repeat(m[:, None], 32, axis=1) * 0.01
+    check_mx_ceil(orc, _bf(blocks.reshape(1, -1)).to(dev))
+
+
+def test_mxfp4_ceil_batch_equals_per_tensor(dev):
+    xs = [synthetic.activation_t3(r, c, seed=40 + r, device=dev) for r, c in ((64, 256), (300, 1024), (5, 4096))]
+    got = fp4q.quantize_batch(xs, "mxfp4", False, mx_ceil=True)
+    for x, g in zip(xs, got):
+        w = fp4q.quantize(x, "mxfp4", False, mx_ceil=True)
+        torch.cuda.synchronize()
+        assert torch.equal(g.codes, w.codes) and torch.equal(g.scales, w.scales)
+        assert abs(g.mse.item() - w.mse.item()) <= 1e-12 * w.mse.item()
+
+
+def test_single_level_nvfp4_full_size_sampled(orc, dev):
+    """Single-level NVFP4 (tensor scale 1): N(0, 0.02^2) weights take E4M3 subnormal
+    block scales; a 14336 x 4096 tensor, sampled rows against the oracle."""
+    name, r, c = synthetic.LLAMA3_8B_LAYER[4]
+    x = synthetic.llm_weight(r, c, seed=synthetic.tensor_seed(2, 0, 4), device=dev)
+    for fmt in ("nvfp4", "nvfp4_razer"):
+        ts = torch.ones(1, dtype=torch.float32, device=dev)
+        q = fp4q.quantize(x, fmt, tensor_scale=ts)
+        torch.cuda.synchronize()
+        pick = np.array([0, 1, 777, r // 2, r - 1])
+        idx = torch.from_numpy(pick).to(dev)
+        rc, rs, _, _ = orc.quantize(bits(x[idx]), fmt, False, tensor_scale=1.0, want_sse=False)
+        assert np.array_equal(q.codes[idx].cpu().numpy(), rc) and np.array_equal(q.scales[idx].cpu().numpy(), rs)
+        assert np.mean((rs & 0x7F) < 0x08) > 0.5                       # most block scales are E4M3 subnormals
+        e = fp4q.error(x, q, fmt)
+        torch.cuda.synchronize()
+        assert rel(q.mse.item(), e.item()) <= 1e-6
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "nvfp4_razer_w"])
+def test_rotated_nvfp4_full_size_sampled(orc, dev, fmt):
+    """Rotated NVFP4 formats on a full 14336 x 4096 tensor: the tensor scale from the
+    rotated absmax, and sampled rows against the oracle (rotated tolerance)."""
+    name, r, c = synthetic.LLAMA3_8B_LAYER[5]
+    x = synthetic.llm_weight(r, c, seed=synthetic.tensor_seed(2, 0, 5), device=dev)
+    q = fp4q.quantize(x, fmt, rotate=True)
+    torch.cuda.synchronize()
+    amax = 0.0
+    for r0 in range(0, r, 4096):
+        amax = max(amax, orc.tensor_amax(bits(x[r0:r0 + 4096]), rotate=True))
+    ts = orc.tensor_scale_from_amax(amax, fmt)
+    assert rel(q.tensor_scale.item(), float(ts)) <= 1e-6
+    pick = np.unique(np.concatenate([[0, r - 1], np.random.default_rng(5).choice(r, 48, replace=False)]))
+    idx = torch.from_numpy(pick).to(dev)
+    rc, rs, _, _ = orc.quantize(bits(x[idx]), fmt, True, tensor_scale=q.tensor_scale.item(), want_sse=False)
+    codes, scales = q.codes[idx].cpu().numpy(), q.scales[idx].cpu().numpy()
+    nib = np.stack([codes & 15, codes >> 4], -1).reshape(len(pick), c)
+    rnib = np.stack([rc & 15, rc >> 4], -1).reshape(len(pick), c)
+    bad = (nib != rnib) | np.repeat(scales != rs, 16, axis=1)
+    assert bad.mean() <= 1e-4
+    e = fp4q.error(x, q, fmt, rotate=True)
+    torch.cuda.synchronize()
+    assert rel(q.mse.item(), e.item()) <= 1e-4
