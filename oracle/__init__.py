@@ -82,6 +82,12 @@ def lib() -> ctypes.CDLL:
         L.orc_mma_scale_byte.argtypes = [i32, i32]; L.orc_mma_scale_byte.restype = i32
         L.orc_mma_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp]; L.orc_mma_pack.restype = i32
         L.orc_gemm.argtypes = [vp, vp, i64, i64, i64, vp, vp, i32]; L.orc_gemm.restype = i32
+        L.orc_f64_to_bf16.argtypes = [f64]; L.orc_f64_to_bf16.restype = ctypes.c_uint16
+        L.orc_f32_to_f16_sat.argtypes = [f32]; L.orc_f32_to_f16_sat.restype = ctypes.c_uint16
+        L.orc_f16_value.argtypes = [ctypes.c_uint16]; L.orc_f16_value.restype = f64
+        L.orc_outlier_capacity.argtypes = [i64, f64]; L.orc_outlier_capacity.restype = i64
+        L.orc_separate_outliers.argtypes = [vp, i64, i64, i64, f64, i64, vp, vp, vp, vp, vp, vp]
+        L.orc_separate_outliers.restype = i32
     return _lib
 
 
@@ -307,3 +313,39 @@ def gemm(a: np.ndarray, w: np.ndarray, nthreads: int | None = None):
     yabs = np.empty((M, N), dtype=np.float64)
     lib().orc_gemm(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(yabs), nthreads or default_threads())
     return y, yabs
+
+
+# ---------------------------------------------------------------- sparse outlier separation
+
+def f64_to_bf16(v: float) -> int:
+    return lib().orc_f64_to_bf16(float(v))
+
+
+def f32_to_f16_sat(v: float) -> int:
+    return lib().orc_f32_to_f16_sat(float(v))
+
+
+def f16_value(h: int) -> float:
+    return lib().orc_f16_value(int(h))
+
+
+def outlier_capacity(cols: int, max_frac: float = 0.02) -> int:
+    return lib().orc_outlier_capacity(int(cols), float(max_frac))
+
+
+def separate_outliers(x: np.ndarray, k: float = 4.0, max_frac: float = 0.02):
+    """Return ``(bulk u16 [rows, cols], cols u16 [rows, cap], vals f16-bits u16 [rows, cap],
+    count i32 [rows], mu f64 [rows], thr f64 [rows])``."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    cap = outlier_capacity(cols, max_frac)
+    bulk = np.empty((rows, cols), dtype=np.uint16)
+    oc = np.zeros((rows, max(cap, 1)), dtype=np.uint16)
+    ov = np.zeros((rows, max(cap, 1)), dtype=np.uint16)
+    cnt = np.zeros(rows, dtype=np.int32)
+    mu = np.zeros(rows, dtype=np.float64)
+    thr = np.zeros(rows, dtype=np.float64)
+    if lib().orc_separate_outliers(_ptr(x), rows, cols, x.strides[0] // 2, float(k), cap, _ptr(bulk), _ptr(oc),
+                                   _ptr(ov), _ptr(cnt), _ptr(mu), _ptr(thr)) != 0:
+        raise ValueError("oracle rejected shape")
+    return bulk, oc[:, :cap], ov[:, :cap], cnt, mu, thr

@@ -62,6 +62,17 @@
  *     (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
  *  R9 W4A4 product: Y = A^ W^T for A^ (M x K) and W^ (N x K) the fp32
  *     reconstructions of two quantized matrices, summed in binary64.
+ *  R11 sparse outlier separation ["XFP: quality-targeted adaptive codebook
+ *     quantization", technical summary sect. 2, sparse outlier separation:
+ *     weights with |w - mu| > k sigma (k = 4 by default, at most 2 % of the
+ *     weights) are kept apart in fp16 at their positions, and the bulk holds
+ *     the group mean there before it is quantized]: the group is a row;
+ *     mu = (sum of the row, in order) / n and sigma = sqrt(sum (x - mu)^2 / n)
+ *     in binary64; with d = |x - mu| the candidates are d > k sigma; when more
+ *     than cap = floor(max_frac * n) qualify, the cap largest d are kept, ties
+ *     to the lower column; kept values are stored as fp16 (nearest even,
+ *     saturating at 65504) in column order, and the bulk row is x with every
+ *     kept position set to RN_bf16(mu).
  *  R10 MXFP4 exponent without clipping [TORQ sect. 2, S-step: the block
  *     scale maps the block maximum onto the largest code]: e is the smallest
  *     integer with a <= 6 * 2^e, clamped to [-127, 125] so that every
@@ -784,5 +795,128 @@ int orc_gemm(const float* a, const float* w, int64_t M, int64_t N, int64_t K, do
     }
     for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
     free(jobs); free(th);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sparse outlier separation (R11)                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Round |v| to a multiple of the quantum 2^qexp, nearest, ties to even multiple. */
+static double round_to_quantum(double a, int qexp)
+{
+    double q = ldexp(a, -qexp);           /* exact: power-of-two scaling */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    return ldexp(r, qexp);
+}
+
+/* binary64 -> bf16 bits, nearest even (8 significant bits, subnormal quantum 2^-133). */
+uint16_t orc_f64_to_bf16(double v)
+{
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+    const double a = fabs(v);
+    int k;
+    (void)frexp(a, &k);                   /* a in [2^(k-1), 2^k) */
+    const int e = k - 1;
+    const double r = round_to_quantum(a, e < -126 ? -133 : e - 7);
+    const uint16_t h = (uint16_t)(bits_from_f32((float)r) >> 16);   /* r is a bf16 value: exact in binary32 */
+    return v < 0.0 ? (uint16_t)(h | 0x8000u) : h;
+}
+
+/* binary32 -> fp16 bits, nearest even (11 significant bits, subnormal quantum
+ * 2^-24), magnitudes above 65504 saturating to 65504. */
+uint16_t orc_f32_to_f16_sat(float f)
+{
+    const double v = (double)f;
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+    const double a = fabs(v);
+    int k;
+    (void)frexp(a, &k);
+    const int e = k - 1;
+    double r = round_to_quantum(a, e < -14 ? -24 : e - 10);
+    if (r > 65504.0) r = 65504.0;
+    uint16_t h;
+    if (r < ldexp(1.0, -14)) {
+        h = (uint16_t)ldexp(r, 24);       /* subnormal: r / 2^-24 */
+    } else {
+        (void)frexp(r, &k);
+        const int ex = k - 1;
+        h = (uint16_t)(((ex + 15) << 10) | (int)(ldexp(r, 10 - ex) - 1024.0));
+    }
+    return v < 0.0 ? (uint16_t)(h | 0x8000u) : h;
+}
+
+double orc_f16_value(uint16_t h)
+{
+    const int ex = (h >> 10) & 31, m = h & 1023;
+    double a;
+    if (ex == 0) a = ldexp((double)m, -24);
+    else if (ex == 31) a = m ? NAN : INFINITY;
+    else a = ldexp(1.0 + m / 1024.0, ex - 15);
+    return (h & 0x8000u) ? -a : a;
+}
+
+int64_t orc_outlier_capacity(int64_t cols, double max_frac) { return (int64_t)floor(max_frac * (double)cols); }
+
+typedef struct { double d; int64_t j; } cand;
+
+static int cand_order(const void* pa, const void* pb)
+{
+    const cand* a = (const cand*)pa; const cand* b = (const cand*)pb;
+    if (a->d != b->d) return a->d > b->d ? -1 : 1;      /* larger deviation first */
+    return a->j < b->j ? -1 : (a->j > b->j);             /* then the lower column */
+}
+
+static int col_order(const void* pa, const void* pb)
+{
+    const cand* a = (const cand*)pa; const cand* b = (const cand*)pb;
+    return a->j < b->j ? -1 : (a->j > b->j);
+}
+
+/* R11 on a rows x cols bf16 matrix (row stride ldx): bulk (rows x cols bf16,
+ * dense), outlier columns and fp16 values ([rows][cap], column order) and the
+ * count per row.  Also returns each row's mu and k sigma when mu / thr are
+ * non-null. */
+int orc_separate_outliers(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, double k, int64_t cap,
+                          uint16_t* bulk, uint16_t* out_cols, uint16_t* out_vals, int32_t* out_count,
+                          double* mu_out, double* thr_out)
+{
+    if (rows < 0 || cols <= 0 || ldx < cols || cap < 0 || cols > 65536) return -1;
+    cand* c = (cand*)malloc(sizeof(cand) * (size_t)cols);
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * ldx;
+        double s = 0.0;
+        for (int64_t j = 0; j < cols; ++j) s += (double)orc_bf16_to_f32(xr[j]);
+        const double mu = s / (double)cols;
+        double v = 0.0;
+        for (int64_t j = 0; j < cols; ++j) {
+            const double t = (double)orc_bf16_to_f32(xr[j]) - mu;
+            v += t * t;
+        }
+        const double thr = k * sqrt(v / (double)cols);
+        int64_t n = 0;
+        for (int64_t j = 0; j < cols; ++j) {
+            const double d = fabs((double)orc_bf16_to_f32(xr[j]) - mu);
+            if (d > thr) c[n++] = (cand){d, j};
+        }
+        if (n > cap) {
+            qsort(c, (size_t)n, sizeof(cand), cand_order);
+            n = cap;
+        }
+        qsort(c, (size_t)n, sizeof(cand), col_order);
+        const uint16_t mub = orc_f64_to_bf16(mu);
+        for (int64_t j = 0; j < cols; ++j) bulk[r * cols + j] = xr[j];
+        for (int64_t i = 0; i < n; ++i) {
+            bulk[r * cols + c[i].j] = mub;
+            out_cols[r * cap + i] = (uint16_t)c[i].j;
+            out_vals[r * cap + i] = orc_f32_to_f16_sat(orc_bf16_to_f32(xr[c[i].j]));
+        }
+        out_count[r] = (int32_t)n;
+        if (mu_out) mu_out[r] = mu;
+        if (thr_out) thr_out[r] = thr;
+    }
+    free(c);
     return 0;
 }

@@ -656,3 +656,100 @@ def test_mxfp4_ceil_never_saturates_and_decodes_as_mxfp4(orc):
     scale = 2.0 ** (s.astype(np.float64) - 127)
     assert np.all(blocks <= 6 * scale)                  # the block maximum fits: no element saturates
     assert sse_c != sse_f
+
+
+# ---------------------------------------------------------------- sparse outlier separation
+
+def _rn_fraction(v: Fraction, quantum: Fraction) -> Fraction:
+    q = v / quantum
+    r = math.floor(q)
+    frac = q - r
+    if frac > Fraction(1, 2) or (frac == Fraction(1, 2) and r % 2):
+        r += 1
+    return r * quantum
+
+
+def test_f64_to_bf16_is_exact_nearest_even(orc):
+    rng = np.random.default_rng(50)
+    vals = list(rng.standard_normal(300) * 10.0 ** rng.integers(-40, 38, 300))
+    for e in (-130, -20, 0, 5):                        # ties and their neighbours
+        for m in (1 + 1 / 256, 1 + 3 / 256, 1.5 + 1 / 256):
+            t = m * 2.0 ** e
+            vals += [t, np.nextafter(t, 0), np.nextafter(t, 10)]
+    for v in vals:
+        fv = Fraction(float(v))
+        e = math.floor(math.log2(abs(float(v))))
+        if Fraction(2) ** (e + 1) <= abs(fv):
+            e += 1
+        if Fraction(2) ** e > abs(fv):
+            e -= 1
+        want = _rn_fraction(abs(fv), Fraction(2) ** (-133 if e < -126 else e - 7))
+        got = orc.f64_to_bf16(float(v))
+        gv = float(np.array([got], np.uint16).view(ml_dtypes.bfloat16)[0])
+        assert Fraction(abs(gv)) == want and (gv < 0) == (v < 0), v
+
+
+def test_f32_to_f16_saturating_matches_numpy(orc):
+    rng = np.random.default_rng(51)
+    vals = np.concatenate([rng.standard_normal(2000).astype(np.float32) * np.float32(10.0) ** rng.integers(-9, 5, 2000),
+                           np.float32([65504, 65519.99, 65520, 7e4, -1e6, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                                       6.1e-5, -0.0, 0.0])])
+    for v in vals:
+        got = orc.f32_to_f16_sat(float(v))
+        ref = np.float16(v) if abs(v) < 65520 else np.float16(np.sign(v) * 65504)
+        assert got == int(np.array([ref]).view(np.uint16)[0]), v
+        assert orc.f16_value(got) == float(ref)
+
+
+def test_outliers_closed_form_rows(orc):
+    """Rows of n - m zeros and m spikes of height h: mu = m h / n, sigma = h sqrt(m (n - m)) / n,
+    and the spikes are outliers exactly when (n - m) / sqrt(m (n - m)) > k."""
+    n = 256
+    rows = []
+    for m in (1, 3, 8, 16, 40):
+        row = np.zeros(n, np.float32)
+        row[np.arange(m) * 5 + 2] = 0.5
+        rows.append(row)
+    x = np.array(rows).astype(ml_dtypes.bfloat16).view(np.uint16)
+    bulk, oc, ov, cnt, mu, thr = orc.separate_outliers(x, k=4.0, max_frac=0.02)
+    cap = orc.outlier_capacity(n, 0.02)
+    assert cap == 5
+    for i, m in enumerate((1, 3, 8, 16, 40)):
+        assert mu[i] == m * 0.5 / n
+        is_out = (n - m) / math.sqrt(m * (n - m)) > 4.0
+        expect = min(m, cap) if is_out else 0
+        assert cnt[i] == expect, (m, cnt[i])
+        cols = oc[i, :cnt[i]]
+        assert list(cols) == list((np.arange(m) * 5 + 2)[:expect])    # ties: the lowest columns
+        assert all(orc.f16_value(v) == 0.5 for v in ov[i, :cnt[i]])
+        b = bulk[i].view(ml_dtypes.bfloat16).astype(np.float64)
+        assert np.all(b[cols] == float(np.array([orc.f64_to_bf16(mu[i])], np.uint16).view(ml_dtypes.bfloat16)[0]))
+
+
+def test_outliers_against_numpy_statistics(orc):
+    """Random LLM-weight rows (with x20 outliers) and rows where the 2 % cap binds:
+    the outlier set equals one built from numpy's mean / std and a sort."""
+    from activation_quantization_block_b200 import synthetic
+    w = synthetic.llm_weight(48, 1024, seed=52).float().numpy()
+    rng = np.random.default_rng(53)
+    w[40:] *= np.where(rng.random((8, 1024)) < 0.1, 20.0, 1.0)      # 10 % spikes: the cap binds
+    x = w.astype(ml_dtypes.bfloat16).view(np.uint16)
+    xf = x.view(ml_dtypes.bfloat16).astype(np.float64)
+    bulk, oc, ov, cnt, mu, thr = orc.separate_outliers(x, k=4.0, max_frac=0.02)
+    cap = orc.outlier_capacity(1024, 0.02)
+    bound = 0
+    for r in range(48):
+        m, s = np.mean(xf[r]), np.std(xf[r])
+        assert abs(m - mu[r]) <= 1e-12 * np.abs(xf[r]).max() and abs(4 * s - thr[r]) <= 1e-12 * thr[r]
+        d = np.abs(xf[r] - m)
+        cand = np.nonzero(d > 4 * s)[0]
+        if len(cand) > cap:
+            bound += 1
+            order = sorted(cand, key=lambda j: (-d[j], j))
+            cand = np.sort(order[:cap])
+        assert list(oc[r, :cnt[r]]) == list(cand)
+        assert np.array_equal(ov[r, :cnt[r]], xf[r, cand].astype(np.float16).view(np.uint16))
+        keep = np.ones(1024, bool)
+        keep[cand] = False
+        assert np.array_equal(bulk[r, keep], x[r, keep])
+    assert bound >= 4                                              # rows where the cap binds
