@@ -223,6 +223,50 @@ fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
     return FP4Q_SUCCESS;
 }
 
+int64_t fp4q_outlier_capacity(int64_t cols, double max_frac)
+{
+    if (cols < 0 || !(max_frac >= 0.0 && max_frac <= 1.0)) return 0;
+    return outlier_capacity(cols, max_frac);
+}
+
+fp4q_status_t fp4q_separate_outliers(const void* x, int64_t rows, int64_t cols, int64_t ldx, double k,
+                                     double max_frac, void* bulk, int64_t ldb, uint16_t* out_cols,
+                                     uint16_t* out_vals, int32_t* out_count, fp4q_stream_t stream)
+{
+    if (rows < 0 || cols < 0 || !(k > 0.0 && k < 1e300) || !(max_frac >= 0.0 && max_frac <= 1.0))
+        return FP4Q_ERROR_INVALID_VALUE;
+    if (cols % 8 != 0 || cols > 65536 || rows >= ((int64_t)1 << 31)) return FP4Q_ERROR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_SUCCESS;
+    fp4q_status_t s;
+    if ((s = check_matrix(x, cols, ldx)) != FP4Q_SUCCESS) return s;
+    if ((s = check_matrix(bulk, cols, ldb)) != FP4Q_SUCCESS) return s;
+    const int64_t cap = outlier_capacity(cols, max_frac);
+    if (out_count == nullptr || (cap > 0 && (out_cols == nullptr || out_vals == nullptr)))
+        return FP4Q_ERROR_INVALID_VALUE;
+    if (!aligned(out_count, 4) || !aligned(out_cols, 2) || !aligned(out_vals, 2)) return FP4Q_ERROR_MISALIGNED;
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_separate_outliers(static_cast<const uint16_t*>(x), rows, cols, ldx, k, cap,
+                                              static_cast<uint16_t*>(bulk), ldb, out_cols, out_vals, out_count,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status_t fp4q_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals, const int32_t* out_count,
+                                    int64_t rows, int64_t cols, int64_t cap, void* y, int64_t ldy,
+                                    fp4q_stream_t stream)
+{
+    if (rows < 0 || cols < 0 || cap < 0 || cap > cols) return FP4Q_ERROR_INVALID_VALUE;
+    if (rows == 0 || cap == 0) return FP4Q_SUCCESS;
+    if (out_cols == nullptr || out_vals == nullptr || out_count == nullptr || y == nullptr)
+        return FP4Q_ERROR_INVALID_VALUE;
+    if (ldy < cols) return FP4Q_ERROR_SHAPE;
+    if (!aligned(y, 2) || !aligned(out_count, 4) || !aligned(out_cols, 2) || !aligned(out_vals, 2))
+        return FP4Q_ERROR_MISALIGNED;
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_scatter_outliers(out_cols, out_vals, out_count, rows, cap, static_cast<uint16_t*>(y),
+                                             ldy, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp4q_mma_planes(fp4q_format_t fmt)
 {
     if (fmt == FP4Q_NVFP4) return 1;

@@ -69,6 +69,14 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
                              int64_t N, int64_t K, uint16_t* y, int64_t ldy, cudaStream_t st);
 cudaError_t read_gemm_device_errors(unsigned int* bits, bool clear);
 
+// Sparse outlier separation (fp4q_outliers.cu).
+int64_t outlier_capacity(int64_t cols, double max_frac);
+cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, double k, int64_t cap,
+                                     uint16_t* bulk, int64_t ldb, uint16_t* out_cols, uint16_t* out_vals,
+                                     int32_t* out_count, cudaStream_t st);
+cudaError_t launch_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals, const int32_t* out_count,
+                                    int64_t rows, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st);
+
 // Tile count of a bf16 matrix's view (see make_view): 16 KB tiles.
 int64_t view_tiles(const Geometry& g);
 

@@ -1,0 +1,291 @@
+// Sparse outlier separation ahead of block quantization, and the scatter that
+// puts the outliers back into a reconstruction.
+//
+// "XFP: quality-targeted adaptive codebook quantization", technical summary
+// sect. 2 (sparse outlier separation): weights with |w - mu| > k sigma (k = 4,
+// at most 2 % of the weights) are kept apart as fp16 values at their
+// positions, and the bulk, with the group mean in their place, is quantized.
+// The group is a matrix row.  One CTA per row:
+//   1. mu = sum / n and sigma = sqrt(sum (x - mu)^2 / n) in fp64 (fixed-order
+//      CTA reductions), threshold T = k sigma;
+//   2. c = #(|x - mu| > T); when c exceeds cap = floor(max_frac * n), T becomes
+//      the cap-th largest deviation, found by bisection on the deviations' fp64
+//      bit patterns (monotone for non-negative values), and the ties at T are
+//      taken from the lowest columns up;
+//   3. one pass in tiles of 2048 elements writes the bulk row (the mean, rounded
+//      to bf16, at every outlier) and the outliers in column order, their slots
+//      from CTA-wide prefix counts.
+// Rows are read from global memory on every pass (L2 keeps a row: at most
+// 128 KB); each thread moves 16 bytes at a time.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp4q_common.cuh"
+
+namespace fp4q {
+
+namespace {
+
+constexpr int kOutThreads = 256;
+constexpr int kOutTile = kOutThreads * 8;   // elements per tile: 8 per thread
+
+struct OutlierArgs {
+    const uint16_t* x;
+    uint16_t* bulk;
+    uint16_t* out_cols;
+    uint16_t* out_vals;
+    int32_t* out_count;
+    int64_t ldx, ldb, cols, cap;
+    double k;
+};
+
+// Sum over the CTA in a fixed order, result in every thread.
+__device__ double cta_sum(double v, double* sh)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < kOutThreads / 32 ? sh[lane] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (lane == 0) sh[32] = v;
+    }
+    __syncthreads();
+    return sh[32];
+}
+
+__device__ long long cta_count(long long v, long long* sh)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < kOutThreads / 32 ? sh[lane] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (lane == 0) sh[32] = v;
+    }
+    __syncthreads();
+    return sh[32];
+}
+
+// Exclusive prefix of v over the CTA in thread order; *total receives the sum.
+__device__ int cta_exclusive_scan(int v, int* sh, int* total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    __syncthreads();
+    if (lane == 31) sh[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kOutThreads / 32 ? sh[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        if (lane < kOutThreads / 32) sh[lane] = wi - w;   // exclusive warp offsets
+        if (lane == kOutThreads / 32 - 1) sh[32] = wi;
+    }
+    __syncthreads();
+    *total = sh[32];
+    return sh[warp] + inc - v;
+}
+
+// Eight bf16 values of x[row] starting at column j (j % 8 == 0), as fp32.
+__device__ __forceinline__ void load8(const uint16_t* row, int64_t j, float* v)
+{
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + j));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16_lo(u[i]);
+        v[2 * i + 1] = bf16_hi(u[i]);
+    }
+}
+
+// binary64 -> bf16 bits, nearest even: truncate to binary32 and, if inexact,
+// set its last bit (round to odd), then round to bf16; binary32 keeps 16 bits
+// more than bf16, so the two roundings equal one.
+__device__ __forceinline__ uint16_t f64_to_bf16_rn(double m)
+{
+    float f = __double2float_rz(m);
+    if ((double)f != m) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a)
+{
+    __shared__ double shd[33];
+    __shared__ long long shl[33];
+    __shared__ int shi[33];
+    const int64_t r = blockIdx.x;
+    const uint16_t* row = a.x + r * a.ldx;
+    const int t = threadIdx.x;
+    const int64_t n = a.cols;
+
+    // 1. mean and deviation
+    double s = 0.0;
+    for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
+        float v[8];
+        load8(row, j, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += (double)v[i];
+    }
+    const double mu = cta_sum(s, shd) / (double)n;
+    s = 0.0;
+    for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
+        float v[8];
+        load8(row, j, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = (double)v[i] - mu;
+            s += d * d;
+        }
+    }
+    double thr = a.k * sqrt(cta_sum(s, shd) / (double)n);
+
+    // 2. count; above the cap, the cap-th largest deviation and its ties
+    auto count_where = [&](auto pred) {
+        long long c = 0;
+        for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
+            float v[8];
+            load8(row, j, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c += pred(fabs((double)v[i] - mu)) ? 1 : 0;
+        }
+        return cta_count(c, shl);
+    };
+    long long tie_need = 0;
+    if (a.cap == 0) {
+        thr = __longlong_as_double(0x7FF0000000000000ll);   // +inf: no slots, no outliers
+    } else if (count_where([&](double d) { return d > thr; }) > a.cap) {
+        // largest u with #(bits(d) >= u) >= cap: the cap-th largest deviation
+        unsigned long long lo = 0ull, hi = 0x7FF0000000000000ull;   // bits of 0 and of +inf
+        while (hi - lo > 1ull) {
+            const unsigned long long mid = lo + (hi - lo) / 2;
+            const long long c = count_where([&](double d) { return (unsigned long long)__double_as_longlong(d) >= mid; });
+            if (c >= a.cap) lo = mid;
+            else hi = mid;
+        }
+        thr = __longlong_as_double((long long)lo);
+        tie_need = a.cap - count_where([&](double d) { return d > thr; });
+    }
+
+    // 3. bulk row and outliers in column order
+    const uint16_t mub = f64_to_bf16_rn(mu);
+    uint16_t* brow = a.bulk + r * a.ldb;
+    int64_t done = 0, ties_seen = 0;
+    for (int64_t j0 = 0; j0 < n; j0 += kOutTile) {
+        const int64_t j = j0 + 8 * (int64_t)t;
+        const bool in = j < n;
+        float v[8];
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (in) {
+            w = __ldg(reinterpret_cast<const uint4*>(row + j));
+            load8(row, j, v);
+        }
+        int gt = 0, eq = 0;
+        uint32_t gmask = 0, emask = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = in ? fabs((double)v[i] - mu) : -1.0;
+            if (d > thr) { gmask |= 1u << i; ++gt; }
+            else if (d == thr && tie_need > 0) { emask |= 1u << i; ++eq; }
+        }
+        int eq_total;
+        const int eq_before = cta_exclusive_scan(eq, shi, &eq_total);
+        // ties kept: those whose rank among the row's ties is below tie_need
+        uint32_t omask = gmask;
+        int rank = (int)(ties_seen + eq_before);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (emask & (1u << i)) {
+                if (rank < tie_need) omask |= 1u << i;
+                ++rank;
+            }
+        ties_seen += eq_total;
+        const int cnt = __popc(omask);
+        int tot;
+        int slot = (int)done + cta_exclusive_scan(cnt, shi, &tot);
+        if (in) {
+            uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (omask & (1u << i)) {
+                    const uint32_t sh = (i & 1) ? 16u : 0u;
+                    u[i >> 1] = (u[i >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
+                    a.out_cols[r * a.cap + slot] = (uint16_t)(j + i);
+                    a.out_vals[r * a.cap + slot] =
+                        __half_as_ushort(__float2half_rn(fminf(fmaxf(v[i], -65504.0f), 65504.0f)));
+                    ++slot;
+                }
+            *reinterpret_cast<uint4*>(brow + j) = make_uint4(u[0], u[1], u[2], u[3]);
+        }
+        done += tot;
+    }
+    if (t == 0) a.out_count[r] = (int32_t)done;
+}
+
+struct ScatterArgs {
+    const uint16_t* out_cols;
+    const uint16_t* out_vals;
+    const int32_t* out_count;
+    uint16_t* y;
+    int64_t rows, cap, ldy;
+};
+
+// One thread per (row, slot): the slot's fp16 value, as bf16, to its column.
+__global__ void __launch_bounds__(256) outlier_scatter_kernel(ScatterArgs a)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.rows * a.cap) return;
+    const int64_t r = i / a.cap, s = i - r * a.cap;
+    if (s >= a.out_count[r]) return;
+    const float v = __half2float(__ushort_as_half(a.out_vals[i]));
+    a.y[r * a.ldy + a.out_cols[i]] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+}  // namespace
+
+int64_t outlier_capacity(int64_t cols, double max_frac) { return (int64_t)floor(max_frac * (double)cols); }
+
+cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, double k, int64_t cap,
+                                     uint16_t* bulk, int64_t ldb, uint16_t* out_cols, uint16_t* out_vals,
+                                     int32_t* out_count, cudaStream_t st)
+{
+    if (rows == 0) return cudaSuccess;
+    OutlierArgs a{x, bulk, out_cols, out_vals, out_count, ldx, ldb, cols, cap, k};
+    outlier_rows_kernel<<<(unsigned)rows, kOutThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals, const int32_t* out_count,
+                                    int64_t rows, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st)
+{
+    const int64_t n = rows * cap;
+    if (n == 0) return cudaSuccess;
+    const int64_t blocks = (n + 255) / 256;
+    if (blocks >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    ScatterArgs a{out_cols, out_vals, out_count, y, rows, cap, ldy};
+    outlier_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4q

@@ -32,7 +32,8 @@ STATUS_NAMES = {
 ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc",
                "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch",
-               "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm")
+               "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm",
+               "fp4q_outlier_capacity", "fp4q_separate_outliers", "fp4q_scatter_outliers")
 
 
 class TensorDesc(ctypes.Structure):
@@ -89,6 +90,13 @@ def lib() -> ctypes.CDLL:
         L.fp4q_mma_pack.restype = i32
         L.fp4q_gemm.argtypes = [vp, vp, i32, vp, vp, vp, i32, vp, i64, i64, i64, vp, i64, vp]
         L.fp4q_gemm.restype = i32
+        f64 = ctypes.c_double
+        L.fp4q_outlier_capacity.argtypes = [i64, f64]
+        L.fp4q_outlier_capacity.restype = i64
+        L.fp4q_separate_outliers.argtypes = [vp, i64, i64, i64, f64, f64, vp, i64, vp, vp, vp, vp]
+        L.fp4q_separate_outliers.restype = i32
+        L.fp4q_scatter_outliers.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp]
+        L.fp4q_scatter_outliers.restype = i32
         _lib = L
     return _lib
 
@@ -194,6 +202,21 @@ def fp4q_mma_pack(codes, scales, rows, cols, fmt, planes, sf, stream=None) -> in
 def fp4q_gemm(a_planes, a_sf, a_np, a_scale, w_planes, w_sf, w_np, w_scale, M, N, K, y, ldy, stream=None) -> int:
     return lib().fp4q_gemm(_ptr(a_planes), _ptr(a_sf), a_np, _ptr(a_scale), _ptr(w_planes), _ptr(w_sf), w_np,
                            _ptr(w_scale), M, N, K, _ptr(y), ldy, _stream(stream))
+
+
+def fp4q_outlier_capacity(cols: int, max_frac: float) -> int:
+    return lib().fp4q_outlier_capacity(cols, max_frac)
+
+
+def fp4q_separate_outliers(x, rows, cols, ldx, k, max_frac, bulk, ldb, out_cols, out_vals, out_count,
+                           stream=None) -> int:
+    return lib().fp4q_separate_outliers(_ptr(x), rows, cols, ldx, k, max_frac, _ptr(bulk), ldb, _ptr(out_cols),
+                                        _ptr(out_vals), _ptr(out_count), _stream(stream))
+
+
+def fp4q_scatter_outliers(out_cols, out_vals, out_count, rows, cols, cap, y, ldy, stream=None) -> int:
+    return lib().fp4q_scatter_outliers(_ptr(out_cols), _ptr(out_vals), _ptr(out_count), rows, cols, cap, _ptr(y),
+                                       ldy, _stream(stream))
 
 
 def tensor_desc(x, q: "Quantized") -> TensorDesc:
@@ -354,4 +377,34 @@ def gemm(a: MmaOperand, w: MmaOperand, out: torch.Tensor | None = None, stream=N
     ldy = y.stride(0) if M > 1 else N
     _check(fp4q_gemm(a.planes, a.sf, a.nplanes, a.tensor_scale, w.planes, w.sf, w.nplanes, w.tensor_scale, M, N, K,
                      y, ldy, stream), "fp4q_gemm")
+    return y
+
+
+class Outliers(NamedTuple):
+    bulk: torch.Tensor       # bf16 [rows, cols]: x with the row mean at every outlier
+    cols: torch.Tensor       # int16 (uint16 bit patterns) [rows, cap]
+    vals: torch.Tensor       # float16 [rows, cap]
+    count: torch.Tensor      # int32 [rows]
+
+
+def separate_outliers(x: torch.Tensor, k: float = 4.0, max_frac: float = 0.02, stream=None) -> Outliers:
+    """Sparse outlier separation of a bf16 CUDA matrix (rows are the groups)."""
+    rows, cols, ld = _rows_cols_ld(x)
+    cap = fp4q_outlier_capacity(cols, max_frac)
+    dev = x.device
+    o = Outliers(torch.empty(rows, cols, dtype=torch.bfloat16, device=dev),
+                 torch.zeros(rows, max(cap, 1), dtype=torch.int16, device=dev),
+                 torch.zeros(rows, max(cap, 1), dtype=torch.float16, device=dev),
+                 torch.zeros(rows, dtype=torch.int32, device=dev))
+    _check(fp4q_separate_outliers(x, rows, cols, ld, k, max_frac, o.bulk, cols, o.cols, o.vals, o.count, stream),
+           "fp4q_separate_outliers")
+    return o
+
+
+def scatter_outliers(o: Outliers, y: torch.Tensor, max_frac: float = 0.02, stream=None) -> torch.Tensor:
+    """Put the outliers of o back into the bf16 reconstruction y (in place)."""
+    rows, cols = y.shape
+    cap = fp4q_outlier_capacity(cols, max_frac)
+    ldy = y.stride(0) if rows > 1 else cols
+    _check(fp4q_scatter_outliers(o.cols, o.vals, o.count, rows, cols, cap, y, ldy, stream), "fp4q_scatter_outliers")
     return y

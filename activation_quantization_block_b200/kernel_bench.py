@@ -33,7 +33,7 @@ from . import fp4q, synthetic
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["quantize", "dequantize", "error", "gemm"], default="quantize")
+    p.add_argument("--op", choices=["quantize", "dequantize", "error", "gemm", "outliers"], default="quantize")
     p.add_argument("--fmt", choices=list(fp4q.FORMATS), default="nvfp4_razer")
     p.add_argument("--rows", type=int, default=14336)
     p.add_argument("--cols", type=int, default=4096)
@@ -54,6 +54,8 @@ def main(argv=None):
     a = p.parse_args(argv)
     if a.op == "gemm":
         return gemm_main(a)
+    if a.op == "outliers":
+        return outliers_main(a)
 
     dev = torch.device("cuda", torch.cuda.current_device())
     gen = {"weight": synthetic.llm_weight, "activation": synthetic.activation_t3,
@@ -119,6 +121,51 @@ def fp4_peak_tflops():
             return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 4"
     except (OSError, ValueError, KeyError):
         return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
+def outliers_main(a):
+    """fp4q_separate_outliers on one seeded tensor (algorithmic bytes: x read, bulk written, outlier
+    slots written); also the reconstruction error of the separated pipeline against direct quantization."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gen = {"weight": synthetic.llm_weight, "activation": synthetic.activation_t3,
+           "mlp": synthetic.mlp_row_scaled}[a.data]
+    x = gen(a.rows, a.cols, seed=a.seed, device=dev)
+    n = x.numel()
+    o = fp4q.separate_outliers(x)
+    cap = fp4q.fp4q_outlier_capacity(a.cols, 0.02)
+    nbytes = 4 * n + a.rows * (4 * cap + 4)
+    flush = None if a.no_flush else torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        return fp4q.fp4q_separate_outliers(x, a.rows, a.cols, a.cols, 4.0, 0.02, o.bulk, a.cols, o.cols, o.vals,
+                                           o.count)
+
+    for _ in range(a.warmup):
+        assert call() == 0
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(a.iters):
+        if flush is not None:
+            flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        st = call()
+        e1.record()
+        assert st == 0, fp4q.fp4q_status_string(st)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    med = statistics.median(times)
+    y = fp4q.scatter_outliers(o, fp4q.dequantize(fp4q.quantize(o.bulk, a.fmt), a.fmt))
+    yx = fp4q.dequantize(fp4q.quantize(x, a.fmt), a.fmt)
+    err_sep = ((y.double() - x.double()) ** 2).mean().item()
+    err_dir = ((yx.double() - x.double()) ** 2).mean().item()
+    print(json.dumps({
+        "op": "outliers", "fmt": a.fmt, "rows": a.rows, "cols": a.cols, "data": a.data,
+        "l2_flushed": flush is not None, "ms_median": med, "ms_min": min(times),
+        "algorithmic_bytes": nbytes, "gbs_median": nbytes / (med / 1e3) / 1e9,
+        "outlier_fraction": o.count.sum().item() / n, "mse_separated": err_sep, "mse_direct": err_dir,
+    }), flush=True)
+    return 0
 
 
 def gemm_main(a):

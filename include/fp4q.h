@@ -306,6 +306,38 @@ FP4Q_API fp4q_status_t fp4q_gemm(const uint8_t* a_planes, const uint8_t* a_sf, i
                                  const uint8_t* w_planes, const uint8_t* w_sf, int w_np, const float* w_scale,
                                  int64_t M, int64_t N, int64_t K, void* y, int64_t ldy, fp4q_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Sparse outlier separation ("XFP: quality-targeted adaptive codebook
+ * quantization", sect. 2): per row r of a bf16 matrix, mu = mean and sigma =
+ * population standard deviation (fp64); outliers are the elements with
+ * |x - mu| > k sigma, at most cap = floor(max_frac * cols) of them (when more
+ * qualify, the cap largest deviations, ties to the lower column).  They are
+ * stored in column order as (column uint16, fp16 value -- nearest even,
+ * saturating at 65504) in slots [r][0, count[r]) of [rows][cap] arrays, and
+ * the bulk matrix is x with mu (rounded to bf16) at their positions, ready for
+ * fp4q_quantize.  A reconstruction is fp4q_dequantize of the bulk's codes
+ * followed by fp4q_scatter_outliers.  mu and sigma are reduced in a fixed
+ * order on the GPU; an element whose deviation lies within a few fp64 ulps of
+ * the threshold may be classified differently from a sequential sum.
+ * ------------------------------------------------------------------------ */
+
+/* floor(max_frac * cols), the outlier slots per row (0 for invalid arguments). */
+FP4Q_API int64_t fp4q_outlier_capacity(int64_t cols, double max_frac);
+
+/* x, bulk: bf16 [rows][ld], ld >= cols and a multiple of 8, 16-byte aligned;
+ * cols a multiple of 8, at most 65536; k > 0 finite; 0 <= max_frac <= 1.
+ * out_cols, out_vals: [rows][cap] uint16 (may be null when cap = 0); out_count:
+ * [rows] int32.  One kernel on `stream`. */
+FP4Q_API fp4q_status_t fp4q_separate_outliers(const void* x, int64_t rows, int64_t cols, int64_t ldx, double k,
+                                              double max_frac, void* bulk, int64_t ldb, uint16_t* out_cols,
+                                              uint16_t* out_vals, int32_t* out_count, fp4q_stream_t stream);
+
+/* y[r][out_cols[r][s]] = bf16(out_vals[r][s]) for s < out_count[r]: puts the
+ * outliers back into a bf16 reconstruction y [rows][ldy]. */
+FP4Q_API fp4q_status_t fp4q_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals,
+                                             const int32_t* out_count, int64_t rows, int64_t cols, int64_t cap,
+                                             void* y, int64_t ldy, fp4q_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

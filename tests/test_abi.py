@@ -222,3 +222,38 @@ def test_gemm_rejects_bad_arguments(kw, expect):
 
 def test_gemm_of_nothing_is_a_no_op():
     assert fp4q.fp4q_gemm(A, A, 1, A, A, A, 1, A, 0, 64, 256, A, 64, 0) == ST["FP4Q_SUCCESS"]
+
+
+def test_outlier_capacity():
+    assert fp4q.fp4q_outlier_capacity(4096, 0.02) == 81
+    assert fp4q.fp4q_outlier_capacity(4096, 0.0) == 0 and fp4q.fp4q_outlier_capacity(4096, 1.5) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(k=0.0), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(max_frac=-0.1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(cols=12, ldx=16, ldb=16), "FP4Q_ERROR_SHAPE"),       # cols a multiple of 8
+    (dict(cols=65544, ldx=65544, ldb=65544), "FP4Q_ERROR_SHAPE"),
+    (dict(bulk=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(out_count=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(x=A + 8), "FP4Q_ERROR_MISALIGNED"),
+    (dict(ldb=60), "FP4Q_ERROR_SHAPE"),
+])
+def test_separate_outliers_rejects_bad_arguments(kw, expect):
+    args = dict(x=A, rows=4, cols=64, ldx=64, k=4.0, max_frac=0.05, bulk=A, ldb=64, out_cols=A, out_vals=A,
+                out_count=A, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_separate_outliers(**args) == ST[expect]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cap=65), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(y=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(ldy=32), "FP4Q_ERROR_SHAPE"),
+    (dict(out_count=A + 2), "FP4Q_ERROR_MISALIGNED"),
+])
+def test_scatter_outliers_rejects_bad_arguments(kw, expect):
+    args = dict(out_cols=A, out_vals=A, out_count=A, rows=4, cols=64, cap=3, y=A, ldy=64, stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_scatter_outliers(**args) == ST[expect]
