@@ -17,15 +17,17 @@
 // (32 x 128-bit, replicated to the four lane quadrants): 512-byte atoms of
 // 128 rows x 4 blocks, byte (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
 //
-// GEMM kernel: one CTA per 128 x 256 output tile, 4 warps.  Thread 0 streams
-// k-tiles of 256 elements (A 16 KB, W 32 KB, scale atoms 6 KB) through a
-// 4-stage ring with TMA (128-byte swizzle, no multicast); thread 32 copies the
-// scale atoms of a landed stage into tensor memory and issues the four
-// 128 x 256 x 64 MMAs, then commits the stage back to the producer; at the end
-// all four warps read the fp32 accumulator from tensor memory (each warp its
-// lane quadrant), scale it by s_a * s_w and store bf16.  Every wait is
-// bounded; a CTA that gives up records kErrPipelineTimeout, waits (bounded)
-// for its copies and MMAs, frees its tensor memory and returns.
+// GEMM kernel: persistent, one CTA per SM walking 128 x 256 output tiles, 6
+// warps.  Thread 0 streams k-tiles of 256 elements (A 16 KB, W 32 KB, scale
+// atoms 6 KB) through a 4-stage ring with TMA (128-byte swizzle, no
+// multicast), running ahead across tile boundaries; thread 32 copies the scale
+// atoms of a landed stage into tensor memory and issues the four
+// 128 x 256 x 64 MMAs, then commits the stage back to the producer; warps 2-5
+// read a finished fp32 accumulator from tensor memory (each warp its lane
+// quadrant), scale it by s_a * s_w, store bf16 and hand the accumulator back.
+// Every wait is bounded; a CTA that gives up records kErrPipelineTimeout,
+// waits (bounded) for its copies and MMAs, frees its tensor memory and
+// returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -143,7 +145,8 @@ constexpr int kBBytes = kBN * kBK / 2;               // 32 KB
 constexpr int kSfaBytes = (kBM / 128) * (kBK / 64) * 512;   // 2 KB
 constexpr int kSfbBytes = (kBN / 128) * (kBK / 64) * 512;   // 4 KB
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-constexpr int kGemmThreads = 128;
+constexpr int kEpilogueWarps = 4;
+constexpr int kGemmThreads = 64 + 32 * kEpilogueWarps;   // loader warp, MMA warp, epilogue warps
 constexpr int kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256;                   // columns: accumulator 0..255, SFA 256..271, SFB 272..303
 constexpr uint32_t kTmemSfb = 272;
@@ -239,23 +242,30 @@ struct GemmArgs {
 };
 
 // Y[m][n] = s_a s_w sum over plane pairs and k of A_p[m][k] W_q[n][k].
+// Persistent: CTA b takes output tiles b, b + G, ...  Warp 0 (one thread)
+// loads, warp 1 (one thread) issues the MMAs and owns the tensor memory,
+// warps 2-5 drain the accumulator (warp w reads lane quadrant w % 4).  The
+// loads run ahead across tile boundaries; the MMAs of a tile wait until the
+// previous tile's accumulator has been read ("acc_empty").
 __global__ void __launch_bounds__(tc::kGemmThreads, 1)
     gemm_w4a4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, GemmArgs g)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bars[2 * kStagesG + 1];   // full[s], empty[s], accumulator done
+    __shared__ uint64_t bars[2 * kStagesG + 3];   // full[s], empty[s], acc_full, acc_empty, drain
     __shared__ uint32_t tmem_base_sh;
 
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int64_t n_tiles_n = (g.N + kBN - 1) / kBN;
-    const int64_t mt = blockIdx.x / n_tiles_n, nt = blockIdx.x - mt * n_tiles_n;
-    const int64_t m0 = mt * kBM, n0 = nt * kBN;
+    const int64_t n_tiles = ((g.M + kBM - 1) / kBM) * n_tiles_n;
+    const int64_t my_tiles = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t bar0 = smem_u32(bars);
     auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(kStagesG + s); };
-    const uint32_t done = bar0 + 8u * (uint32_t)(2 * kStagesG);
+    const uint32_t acc_full = bar0 + 8u * (uint32_t)(2 * kStagesG);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain = acc_full + 16u;
     auto stage_a = [&](int s) { return base + (uint32_t)(s * kStageBytes); };
     auto stage_b = [&](int s) { return stage_a(s) + kABytes; };
     auto stage_sfa = [&](int s) { return stage_b(s) + kBBytes; };
@@ -266,7 +276,9 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
         }
-        mbar_init(done, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpilogueWarps);
+        mbar_init(drain, 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -281,99 +293,128 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
     const uint32_t tmem = tmem_base_sh;
 
     const int64_t kt_per_seg = g.K / kBK;
-    const int64_t iters = kt_per_seg * g.a_planes * g.w_planes;
+    const int64_t iters = kt_per_seg * g.a_planes * g.w_planes;   // k-tiles per output tile
     const int64_t atoms_k = g.K / 64;                       // scale atoms per 128-row block
     const int64_t half_k = g.K / 2;                         // bytes of one plane row
     const int64_t n_rb = (g.N + 127) / 128;                 // 128-row blocks of W's scale atoms
-    const bool second_rb = 2 * nt + 1 < n_rb;
-    const uint32_t stage_tx = (uint32_t)(kABytes + kBBytes + kSfaBytes + (second_rb ? kSfbBytes : kSfbBytes / 2));
-    bool ok = true;
+    auto tile_mn = [&](int64_t j, int64_t& mt, int64_t& nt) {
+        const int64_t tile = (int64_t)blockIdx.x + j * gridDim.x;
+        mt = tile / n_tiles_n;
+        nt = tile - mt * n_tiles_n;
+    };
 
     if (t == 0) {
-        // ---- producer ----
-        int64_t issued = 0;
-        for (int64_t i = 0; i < iters; ++i) {
-            const int s = (int)(i % kStagesG);
-            if (i >= kStagesG && !mbar_wait(empty(s), (uint32_t)(((i / kStagesG) - 1) & 1))) {
-                ok = false;
-                break;
+        // ---- producer: k-tiles of every output tile, one ring across tiles ----
+        int64_t gi = 0;   // k-tiles issued so far
+        bool ok = true;
+        for (int64_t j = 0; j < my_tiles && ok; ++j) {
+            int64_t mt, nt;
+            tile_mn(j, mt, nt);
+            const bool second_rb = 2 * nt + 1 < n_rb;
+            const uint32_t tx = (uint32_t)(kABytes + kBBytes + kSfaBytes + (second_rb ? kSfbBytes : kSfbBytes / 2));
+            for (int64_t i = 0; i < iters; ++i, ++gi) {
+                const int s = (int)(gi % kStagesG);
+                if (gi >= kStagesG && !mbar_wait(empty(s), (uint32_t)(((gi / kStagesG) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const int64_t seg = i / kt_per_seg, kt = i - seg * kt_per_seg;
+                const int64_t pa = seg % g.a_planes, pw = seg / g.a_planes;
+                mbar_arm(full(s), tx);
+                tc::tma_load_2d(stage_a(s), &amap, (int)(pa * half_k + kt * (kBK / 2)), (int)(mt * kBM), full(s));
+                tc::tma_load_2d(stage_b(s), &wmap, (int)(pw * half_k + kt * (kBK / 2)), (int)(nt * kBN), full(s));
+                tc::bulk_load(stage_sfa(s), g.a_sf + (mt * atoms_k + 4 * kt) * 512, kSfaBytes, full(s));
+                tc::bulk_load(stage_sfb(s), g.w_sf + ((2 * nt) * atoms_k + 4 * kt) * 512, kSfbBytes / 2, full(s));
+                if (second_rb)
+                    tc::bulk_load(stage_sfb(s) + kSfbBytes / 2, g.w_sf + ((2 * nt + 1) * atoms_k + 4 * kt) * 512,
+                                  kSfbBytes / 2, full(s));
             }
-            const int64_t seg = i / kt_per_seg, kt = i - seg * kt_per_seg;
-            const int64_t pa = seg % g.a_planes, pw = seg / g.a_planes;
-            mbar_arm(full(s), stage_tx);
-            tc::tma_load_2d(stage_a(s), &amap, (int)(pa * half_k + kt * (kBK / 2)), (int)m0, full(s));
-            tc::tma_load_2d(stage_b(s), &wmap, (int)(pw * half_k + kt * (kBK / 2)), (int)n0, full(s));
-            tc::bulk_load(stage_sfa(s), g.a_sf + (mt * atoms_k + 4 * kt) * 512, kSfaBytes, full(s));
-            tc::bulk_load(stage_sfb(s), g.w_sf + ((2 * nt) * atoms_k + 4 * kt) * 512, kSfbBytes / 2, full(s));
-            if (second_rb)
-                tc::bulk_load(stage_sfb(s) + kSfbBytes / 2, g.w_sf + ((2 * nt + 1) * atoms_k + 4 * kt) * 512,
-                              kSfbBytes / 2, full(s));
-            ++issued;
         }
         if (!ok) {
             atomicOr(&g_device_error, kErrPipelineTimeout);
-            // copies still in flight: stages issued but possibly not landed
-            for (int64_t q = issued - kStagesG < 0 ? 0 : issued - kStagesG; q < issued; ++q)
+            for (int64_t q = gi - kStagesG < 0 ? 0 : gi - kStagesG; q < gi; ++q)   // copies still in flight
                 mbar_wait(full((int)(q % kStagesG)), (uint32_t)((q / kStagesG) & 1));
         }
     } else if (t == 32) {
         // ---- MMA issuer ----
-        for (int64_t i = 0; i < iters; ++i) {
-            const int s = (int)(i % kStagesG);
-            if (!mbar_wait(full(s), (uint32_t)((i / kStagesG) & 1))) {
+        int64_t gi = 0;
+        bool ok = true;
+        for (int64_t j = 0; j < my_tiles && ok; ++j) {
+            if (j > 0 && !mbar_wait(acc_empty, (uint32_t)((j - 1) & 1))) {   // previous accumulator drained
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            // scale atoms -> tensor memory: SFA 4 columns per MMA, SFB 8 (two 128-row blocks)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                tc::copy_atom_to_tmem(tmem + kTmemSfa + 4u * j, tc::desc_atom(stage_sfa(s) + 512u * j));
-                tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * j, tc::desc_atom(stage_sfb(s) + 512u * j));
-                tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * j + 4u,
-                                      tc::desc_atom(stage_sfb(s) + kSfbBytes / 2 + 512u * j));
-            }
-            const uint64_t da = tc::desc_sw128(stage_a(s)), db = tc::desc_sw128(stage_b(s));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)   // K = 64 per MMA: 32 bytes along the swizzled row
-                tc::mma_block16(tmem, da + 2u * j, db + 2u * j, tmem + kTmemSfa + 4u * j, tmem + kTmemSfb + 8u * j,
-                                (i > 0 || j > 0) ? 1u : 0u);
-            tc::commit_to(empty(s));
-        }
-        if (!ok) atomicOr(&g_device_error, kErrPipelineTimeout);
-        tc::commit_to(done);   // arrives when every MMA issued above has completed
-    }
-    __syncwarp();
-
-    // ---- epilogue: all four warps, warp w owns accumulator rows 32w..32w+31 ----
-    const bool acc_ready = mbar_wait(done, 0u);
-    tc::fence_after_sync();
-    if (!acc_ready) {
-        if (lane == 0) atomicOr(&g_device_error, kErrPipelineTimeout);
-    } else if (iters > 0) {
-        const float alpha = __fmul_rn(*g.a_scale, *g.w_scale);
-        const int64_t m = m0 + 32 * warp + lane;
-        const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-#pragma unroll 1
-        for (int c = 0; c < kBN; c += 32) {
-            if (n0 + c >= g.N) break;   // uniform across the warp
-            float v[32];
-            tc::tmem_ld32(trow + (uint32_t)c, v);
-            if (m < g.M) {
-                uint16_t* yrow = g.y + m * g.ldy + n0 + c;
+            for (int64_t i = 0; i < iters; ++i, ++gi) {
+                const int s = (int)(gi % kStagesG);
+                if (!mbar_wait(full(s), (uint32_t)((gi / kStagesG) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                // scale atoms -> tensor memory: SFA 4 columns per MMA, SFB 8 (two 128-row blocks)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    if (n0 + c + 8 * q >= g.N) break;
-                    uint4 o;
-                    o.x = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 0]), __fmul_rn(alpha, v[8 * q + 1]));
-                    o.y = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 2]), __fmul_rn(alpha, v[8 * q + 3]));
-                    o.z = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 4]), __fmul_rn(alpha, v[8 * q + 5]));
-                    o.w = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 6]), __fmul_rn(alpha, v[8 * q + 7]));
-                    *reinterpret_cast<uint4*>(yrow + 8 * q) = o;
+                    tc::copy_atom_to_tmem(tmem + kTmemSfa + 4u * q, tc::desc_atom(stage_sfa(s) + 512u * q));
+                    tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * q, tc::desc_atom(stage_sfb(s) + 512u * q));
+                    tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * q + 4u,
+                                          tc::desc_atom(stage_sfb(s) + kSfbBytes / 2 + 512u * q));
+                }
+                const uint64_t da = tc::desc_sw128(stage_a(s)), db = tc::desc_sw128(stage_b(s));
+#pragma unroll
+                for (int q = 0; q < 4; ++q)   // K = 64 per MMA: 32 bytes along the swizzled row
+                    tc::mma_block16(tmem, da + 2u * q, db + 2u * q, tmem + kTmemSfa + 4u * q,
+                                    tmem + kTmemSfb + 8u * q, (i > 0 || q > 0) ? 1u : 0u);
+                tc::commit_to(empty(s));
+            }
+            if (ok) tc::commit_to(acc_full);   // arrives when the tile's MMAs have completed
+        }
+        if (!ok) {
+            atomicOr(&g_device_error, kErrPipelineTimeout);
+            tc::commit_to(drain);              // wait (bounded) for the MMAs issued so far
+            mbar_wait(drain, 0u);
+        }
+    } else if (warp >= 2) {
+        // ---- epilogue: warp w reads accumulator rows 32 (w % 4) .. + 31 ----
+        const int quad = warp & 3;
+        const float alpha = __fmul_rn(*g.a_scale, *g.w_scale);
+        const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
+        for (int64_t j = 0; j < my_tiles; ++j) {
+            if (!mbar_wait(acc_full, (uint32_t)(j & 1))) {
+                if (lane == 0) atomicOr(&g_device_error, kErrPipelineTimeout);
+                break;
+            }
+            tc::fence_after_sync();
+            int64_t mt, nt;
+            tile_mn(j, mt, nt);
+            const int64_t m = mt * kBM + 32 * quad + lane, n0 = nt * kBN;
+#pragma unroll 1
+            for (int c = 0; c < kBN; c += 32) {
+                if (n0 + c >= g.N) break;   // uniform across the warp
+                float v[32];
+                tc::tmem_ld32(trow + (uint32_t)c, v);
+                if (m < g.M) {
+                    uint16_t* yrow = g.y + m * g.ldy + n0 + c;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (n0 + c + 8 * q >= g.N) break;
+                        uint4 o;
+                        o.x = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 0]), __fmul_rn(alpha, v[8 * q + 1]));
+                        o.y = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 2]), __fmul_rn(alpha, v[8 * q + 3]));
+                        o.z = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 4]), __fmul_rn(alpha, v[8 * q + 5]));
+                        o.w = pack_bf16x2_rn(__fmul_rn(alpha, v[8 * q + 6]), __fmul_rn(alpha, v[8 * q + 7]));
+                        *reinterpret_cast<uint4*>(yrow + 8 * q) = o;
+                    }
                 }
             }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty) : "memory");
         }
     }
+    __syncwarp();
+    // Every MMA has completed here: the epilogue waited for each tile's commit,
+    // or the MMA thread drained its own after a failure.
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 1) {
@@ -419,10 +460,11 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
     g.w_planes = w_np;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
     if (tiles >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const int64_t grid = tiles < sm_count() ? tiles : sm_count();   // persistent: one CTA per SM
     const cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                kGemmSmem);
     if (e != cudaSuccess) return e;
-    gemm_w4a4_kernel<<<(unsigned)tiles, kGemmThreads, kGemmSmem, st>>>(amap, wmap, g);
+    gemm_w4a4_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmem, st>>>(amap, wmap, g);
     return cudaGetLastError();
 }
 

@@ -15,8 +15,10 @@
 //   3. one pass in tiles of 2048 elements writes the bulk row (the mean, rounded
 //      to bf16, at every outlier) and the outliers in column order, their slots
 //      from CTA-wide prefix counts.
-// Rows are read from global memory on every pass (L2 keeps a row: at most
-// 128 KB); each thread moves 16 bytes at a time.
+// The row is read from global memory once, into shared memory, and every pass
+// reads it there; each thread moves 16 bytes at a time.  Rows of up to 8192
+// elements take one warp each (8 rows per CTA, warp reductions and scans
+// only); longer rows take a CTA each.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -108,10 +110,26 @@ __device__ int cta_exclusive_scan(int v, int* sh, int* total)
     return sh[warp] + inc - v;
 }
 
-// Eight bf16 values of x[row] starting at column j (j % 8 == 0), as fp32.
-__device__ __forceinline__ void load8(const uint16_t* row, int64_t j, float* v)
+// Copy n16 16-byte chunks from global to shared memory, `stride` threads
+// taking chunk i, i + stride, ...: eight loads in flight per thread.
+__device__ __forceinline__ void copy_row(uint4* dst, const uint4* src, int64_t n16, int64_t i, int64_t stride)
 {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + j));
+    for (; i < n16; i += 8 * stride) {
+        uint4 r[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (i + q * stride < n16) r[q] = __ldg(src + i + q * stride);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (i + q * stride < n16) dst[i + q * stride] = r[q];
+    }
+}
+
+// Eight bf16 values of the row in shared memory (byte address srow) from
+// column j (j % 8 == 0), as fp32.
+__device__ __forceinline__ void load8(uint32_t srow, int64_t j, float* v)
+{
+    const uint4 w = lds128(srow + 2u * (uint32_t)j);
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -132,34 +150,39 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rn(double m)
 
 __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a)
 {
+    extern __shared__ uint4 srow_raw[];
     __shared__ double shd[33];
     __shared__ long long shl[33];
     __shared__ int shi[33];
     const int64_t r = blockIdx.x;
-    const uint16_t* row = a.x + r * a.ldx;
     const int t = threadIdx.x;
     const int64_t n = a.cols;
+    const uint32_t row = smem_u32(srow_raw);
+    copy_row(srow_raw, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n / 8, t, kOutThreads);
+    __syncthreads();
 
-    // 1. mean and deviation
-    double s = 0.0;
+    // 1. mean and deviation (eight partial sums per thread, combined in a fixed order)
+    double p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
         float v[8];
         load8(row, j, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s += (double)v[i];
+        for (int i = 0; i < 8; ++i) p[i] += (double)v[i];
     }
-    const double mu = cta_sum(s, shd) / (double)n;
-    s = 0.0;
+    const double mu = cta_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])), shd) / (double)n;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = 0.0;
     for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
         float v[8];
         load8(row, j, v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const double d = (double)v[i] - mu;
-            s += d * d;
+            p[i] = fma(d, d, p[i]);
         }
     }
-    double thr = a.k * sqrt(cta_sum(s, shd) / (double)n);
+    double thr = a.k * sqrt(cta_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])), shd) /
+                            (double)n);
 
     // 2. count; above the cap, the cap-th largest deviation and its ties
     auto count_where = [&](auto pred) {
@@ -198,7 +221,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
         float v[8];
         uint4 w = make_uint4(0, 0, 0, 0);
         if (in) {
-            w = __ldg(reinterpret_cast<const uint4*>(row + j));
+            w = lds128(row + 2u * (uint32_t)j);
             load8(row, j, v);
         }
         int gt = 0, eq = 0;
@@ -243,6 +266,154 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
     if (t == 0) a.out_count[r] = (int32_t)done;
 }
 
+// The same, one warp per row (rows of at most 8192 elements): warp w of CTA b
+// takes row R b + w (R rows per CTA, 8 or as many as 48 KB of shared memory
+// holds), its copy in shared memory at w * cols * 2 bytes.  Sums are
+// xor-butterflies, so every lane holds the same, bit for bit.
+constexpr int kRowsPerCta = 8;
+
+__device__ __forceinline__ double warp_sum(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_int(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// Exclusive prefix over the warp's lanes; *total receives the sum.
+__device__ __forceinline__ int warp_exclusive_scan(int v, int* total)
+{
+    const int lane = threadIdx.x & 31;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    *total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+    return inc - v;
+}
+
+__global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(OutlierArgs a, int64_t rows)
+{
+    extern __shared__ uint4 srows_raw[];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;
+    if (r >= rows) return;   // warp-uniform
+    const int64_t n = a.cols, n8 = n / 8;
+    uint4* srow = srows_raw + (int64_t)w * n8;
+    const uint32_t row = smem_u32(srow);
+    copy_row(srow, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n8, lane, 32);
+    __syncwarp();
+
+    // eight independent partial sums per lane (one per position in the 16-byte
+    // chunk), combined in a fixed order: the additions overlap instead of
+    // forming one chain of fp64 latencies
+    double p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int64_t i = lane; i < n8; i += 32) {
+        float v[8];
+        load8(row, 8 * i, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) p[q] += (double)v[q];
+    }
+    const double mu = warp_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]))) / (double)n;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = 0.0;
+    for (int64_t i = lane; i < n8; i += 32) {
+        float v[8];
+        load8(row, 8 * i, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const double d = (double)v[q] - mu;
+            p[q] = fma(d, d, p[q]);
+        }
+    }
+    double thr =
+        a.k * sqrt(warp_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]))) / (double)n);
+
+    auto count_where = [&](auto pred) {
+        int c = 0;
+        for (int64_t i = lane; i < n8; i += 32) {
+            float v[8];
+            load8(row, 8 * i, v);
+            uint32_t m = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) m |= pred(fabs((double)v[q] - mu)) ? 1u << q : 0u;
+            c += __popc(m);
+        }
+        return (long long)warp_sum_int(c);
+    };
+    long long tie_need = 0;
+    if (a.cap == 0) {
+        thr = __longlong_as_double(0x7FF0000000000000ll);
+    } else if (count_where([&](double d) { return d > thr; }) > a.cap) {
+        unsigned long long lo = 0ull, hi = 0x7FF0000000000000ull;
+        while (hi - lo > 1ull) {
+            const unsigned long long mid = lo + (hi - lo) / 2;
+            const long long c = count_where([&](double d) { return (unsigned long long)__double_as_longlong(d) >= mid; });
+            if (c >= a.cap) lo = mid;
+            else hi = mid;
+        }
+        thr = __longlong_as_double((long long)lo);
+        tie_need = a.cap - count_where([&](double d) { return d > thr; });
+    }
+
+    const uint16_t mub = f64_to_bf16_rn(mu);
+    uint16_t* brow = a.bulk + r * a.ldb;
+    int64_t done = 0, ties_seen = 0;
+    for (int64_t i0 = 0; i0 < n8; i0 += 32) {
+        const int64_t i = i0 + lane;
+        const bool in = i < n8;
+        float v[8];
+        uint4 wd = make_uint4(0, 0, 0, 0);
+        if (in) {
+            wd = lds128(row + 16u * (uint32_t)i);
+            load8(row, 8 * i, v);
+        }
+        uint32_t gmask = 0, emask = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const double d = in ? fabs((double)v[q] - mu) : -1.0;
+            if (d > thr) gmask |= 1u << q;
+            else if (d == thr && tie_need > 0) emask |= 1u << q;
+        }
+        int eq_total;
+        int rank = (int)ties_seen + warp_exclusive_scan(__popc(emask), &eq_total);
+        uint32_t omask = gmask;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (emask & (1u << q)) {
+                if (rank < tie_need) omask |= 1u << q;
+                ++rank;
+            }
+        ties_seen += eq_total;
+        int tot;
+        int slot = (int)done + warp_exclusive_scan(__popc(omask), &tot);
+        if (in) {
+            uint32_t u[4] = {wd.x, wd.y, wd.z, wd.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (omask & (1u << q)) {
+                    const uint32_t sh = (q & 1) ? 16u : 0u;
+                    u[q >> 1] = (u[q >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
+                    a.out_cols[r * a.cap + slot] = (uint16_t)(8 * i + q);
+                    a.out_vals[r * a.cap + slot] =
+                        __half_as_ushort(__float2half_rn(fminf(fmaxf(v[q], -65504.0f), 65504.0f)));
+                    ++slot;
+                }
+            *reinterpret_cast<uint4*>(brow + 8 * i) = make_uint4(u[0], u[1], u[2], u[3]);
+        }
+        done += tot;
+    }
+    if (lane == 0) a.out_count[r] = (int32_t)done;
+}
+
 struct ScatterArgs {
     const uint16_t* out_cols;
     const uint16_t* out_vals;
@@ -272,7 +443,21 @@ cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t co
 {
     if (rows == 0) return cudaSuccess;
     OutlierArgs a{x, bulk, out_cols, out_vals, out_count, ldx, ldb, cols, cap, k};
-    outlier_rows_kernel<<<(unsigned)rows, kOutThreads, 0, st>>>(a);
+    if (cols <= 8192) {   // one warp per row, at most 48 KB of rows per CTA
+        int64_t rpc = (48 * 1024) / (cols * 2);
+        rpc = rpc < 1 ? 1 : (rpc > kRowsPerCta ? kRowsPerCta : rpc);
+        const int smem = (int)(rpc * cols * 2);
+        const int64_t blocks = (rows + rpc - 1) / rpc;
+        outlier_rows_warp_kernel<<<(unsigned)blocks, (unsigned)(32 * rpc), smem, st>>>(a, rows);
+        return cudaGetLastError();
+    }
+    const int smem = (int)(cols * 2);   // the row, at most 128 KB
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(outlier_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   smem);
+        if (e != cudaSuccess) return e;
+    }
+    outlier_rows_kernel<<<(unsigned)rows, kOutThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
