@@ -148,8 +148,13 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kEpilogueWarps = 4;
 constexpr int kGemmThreads = 64 + 32 * kEpilogueWarps;   // loader warp, MMA warp, epilogue warps
 constexpr int kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256;                   // columns: accumulator 0..255, SFA 256..271, SFB 272..303
-constexpr uint32_t kTmemSfb = 272;
+// Tensor-memory columns: accumulator 0..255, then per stage s the scale
+// factors of that stage's k-tile (A 16 columns, W 32), so that copying the
+// next stage's scales never waits for the MMAs reading this stage's.
+constexpr uint32_t kTmemSf0 = 256;
+constexpr uint32_t kTmemSfStage = 48;
+constexpr uint32_t kTmemSfbOff = 16;
+static_assert(kTmemSf0 + kStagesG * kTmemSfStage <= (uint32_t)kTmemCols, "scale factors exceed the allocation");
 constexpr int kGemmSmem = kStagesG * kStageBytes + 1024 + 256;
 
 // Instruction descriptor of kind::mxf4nvf4 with 16-element UE4M3 scales:
@@ -353,18 +358,18 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
                 }
                 tc::fence_after_sync();
                 // scale atoms -> tensor memory: SFA 4 columns per MMA, SFB 8 (two 128-row blocks)
+                const uint32_t sfa = tmem + kTmemSf0 + kTmemSfStage * (uint32_t)s, sfb = sfa + kTmemSfbOff;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    tc::copy_atom_to_tmem(tmem + kTmemSfa + 4u * q, tc::desc_atom(stage_sfa(s) + 512u * q));
-                    tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * q, tc::desc_atom(stage_sfb(s) + 512u * q));
-                    tc::copy_atom_to_tmem(tmem + kTmemSfb + 8u * q + 4u,
-                                          tc::desc_atom(stage_sfb(s) + kSfbBytes / 2 + 512u * q));
+                    tc::copy_atom_to_tmem(sfa + 4u * q, tc::desc_atom(stage_sfa(s) + 512u * q));
+                    tc::copy_atom_to_tmem(sfb + 8u * q, tc::desc_atom(stage_sfb(s) + 512u * q));
+                    tc::copy_atom_to_tmem(sfb + 8u * q + 4u, tc::desc_atom(stage_sfb(s) + kSfbBytes / 2 + 512u * q));
                 }
                 const uint64_t da = tc::desc_sw128(stage_a(s)), db = tc::desc_sw128(stage_b(s));
 #pragma unroll
                 for (int q = 0; q < 4; ++q)   // K = 64 per MMA: 32 bytes along the swizzled row
-                    tc::mma_block16(tmem, da + 2u * q, db + 2u * q, tmem + kTmemSfa + 4u * q,
-                                    tmem + kTmemSfb + 8u * q, (i > 0 || q > 0) ? 1u : 0u);
+                    tc::mma_block16(tmem, da + 2u * q, db + 2u * q, sfa + 4u * q, sfb + 8u * q,
+                                    (i > 0 || q > 0) ? 1u : 0u);
                 tc::commit_to(empty(s));
             }
             if (ok) tc::commit_to(acc_full);   // arrives when the tile's MMAs have completed
