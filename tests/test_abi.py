@@ -257,3 +257,11 @@ def test_scatter_outliers_rejects_bad_arguments(kw, expect):
     args = dict(out_cols=A, out_vals=A, out_count=A, rows=4, cols=64, cap=3, y=A, ldy=64, stream=0)
     args.update(kw)
     assert fp4q.fp4q_scatter_outliers(**args) == ST[expect]
+
+
+def test_build_entry_expects_the_header_abi_version():
+    """__graft_entry__.build() checks the loaded library's ABI version against a literal."""
+    ver = re.search(r"#define FP4Q_ABI_VERSION (\d+)", open(HEADER).read()).group(1)
+    entry = open(os.path.join(ROOT, "__graft_entry__.py")).read()
+    assert f"fp4q_abi_version() == {ver}" in entry
+    assert fp4q.fp4q_abi_version() == int(ver)
