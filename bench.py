@@ -186,6 +186,30 @@ def cpu_baseline_leg():
                       f"computed tensor scale + MSE, {nthreads} threads"}
 
 
+# ---------------------------------------------------------------- multi-rank host logic
+
+def rank_layer_seed(layer: int, rank: int, layers: int) -> int:
+    """Layer index used for the seeds of rank `rank`'s copy of the weight set: every rank
+    quantizes its own set (weak scaling), disjoint from the others'."""
+    return layer + rank * layers
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The job's time: the maximum of the ranks' device-timed values (all_reduce MAX)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(elements_per_rank: int, world: int, steps: int, ms: float) -> float:
+    """Whole-job elements/s: the units all ranks processed over the (max-over-ranks) time."""
+    return elements_per_rank * world * steps / (ms / 1e3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -244,7 +268,7 @@ def main():
     tensors = []
     for layer in range(args.layers):
         for i, (name, r, c) in enumerate(layer_shapes()):
-            seed = synthetic.tensor_seed(2, layer + rank * args.layers, i)
+            seed = synthetic.tensor_seed(2, rank_layer_seed(layer, rank, args.layers), i)
             x = synthetic.llm_weight(r, c, seed=seed, device=dev)
             q = fp4q.Quantized(torch.empty(r, c // 2, dtype=torch.uint8, device=dev),
                                torch.empty(r, c // 16, dtype=torch.uint8, device=dev),
@@ -315,13 +339,9 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_per_step = ms / args.steps
-    value = elements * world / (ms / 1e3) * args.steps
+    value = job_throughput(elements, world, args.steps, ms)
 
     # per-call durations -> roofline of the call (its launches run back to back on the stream)
     call_ms = [ev[s][2 * k].elapsed_time(ev[s][2 * k + 1]) for s in range(args.steps) for k in range(len(calls))]
