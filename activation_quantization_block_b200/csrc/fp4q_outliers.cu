@@ -349,11 +349,78 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
         }
         return (long long)warp_sum_int(c);
     };
-    long long tie_need = 0;
-    if (a.cap == 0) {
-        thr = __longlong_as_double(0x7FF0000000000000ll);
-    } else if (count_where([&](double d) { return d > thr; }) > a.cap) {
-        unsigned long long lo = 0ull, hi = 0x7FF0000000000000ull;
+    const uint16_t mub = f64_to_bf16_rn(mu);
+    uint16_t* brow = a.bulk + r * a.ldb;
+    // One pass: bulk row and outlier slots for threshold t (and, when tie_need > 0,
+    // the first tie_need elements with d == t).  d > t is decided in fp32 where
+    // |d32 - t32| exceeds a band covering the fp32 roundings of mu, t and d (each
+    // at most 2^-24 relative; the band is 2^-20 of |mu| + t), in fp64 elsewhere.
+    // Slots past the capacity are not written.  Returns the row's count.
+    auto compact = [&](double t, long long tie_need, bool none) -> long long {
+        const float mu32 = (float)mu, t32 = (float)t;
+        const float band = 0x1p-20f * (fabsf(mu32) + t32);
+        long long done = 0, ties_seen = 0;
+        for (int64_t i0 = 0; i0 < n8; i0 += 32) {
+            const int64_t i = i0 + lane;
+            const bool in = i < n8;
+            float v[8];
+            uint4 wd = make_uint4(0, 0, 0, 0);
+            if (in) {
+                wd = lds128(row + 16u * (uint32_t)i);
+                load8(row, 8 * i, v);
+            }
+            uint32_t gmask = 0, emask = 0;
+            if (in && !none) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float d32 = fabsf(v[q] - mu32);
+                    if (d32 - t32 > band && d32 <= 3.4e38f) {
+                        gmask |= 1u << q;
+                    } else if (!(d32 - t32 < -band)) {   // near the threshold (or non-finite): fp64
+                        const double d = fabs((double)v[q] - mu);
+                        if (d > t) gmask |= 1u << q;
+                        else if (d == t && tie_need > 0) emask |= 1u << q;
+                    }
+                }
+            }
+            int eq_total;
+            int rank = (int)ties_seen + warp_exclusive_scan(__popc(emask), &eq_total);
+            uint32_t omask = gmask;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (emask & (1u << q)) {
+                    if (rank < tie_need) omask |= 1u << q;
+                    ++rank;
+                }
+            ties_seen += eq_total;
+            int tot;
+            long long slot = done + warp_exclusive_scan(__popc(omask), &tot);
+            if (in) {
+                uint32_t u[4] = {wd.x, wd.y, wd.z, wd.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (omask & (1u << q)) {
+                        const uint32_t sh = (q & 1) ? 16u : 0u;
+                        u[q >> 1] = (u[q >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
+                        if (slot < a.cap) {
+                            a.out_cols[r * a.cap + slot] = (uint16_t)(8 * i + q);
+                            a.out_vals[r * a.cap + slot] =
+                                __half_as_ushort(__float2half_rn(fminf(fmaxf(v[q], -65504.0f), 65504.0f)));
+                        }
+                        ++slot;
+                    }
+                *reinterpret_cast<uint4*>(brow + 8 * i) = make_uint4(u[0], u[1], u[2], u[3]);
+            }
+            done += tot;
+        }
+        return done;
+    };
+
+    // Speculatively with k sigma (the usual case: the count stays within the cap);
+    // otherwise the cap-th largest deviation, its ties, and the pass again.
+    long long total = compact(thr, 0, a.cap == 0);
+    if (a.cap > 0 && total > a.cap) {
+        unsigned long long lo = 0ull, hi = 0x7FF0000000000000ull;   // bits of 0 and of +inf
         while (hi - lo > 1ull) {
             const unsigned long long mid = lo + (hi - lo) / 2;
             const long long c = count_where([&](double d) { return (unsigned long long)__double_as_longlong(d) >= mid; });
@@ -361,57 +428,9 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
             else hi = mid;
         }
         thr = __longlong_as_double((long long)lo);
-        tie_need = a.cap - count_where([&](double d) { return d > thr; });
+        total = compact(thr, a.cap - count_where([&](double d) { return d > thr; }), false);
     }
-
-    const uint16_t mub = f64_to_bf16_rn(mu);
-    uint16_t* brow = a.bulk + r * a.ldb;
-    int64_t done = 0, ties_seen = 0;
-    for (int64_t i0 = 0; i0 < n8; i0 += 32) {
-        const int64_t i = i0 + lane;
-        const bool in = i < n8;
-        float v[8];
-        uint4 wd = make_uint4(0, 0, 0, 0);
-        if (in) {
-            wd = lds128(row + 16u * (uint32_t)i);
-            load8(row, 8 * i, v);
-        }
-        uint32_t gmask = 0, emask = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const double d = in ? fabs((double)v[q] - mu) : -1.0;
-            if (d > thr) gmask |= 1u << q;
-            else if (d == thr && tie_need > 0) emask |= 1u << q;
-        }
-        int eq_total;
-        int rank = (int)ties_seen + warp_exclusive_scan(__popc(emask), &eq_total);
-        uint32_t omask = gmask;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (emask & (1u << q)) {
-                if (rank < tie_need) omask |= 1u << q;
-                ++rank;
-            }
-        ties_seen += eq_total;
-        int tot;
-        int slot = (int)done + warp_exclusive_scan(__popc(omask), &tot);
-        if (in) {
-            uint32_t u[4] = {wd.x, wd.y, wd.z, wd.w};
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (omask & (1u << q)) {
-                    const uint32_t sh = (q & 1) ? 16u : 0u;
-                    u[q >> 1] = (u[q >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
-                    a.out_cols[r * a.cap + slot] = (uint16_t)(8 * i + q);
-                    a.out_vals[r * a.cap + slot] =
-                        __half_as_ushort(__float2half_rn(fminf(fmaxf(v[q], -65504.0f), 65504.0f)));
-                    ++slot;
-                }
-            *reinterpret_cast<uint4*>(brow + 8 * i) = make_uint4(u[0], u[1], u[2], u[3]);
-        }
-        done += tot;
-    }
-    if (lane == 0) a.out_count[r] = (int32_t)done;
+    if (lane == 0) a.out_count[r] = (int32_t)total;
 }
 
 struct ScatterArgs {

@@ -81,23 +81,37 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_record(kernel_key: str):
-    """DRAM bytes per element from the committed ncu capture, if it was taken on the current source."""
+# The translation units the measured kernels are built from: a traffic record
+# stays valid until one of these files changes.
+TRAFFIC_SOURCES = {
+    "quantize_batch": ("fp4q_batch.cu", "fp4q_launch.cuh", "fp4q_common.cuh", "fp4q_device.cuh", "fp4q_tma.cuh",
+                       "fp4q_internal.h"),
+    "quantize": ("fp4q_kernels.cu", "fp4q_launch.cuh", "fp4q_common.cuh", "fp4q_device.cuh", "fp4q_tma.cuh",
+                 "fp4q_internal.h"),
+}
+
+
+def kernel_source_sha256(kernel_key: str) -> str:
     from activation_quantization_block_b200 import _build
     import hashlib
+    files = TRAFFIC_SOURCES["quantize_batch" if kernel_key.startswith("quantize_batch") else "quantize"]
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(_build.CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_record(kernel_key: str):
+    """DRAM bytes per element from the committed ncu capture, if it was taken on the kernel's current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    h = hashlib.sha256()
-    for p in _build.sources() + sorted(os.path.join(_build.CSRC, f) for f in os.listdir(_build.CSRC)
-                                        if f.endswith((".cuh", ".h"))):
-        with open(p, "rb") as f:
-            h.update(f.read())
     entry = rec.get(kernel_key)
-    if not entry or entry.get("source_sha256") != h.hexdigest():
+    if not entry or entry.get("source_sha256") != kernel_source_sha256(kernel_key):
         return None
     return float(entry["dram_bytes_per_element"])
 
