@@ -104,8 +104,14 @@ def main(argv=None):
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     med, best = statistics.median(times), min(times)
+    mse_value = None
+    if a.op == "quantize" and not a.no_mse:
+        mse_value = mse.item()
+    elif a.op == "error":
+        mse_value = mse.item()
     print(json.dumps({
         "op": a.op, "fmt": a.fmt, "rotate": a.rotate, "mse": not a.no_mse, "scale_given": a.scale_given,
+        "mse_value": mse_value,
         "mx_ceil": a.mx_ceil,
         "rows": a.rows, "cols": a.cols, "data": a.data, "l2_flushed": flush is not None,
         "ms_median": med, "ms_min": best, "elements_per_s": n / (med / 1e3),
