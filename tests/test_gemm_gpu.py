@@ -117,3 +117,22 @@ def test_gemm_large_sampled(orc, dev):
     yf = y[idx].float().cpu().numpy().astype(np.float64)
     tol = 2.0 ** -8 * np.abs(Y) + (4 * K / 64 + 70) * 2.0 ** -24 * Yabs
     assert np.all(np.abs(yf - Y) <= tol)
+
+
+@pytest.mark.parametrize("M,N,K,ldy", [(1, 264, 512, 264), (130, 520, 1280, 528), (257, 8, 768, 16)])
+def test_gemm_ragged_shapes_and_strided_output(orc, dev, M, N, K, ldy):
+    """M and N off the 128 / 256 tile grid, K an odd number of 256-element k-tiles, and an output
+    row stride above N (the columns past N stay untouched)."""
+    a = synthetic.activation_t3(M, K, seed=M, device="cpu").to(dev)
+    w = synthetic.llm_weight(N, K, seed=N, device="cpu").to(dev)
+    qa, qw = _quantized(orc, a, "nvfp4_razer"), _quantized(orc, w, "nvfp4_razer_w")
+    buf = torch.full((M, ldy), -3.0, dtype=torch.bfloat16, device=dev)
+    y = fp4q.gemm(fp4q.mma_operand(qa, "nvfp4_razer"), fp4q.mma_operand(qw, "nvfp4_razer_w"), out=buf[:, :N])
+    torch.cuda.synchronize()
+    if ldy > N:
+        assert torch.all(buf[:, N:] == -3.0)
+    ah, _ = orc.dequantize(qa.codes.cpu().numpy(), qa.scales.cpu().numpy(), qa.tensor_scale.item(), "nvfp4_razer")
+    wh, _ = orc.dequantize(qw.codes.cpu().numpy(), qw.scales.cpu().numpy(), qw.tensor_scale.item(), "nvfp4_razer_w")
+    Y, Yabs = orc.gemm(ah, wh)
+    yf = y.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(yf - Y) <= 2.0 ** -8 * np.abs(Y) + (4 * K / 64 + 70) * 2.0 ** -24 * Yabs)

@@ -98,3 +98,17 @@ def test_separated_pipeline_lowers_the_error(orc, dev, fmt):
     assert np.array_equal(synthetic.bf16_bits(o.bulk[pick]), bulk)
     rc, rs, _, _ = orc.quantize(bulk, fmt, tensor_scale=qb.tensor_scale.item(), want_sse=False)
     assert np.array_equal(qb.codes[pick].cpu().numpy(), rc) and np.array_equal(qb.scales[pick].cpu().numpy(), rs)
+
+
+def test_separation_of_a_strided_matrix(orc, dev):
+    """x with a row stride above cols: the same result as its dense copy."""
+    big = _inputs(48, 2048 + 64, seed=77).to(dev)
+    x = big[:, :2048]
+    assert x.stride(0) == 2048 + 64
+    o = fp4q.separate_outliers(x)
+    od = fp4q.separate_outliers(x.contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(o.bulk, od.bulk) and torch.equal(o.count, od.count)
+    assert torch.equal(o.cols, od.cols) and torch.equal(o.vals, od.vals)
+    bulk, _, _, cnt, _, _ = orc.separate_outliers(synthetic.bf16_bits(x.contiguous()))
+    assert np.array_equal(synthetic.bf16_bits(o.bulk), bulk) and np.array_equal(o.count.cpu().numpy(), cnt)
