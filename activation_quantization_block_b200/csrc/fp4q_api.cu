@@ -236,8 +236,15 @@ fp4q_status_t fp4q_separate_outliers(const void* x, int64_t rows, int64_t cols, 
     if (rows < 0 || cols < 0 || !(k > 0.0 && k < 1e300) || !(max_frac >= 0.0 && max_frac <= 1.0))
         return FP4Q_ERROR_INVALID_VALUE;
     if (cols % 8 != 0 || cols > 65536 || rows >= ((int64_t)1 << 31)) return FP4Q_ERROR_SHAPE;
-    if (rows == 0 || cols == 0) return FP4Q_SUCCESS;
+    if (rows == 0) return FP4Q_SUCCESS;
     fp4q_status_t s;
+    if (cols == 0) {   // no elements: every row has no outliers
+        if (out_count == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+        if (!aligned(out_count, 4)) return FP4Q_ERROR_MISALIGNED;
+        if ((s = check_device()) != FP4Q_SUCCESS) return s;
+        return from_cuda(cudaMemsetAsync(out_count, 0, sizeof(int32_t) * (size_t)rows,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+    }
     if ((s = check_matrix(x, cols, ldx)) != FP4Q_SUCCESS) return s;
     if ((s = check_matrix(bulk, cols, ldb)) != FP4Q_SUCCESS) return s;
     const int64_t cap = outlier_capacity(cols, max_frac);
