@@ -17,14 +17,16 @@
 // (32 x 128-bit, replicated to the four lane quadrants): 512-byte atoms of
 // 128 rows x 4 blocks, byte (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
 //
-// GEMM kernel: persistent, one CTA per SM walking 128 x 256 output tiles, 6
-// warps.  Thread 0 streams k-tiles of 256 elements (A 16 KB, W 32 KB, scale
-// atoms 6 KB) through a 4-stage ring with TMA (128-byte swizzle, no
-// multicast), running ahead across tile boundaries; thread 32 copies the scale
-// atoms of a landed stage into tensor memory and issues the four
-// 128 x 256 x 64 MMAs, then commits the stage back to the producer; warps 2-5
-// read a finished fp32 accumulator from tensor memory (each warp its lane
+// GEMM kernel: persistent, two CTAs per SM walking 128 x 128 output tiles, 6
+// warps each.  Thread 0 streams k-tiles of 256 elements (A 16 KB, W 16 KB,
+// scale atoms 4 KB) through a 3-stage ring with TMA (128-byte swizzle, each CTA
+// loading its own tiles), running ahead across tile boundaries; thread 32
+// copies the scale atoms of a landed stage into tensor memory and issues the
+// four 128 x 128 x 64 MMAs, then commits the stage back to the producer; warps
+// 2-5 read a finished fp32 accumulator from tensor memory (each warp its lane
 // quadrant), scale it by s_a * s_w, store bf16 and hand the accumulator back.
+// Two CTAs per SM (111 KB of shared memory and 256 tensor-memory columns each)
+// keep two MMA streams per SM; one CTA of 128 x 256 tiles ran 8-11 % slower.
 // Every wait is bounded; a CTA that gives up records kErrPipelineTimeout,
 // waits (bounded) for its copies and MMAs, frees its tensor memory and
 // returns.
@@ -138,21 +140,23 @@ cudaError_t launch_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t
 
 namespace tc {
 
-constexpr int kBM = 128, kBN = 256, kBK = 256;       // tile: rows of A, rows of W, elements of K
-constexpr int kStagesG = 4;
+constexpr int kBM = 128, kBN = 128, kBK = 256;       // tile: rows of A, rows of W, elements of K
+constexpr int kStagesG = 3;
+constexpr int kCtasPerSm = 2;
 constexpr int kABytes = kBM * kBK / 2;               // 16 KB
-constexpr int kBBytes = kBN * kBK / 2;               // 32 KB
+constexpr int kBBytes = kBN * kBK / 2;               // 16 KB
 constexpr int kSfaBytes = (kBM / 128) * (kBK / 64) * 512;   // 2 KB
-constexpr int kSfbBytes = (kBN / 128) * (kBK / 64) * 512;   // 4 KB
+constexpr int kSfbBytes = (kBN / 128) * (kBK / 64) * 512;   // 2 KB
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kEpilogueWarps = 4;
 constexpr int kGemmThreads = 64 + 32 * kEpilogueWarps;   // loader warp, MMA warp, epilogue warps
-constexpr int kTmemCols = 512;
-// Tensor-memory columns: accumulator 0..255, then per stage s the scale
-// factors of that stage's k-tile (A 16 columns, W 32), so that copying the
-// next stage's scales never waits for the MMAs reading this stage's.
-constexpr uint32_t kTmemSf0 = 256;
-constexpr uint32_t kTmemSfStage = 48;
+constexpr int kTmemCols = 256;
+// Tensor-memory columns: accumulator 0..127, then per stage s the scale
+// factors of that stage's k-tile (A 16 columns, W 16: four MMAs of 4 columns
+// each), so that copying the next stage's scales never waits for the MMAs
+// reading this stage's.
+constexpr uint32_t kTmemSf0 = kBN;
+constexpr uint32_t kTmemSfStage = 32;
 constexpr uint32_t kTmemSfbOff = 16;
 static_assert(kTmemSf0 + kStagesG * kTmemSfStage <= (uint32_t)kTmemCols, "scale factors exceed the allocation");
 constexpr int kGemmSmem = kStagesG * kStageBytes + 1024 + 256;
@@ -247,12 +251,12 @@ struct GemmArgs {
 };
 
 // Y[m][n] = s_a s_w sum over plane pairs and k of A_p[m][k] W_q[n][k].
-// Persistent: CTA b takes output tiles b, b + G, ...  Warp 0 (one thread)
+// Persistent: CTA b of G takes output tiles b, b + G, ...  Warp 0 (one thread)
 // loads, warp 1 (one thread) issues the MMAs and owns the tensor memory,
 // warps 2-5 drain the accumulator (warp w reads lane quadrant w % 4).  The
 // loads run ahead across tile boundaries; the MMAs of a tile wait until the
 // previous tile's accumulator has been read ("acc_empty").
-__global__ void __launch_bounds__(tc::kGemmThreads, 1)
+__global__ void __launch_bounds__(tc::kGemmThreads, tc::kCtasPerSm)
     gemm_w4a4_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, GemmArgs g)
 {
     using namespace tc;
@@ -301,7 +305,6 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
     const int64_t iters = kt_per_seg * g.a_planes * g.w_planes;   // k-tiles per output tile
     const int64_t atoms_k = g.K / 64;                       // scale atoms per 128-row block
     const int64_t half_k = g.K / 2;                         // bytes of one plane row
-    const int64_t n_rb = (g.N + 127) / 128;                 // 128-row blocks of W's scale atoms
     auto tile_mn = [&](int64_t j, int64_t& mt, int64_t& nt) {
         const int64_t tile = (int64_t)blockIdx.x + j * gridDim.x;
         mt = tile / n_tiles_n;
@@ -315,8 +318,7 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
         for (int64_t j = 0; j < my_tiles && ok; ++j) {
             int64_t mt, nt;
             tile_mn(j, mt, nt);
-            const bool second_rb = 2 * nt + 1 < n_rb;
-            const uint32_t tx = (uint32_t)(kABytes + kBBytes + kSfaBytes + (second_rb ? kSfbBytes : kSfbBytes / 2));
+            const uint32_t tx = (uint32_t)(kABytes + kBBytes + kSfaBytes + kSfbBytes);
             for (int64_t i = 0; i < iters; ++i, ++gi) {
                 const int s = (int)(gi % kStagesG);
                 if (gi >= kStagesG && !mbar_wait(empty(s), (uint32_t)(((gi / kStagesG) - 1) & 1))) {
@@ -329,10 +331,7 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
                 tc::tma_load_2d(stage_a(s), &amap, (int)(pa * half_k + kt * (kBK / 2)), (int)(mt * kBM), full(s));
                 tc::tma_load_2d(stage_b(s), &wmap, (int)(pw * half_k + kt * (kBK / 2)), (int)(nt * kBN), full(s));
                 tc::bulk_load(stage_sfa(s), g.a_sf + (mt * atoms_k + 4 * kt) * 512, kSfaBytes, full(s));
-                tc::bulk_load(stage_sfb(s), g.w_sf + ((2 * nt) * atoms_k + 4 * kt) * 512, kSfbBytes / 2, full(s));
-                if (second_rb)
-                    tc::bulk_load(stage_sfb(s) + kSfbBytes / 2, g.w_sf + ((2 * nt + 1) * atoms_k + 4 * kt) * 512,
-                                  kSfbBytes / 2, full(s));
+                tc::bulk_load(stage_sfb(s), g.w_sf + (nt * atoms_k + 4 * kt) * 512, kSfbBytes, full(s));
             }
         }
         if (!ok) {
@@ -357,18 +356,17 @@ __global__ void __launch_bounds__(tc::kGemmThreads, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                // scale atoms -> tensor memory: SFA 4 columns per MMA, SFB 8 (two 128-row blocks)
+                // scale atoms -> tensor memory: 4 columns per MMA for A and for W
                 const uint32_t sfa = tmem + kTmemSf0 + kTmemSfStage * (uint32_t)s, sfb = sfa + kTmemSfbOff;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     tc::copy_atom_to_tmem(sfa + 4u * q, tc::desc_atom(stage_sfa(s) + 512u * q));
-                    tc::copy_atom_to_tmem(sfb + 8u * q, tc::desc_atom(stage_sfb(s) + 512u * q));
-                    tc::copy_atom_to_tmem(sfb + 8u * q + 4u, tc::desc_atom(stage_sfb(s) + kSfbBytes / 2 + 512u * q));
+                    tc::copy_atom_to_tmem(sfb + 4u * q, tc::desc_atom(stage_sfb(s) + 512u * q));
                 }
                 const uint64_t da = tc::desc_sw128(stage_a(s)), db = tc::desc_sw128(stage_b(s));
 #pragma unroll
                 for (int q = 0; q < 4; ++q)   // K = 64 per MMA: 32 bytes along the swizzled row
-                    tc::mma_block16(tmem, da + 2u * q, db + 2u * q, sfa + 4u * q, sfb + 8u * q,
+                    tc::mma_block16(tmem, da + 2u * q, db + 2u * q, sfa + 4u * q, sfb + 4u * q,
                                     (i > 0 || q > 0) ? 1u : 0u);
                 tc::commit_to(empty(s));
             }
@@ -465,7 +463,8 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
     g.w_planes = w_np;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
     if (tiles >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-    const int64_t grid = tiles < sm_count() ? tiles : sm_count();   // persistent: one CTA per SM
+    const int64_t cap = (int64_t)kCtasPerSm * sm_count();           // persistent: two CTAs per SM
+    const int64_t grid = tiles < cap ? tiles : cap;
     const cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                kGemmSmem);
     if (e != cudaSuccess) return e;
