@@ -213,14 +213,22 @@ fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
     if (bits == nullptr) return FP4Q_ERROR_INVALID_VALUE;
     fp4q_status_t s = check_device();
     if (s != FP4Q_SUCCESS) return s;
-    unsigned int v = 0, w = 0, u = 0;
+    unsigned int v = 0, w = 0, u = 0, z = 0;
     if (read_device_errors(&v, clear != 0) != cudaSuccess || read_batch_device_errors(&w, clear != 0) != cudaSuccess ||
-        read_gemm_device_errors(&u, clear != 0) != cudaSuccess) {
+        read_gemm_device_errors(&u, clear != 0) != cudaSuccess ||
+        read_selftest_device_errors(&z, clear != 0) != cudaSuccess) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }
-    *bits = v | w | u;
+    *bits = v | w | u | z;
     return FP4Q_SUCCESS;
+}
+
+fp4q_status_t fp4q_selftest_timeout(fp4q_stream_t stream)
+{
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_timeout_selftest(reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int64_t fp4q_outlier_capacity(int64_t cols, double max_frac)

@@ -69,6 +69,10 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
                              int64_t N, int64_t K, uint16_t* y, int64_t ldy, cudaStream_t st);
 cudaError_t read_gemm_device_errors(unsigned int* bits, bool clear);
 
+// Failure-path self-test (fp4q_selftest.cu).
+cudaError_t launch_timeout_selftest(cudaStream_t st);
+cudaError_t read_selftest_device_errors(unsigned int* bits, bool clear);
+
 // Sparse outlier separation (fp4q_outliers.cu).
 int64_t outlier_capacity(int64_t cols, double max_frac);
 cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, double k, int64_t cap,

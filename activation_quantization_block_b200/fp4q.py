@@ -33,7 +33,8 @@ ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_quantize", "fp4q_dequantize", "fp4q_error", "fp4q_quantize_noalloc",
                "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch",
                "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm",
-               "fp4q_outlier_capacity", "fp4q_separate_outliers", "fp4q_scatter_outliers")
+               "fp4q_outlier_capacity", "fp4q_separate_outliers", "fp4q_scatter_outliers",
+               "fp4q_selftest_timeout")
 
 
 class TensorDesc(ctypes.Structure):
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.fp4q_separate_outliers.restype = i32
         L.fp4q_scatter_outliers.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp]
         L.fp4q_scatter_outliers.restype = i32
+        L.fp4q_selftest_timeout.argtypes = [vp]
+        L.fp4q_selftest_timeout.restype = i32
         _lib = L
     return _lib
 
@@ -202,6 +205,10 @@ def fp4q_mma_pack(codes, scales, rows, cols, fmt, planes, sf, stream=None) -> in
 def fp4q_gemm(a_planes, a_sf, a_np, a_scale, w_planes, w_sf, w_np, w_scale, M, N, K, y, ldy, stream=None) -> int:
     return lib().fp4q_gemm(_ptr(a_planes), _ptr(a_sf), a_np, _ptr(a_scale), _ptr(w_planes), _ptr(w_sf), w_np,
                            _ptr(w_scale), M, N, K, _ptr(y), ldy, _stream(stream))
+
+
+def fp4q_selftest_timeout(stream=None) -> int:
+    return lib().fp4q_selftest_timeout(_stream(stream))
 
 
 def fp4q_outlier_capacity(cols: int, max_frac: float) -> int:

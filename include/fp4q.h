@@ -225,6 +225,13 @@ FP4Q_API fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* 
  * fails. */
 FP4Q_API fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear);
 
+/* Exercise the failure path above: one kernel arms a pipeline barrier that no
+ * copy will complete and waits on it with the library's bounded wait.  After
+ * 2 s the wait gives up and sets FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT; nothing
+ * faults, traps or hangs, and the context stays usable.  Enqueues one kernel
+ * on `stream`. */
+FP4Q_API fp4q_status_t fp4q_selftest_timeout(fp4q_stream_t stream);
+
 /* Bytes of device scratch held inside the library for fp4q_quantize_noalloc. */
 #define FP4Q_NOALLOC_SCRATCH_BYTES 49152
 

@@ -49,3 +49,27 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(fmt, rotate):
         assert torch.equal(got[1], ref[1])                     # scales: bit-exact
         assert torch.equal(got[2], ref[2])                     # tensor scale: bit-exact
         assert abs(got[3].item() - ref[3].item()) <= 1e-5 * ref[3].item()   # MSE: 1e-5 relative
+
+
+def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
+    """Failure path on the GPU without a fault: a barrier that nothing completes.
+    The bounded wait gives up after 2 s, the error word says so, and the next
+    call quantizes correctly."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import time
+    dev = torch.device("cuda:0")
+    assert fp4q.fp4q_device_errors(clear=True)[0] == 0
+    t0 = time.perf_counter()
+    assert fp4q.fp4q_selftest_timeout() == 0
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 >= 1.5                       # the wait ran to its limit
+    st, bits = fp4q.fp4q_device_errors(clear=True)
+    assert st == 0 and bits == 0x1                                # FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT
+    assert fp4q.fp4q_device_errors()[1] == 0                      # cleared
+    x = synthetic.llm_weight(256, 1024, seed=5, device=dev)
+    q = fp4q.quantize(x, "nvfp4_razer")
+    y = fp4q.dequantize(q, "nvfp4_razer")
+    torch.cuda.synchronize()
+    assert fp4q.fp4q_device_errors()[1] == 0
+    assert torch.isfinite(q.mse).all() and 0 < q.mse.item() < 1e-4 and y.shape == x.shape
