@@ -5,20 +5,19 @@
 // sect. 2 (sparse outlier separation): weights with |w - mu| > k sigma (k = 4,
 // at most 2 % of the weights) are kept apart as fp16 values at their
 // positions, and the bulk, with the group mean in their place, is quantized.
-// The group is a matrix row.  One CTA per row:
+// The group is a matrix row, handled by one warp (rows of up to 8192 elements)
+// or one CTA, the row copied once into shared memory:
 //   1. mu = sum / n and sigma = sqrt(sum (x - mu)^2 / n) in fp64 (fixed-order
-//      CTA reductions), threshold T = k sigma;
-//   2. c = #(|x - mu| > T); when c exceeds cap = floor(max_frac * n), T becomes
+//      reductions), threshold T = k sigma;
+//   2. one pass writes the bulk row (the mean, rounded to bf16, at every
+//      outlier) and the outliers in column order, their slots from prefix
+//      counts; |x - mu| > T is decided in fp32 outside a guard band that covers
+//      the fp32 roundings, in fp64 inside it;
+//   3. only if that pass counted more than cap = floor(max_frac * n): T becomes
 //      the cap-th largest deviation, found by bisection on the deviations' fp64
-//      bit patterns (monotone for non-negative values), and the ties at T are
-//      taken from the lowest columns up;
-//   3. one pass in tiles of 2048 elements writes the bulk row (the mean, rounded
-//      to bf16, at every outlier) and the outliers in column order, their slots
-//      from CTA-wide prefix counts.
-// The row is read from global memory once, into shared memory, and every pass
-// reads it there; each thread moves 16 bytes at a time.  Rows of up to 8192
-// elements take one warp each (8 rows per CTA, warp reductions and scans
-// only); longer rows take a CTA each.
+//      bit patterns (monotone for non-negative values), ties at T are taken
+//      from the lowest columns up, and step 2 runs again.
+// Each thread moves 16 bytes at a time.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -184,7 +183,9 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
     double thr = a.k * sqrt(cta_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])), shd) /
                             (double)n);
 
-    // 2. count; above the cap, the cap-th largest deviation and its ties
+    // 2. bulk row and outliers in column order, speculatively with k sigma (the
+    // count stays within the cap in the usual case); above the cap, the cap-th
+    // largest deviation, its ties from the lowest column up, and the pass again.
     auto count_where = [&](auto pred) {
         long long c = 0;
         for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
@@ -195,11 +196,71 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
         }
         return cta_count(c, shl);
     };
-    long long tie_need = 0;
-    if (a.cap == 0) {
-        thr = __longlong_as_double(0x7FF0000000000000ll);   // +inf: no slots, no outliers
-    } else if (count_where([&](double d) { return d > thr; }) > a.cap) {
-        // largest u with #(bits(d) >= u) >= cap: the cap-th largest deviation
+    const uint16_t mub = f64_to_bf16_rn(mu);
+    uint16_t* brow = a.bulk + r * a.ldb;
+    // d > t in fp32 outside a band covering the fp32 roundings of mu, t and d
+    // (2^-20 of |mu| + t), in fp64 inside it; slots past the capacity are not written
+    auto compact = [&](double t, long long tie_need, bool none) -> long long {
+        const float mu32 = (float)mu, t32 = (float)t;
+        const float band = 0x1p-20f * (fabsf(mu32) + t32);
+        long long done = 0, ties_seen = 0;
+        for (int64_t j0 = 0; j0 < n; j0 += kOutTile) {
+            const int64_t j = j0 + 8 * (int64_t)threadIdx.x;
+            const bool in = j < n;
+            float v[8];
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (in) {
+                w = lds128(row + 2u * (uint32_t)j);
+                load8(row, j, v);
+            }
+            uint32_t gmask = 0, emask = 0;
+            if (in && !none) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float d32 = fabsf(v[i] - mu32);
+                    if (d32 - t32 > band && d32 <= 3.4e38f) {
+                        gmask |= 1u << i;
+                    } else if (!(d32 - t32 < -band)) {
+                        const double d = fabs((double)v[i] - mu);
+                        if (d > t) gmask |= 1u << i;
+                        else if (d == t && tie_need > 0) emask |= 1u << i;
+                    }
+                }
+            }
+            int eq_total;
+            int rank = (int)ties_seen + cta_exclusive_scan(__popc(emask), shi, &eq_total);
+            uint32_t omask = gmask;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (emask & (1u << i)) {
+                    if (rank < tie_need) omask |= 1u << i;
+                    ++rank;
+                }
+            ties_seen += eq_total;
+            int tot;
+            long long slot = done + cta_exclusive_scan(__popc(omask), shi, &tot);
+            if (in) {
+                uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (omask & (1u << i)) {
+                        const uint32_t sh = (i & 1) ? 16u : 0u;
+                        u[i >> 1] = (u[i >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
+                        if (slot < a.cap) {
+                            a.out_cols[r * a.cap + slot] = (uint16_t)(j + i);
+                            a.out_vals[r * a.cap + slot] =
+                                __half_as_ushort(__float2half_rn(fminf(fmaxf(v[i], -65504.0f), 65504.0f)));
+                        }
+                        ++slot;
+                    }
+                *reinterpret_cast<uint4*>(brow + j) = make_uint4(u[0], u[1], u[2], u[3]);
+            }
+            done += tot;
+        }
+        return done;
+    };
+    long long total = compact(thr, 0, a.cap == 0);
+    if (a.cap > 0 && total > a.cap) {
         unsigned long long lo = 0ull, hi = 0x7FF0000000000000ull;   // bits of 0 and of +inf
         while (hi - lo > 1ull) {
             const unsigned long long mid = lo + (hi - lo) / 2;
@@ -208,62 +269,9 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
             else hi = mid;
         }
         thr = __longlong_as_double((long long)lo);
-        tie_need = a.cap - count_where([&](double d) { return d > thr; });
+        total = compact(thr, a.cap - count_where([&](double d) { return d > thr; }), false);
     }
-
-    // 3. bulk row and outliers in column order
-    const uint16_t mub = f64_to_bf16_rn(mu);
-    uint16_t* brow = a.bulk + r * a.ldb;
-    int64_t done = 0, ties_seen = 0;
-    for (int64_t j0 = 0; j0 < n; j0 += kOutTile) {
-        const int64_t j = j0 + 8 * (int64_t)t;
-        const bool in = j < n;
-        float v[8];
-        uint4 w = make_uint4(0, 0, 0, 0);
-        if (in) {
-            w = lds128(row + 2u * (uint32_t)j);
-            load8(row, j, v);
-        }
-        int gt = 0, eq = 0;
-        uint32_t gmask = 0, emask = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const double d = in ? fabs((double)v[i] - mu) : -1.0;
-            if (d > thr) { gmask |= 1u << i; ++gt; }
-            else if (d == thr && tie_need > 0) { emask |= 1u << i; ++eq; }
-        }
-        int eq_total;
-        const int eq_before = cta_exclusive_scan(eq, shi, &eq_total);
-        // ties kept: those whose rank among the row's ties is below tie_need
-        uint32_t omask = gmask;
-        int rank = (int)(ties_seen + eq_before);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (emask & (1u << i)) {
-                if (rank < tie_need) omask |= 1u << i;
-                ++rank;
-            }
-        ties_seen += eq_total;
-        const int cnt = __popc(omask);
-        int tot;
-        int slot = (int)done + cta_exclusive_scan(cnt, shi, &tot);
-        if (in) {
-            uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (omask & (1u << i)) {
-                    const uint32_t sh = (i & 1) ? 16u : 0u;
-                    u[i >> 1] = (u[i >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
-                    a.out_cols[r * a.cap + slot] = (uint16_t)(j + i);
-                    a.out_vals[r * a.cap + slot] =
-                        __half_as_ushort(__float2half_rn(fminf(fmaxf(v[i], -65504.0f), 65504.0f)));
-                    ++slot;
-                }
-            *reinterpret_cast<uint4*>(brow + j) = make_uint4(u[0], u[1], u[2], u[3]);
-        }
-        done += tot;
-    }
-    if (t == 0) a.out_count[r] = (int32_t)done;
+    if (t == 0) a.out_count[r] = (int32_t)total;
 }
 
 // The same, one warp per row (rows of at most 8192 elements): warp w of CTA b
