@@ -260,22 +260,39 @@ __device__ __forceinline__ float exp2i(int k)
 
 // y <- H32 y (Sylvester order: H_ij = (-1)^popcount(i & j)), fp32 butterflies,
 // then y <- RN(y * RN(1/sqrt 32)).  The transform is its own inverse.
+// Stage h = 1 pairs neighbours and runs scalar; stages h = 2..16 pair whole
+// pairs (y[i], y[i+1]) with (y[i+h], y[i+h+1]) and run two butterflies per
+// packed add / sub.  Every lane rounds as the scalar operation would, so the
+// result is the same bit for bit.
 __device__ __forceinline__ void wht32_inplace(float* y)
 {
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
+    for (int i = 0; i < 32; i += 2) {
+        const float a = y[i], b = y[i + 1];
+        y[i] = a + b;
+        y[i + 1] = a - b;
+    }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+    for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
             if ((i & h) == 0) {
-                float a = y[i], b = y[i + h];
-                y[i] = a + b;
-                y[i + h] = a - b;
+                const float2 a = make_float2(y[i], y[i + 1]), b = make_float2(y[i + h], y[i + h + 1]);
+                const float2 s = add2_rn(a, b), d = sub2_rn(a, b);
+                y[i] = s.x;
+                y[i + 1] = s.y;
+                y[i + h] = d.x;
+                y[i + h + 1] = d.y;
             }
         }
     }
     const float c = wht_scale();
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(y[i], c);
+    for (int i = 0; i < 32; i += 2) {
+        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(c, c));
+        y[i] = p.x;
+        y[i + 1] = p.y;
+    }
 }
 
 // ---- loads / stores -------------------------------------------------------
