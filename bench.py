@@ -377,7 +377,7 @@ def main():
     # ---- end to end from pinned host memory -------------------------------------------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, tensors, fmt, L, dev)
+        e2e = run_e2e(args, tensors, fmt, L, dev, world)
 
     del tensors
     torch.cuda.empty_cache()
@@ -408,11 +408,13 @@ def main():
     return 0
 
 
-def run_e2e(args, tensors, fmt, L, dev):
+def run_e2e(args, tensors, fmt, L, dev, world=1):
     """Same metric from pinned host buffers: every step copies each group of
     tensors in (one layer in batch mode, one tensor per call otherwise),
     quantizes it and copies codes, scales, tensor scales and MSEs back; copies
-    of one group overlap the kernels of the other (two buffer sets, 3 streams)."""
+    of one group overlap the kernels of the other (two buffer sets, 3 streams).
+    With several ranks the job's value is all ranks' elements over the slowest
+    rank's time, and the bytes are all ranks' copies."""
     import torch
     from activation_quantization_block_b200 import fp4q
     per = len(layer_shapes()) if args.mode == "batch" else 1
@@ -487,10 +489,10 @@ def run_e2e(args, tensors, fmt, L, dev):
         step()
     t1.record(d2h)     # the last D2H is ordered after every copy and kernel of the steps
     torch.cuda.synchronize()
-    dt = t0.elapsed_time(t1) / 1e3 / args.e2e_steps
-    elements = sum(h.numel() for h in host_in)
+    dt = max_over_ranks(t0.elapsed_time(t1), world, dev) / 1e3 / args.e2e_steps
+    elements = sum(h.numel() for h in host_in) * world
     h2d_bytes = 2 * elements
-    d2h_bytes = sum(o.codes.numel() + o.scales.numel() + 4 + 8 for o in host_out)
+    d2h_bytes = sum(o.codes.numel() + o.scales.numel() + 4 + 8 for o in host_out) * world
     # the host copies equal the device results
     ok = all(torch.equal(host_out[k].codes, tensors[k][2].codes.cpu()) for k in (0, len(tensors) - 1))
     return {"value": elements / dt, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
