@@ -753,3 +753,81 @@ def test_outliers_against_numpy_statistics(orc):
         keep[cand] = False
         assert np.array_equal(bulk[r, keep], x[r, keep])
     assert bound >= 4                                              # rows where the cap binds
+
+
+# ---------------------------------------------------------------- negation symmetry and constants
+
+def _special_gains(blk_x, sb, ts, fmt):
+    """Exact gains (Fractions) of each special value for one 16-block, from the
+    block's scaled values as the encoder forms them."""
+    wmode = fmt == "nvfp4_razer_w"
+    sval = bf.E3M3[sb & 0x3F] if wmode else bf.e4m3_from_bits(sb & 0x7F)
+    den = np.float32(np.float32(sval) * np.float32(ts))
+    r = np.float32(np.float32(1) / den)
+    v = [np.float32(np.float32(x) * r) for x in blk_x]
+    specials = (5.0, -5.0, 2.5, -2.5) if wmode else (5.0, -5.0)
+    gains = []
+    for sp in specials:
+        g = Fraction(0)
+        for vi in v:
+            fv = Fraction(float(vi))
+            q = Fraction(bf.E2M1[bf.e2m1_nearest(float(vi))])
+            if abs(fv - sp) < abs(fv - q):
+                g += (fv - q) ** 2 - (fv - sp) ** 2
+        gains.append(g)
+    return gains
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "nvfp4_razer_w", "mxfp4", "mxfp4_ceil"])
+def test_negating_the_input_negates_the_encoding(orc, fmt):
+    """quantize(-x): the same block scale magnitudes and error; nonzero codes flip
+    their sign bit; RaZeR selectors flip their sign (activation bit 7; weight bit 6,
+    so +5 <-> -5 and +2.5 <-> -2.5) -- except in blocks where the best gains of a
+    special value and its negation tie, which both encodings resolve to the
+    positive one (the lower selector): those are checked to be exact ties."""
+    from activation_quantization_block_b200 import synthetic
+    x = synthetic.llm_weight(32, 256, seed=45)
+    xb = synthetic.bf16_bits(x)
+    nb = synthetic.bf16_bits(-x)
+    xf = bf.bits_to_f32(xb)
+    c, s, ts, sse = orc.quantize(xb, fmt, nthreads=2)
+    cn, sn, tsn, ssen = orc.quantize(nb, fmt, nthreads=2)
+    assert ts == tsn
+    B = 32 if fmt.startswith("mxfp4") else 16
+    q = bf.unpack_codes(c, 256).reshape(32, 256 // B, B)
+    qn = bf.unpack_codes(cn, 256).reshape(32, 256 // B, B)
+    mag_mask = {"nvfp4": 0xFF, "nvfp4_razer": 0x7F, "nvfp4_razer_w": 0x3F}.get(fmt, 0xFF)
+    assert np.array_equal(s & mag_mask, sn & mag_mask)
+    ties = 0
+    for r in range(32):
+        for b in range(256 // B):
+            a, an = q[r, b], qn[r, b]
+            sel_flip = {"nvfp4_razer": 0x80, "nvfp4_razer_w": 0x40}.get(fmt, 0)
+            special = a == 8
+            mirrored = (np.array_equal(an[(a & 7) != 0], a[(a & 7) != 0] ^ 8) and
+                        np.array_equal(an[(a & 7) == 0], a[(a & 7) == 0]))
+            if fmt in ("nvfp4_razer", "nvfp4_razer_w") and special.any():
+                mirrored = mirrored and int(sn[r, b]) == int(s[r, b]) ^ sel_flip
+            elif fmt in ("nvfp4_razer", "nvfp4_razer_w"):
+                mirrored = mirrored and int(sn[r, b]) == int(s[r, b])
+            if not mirrored:
+                assert fmt in ("nvfp4_razer", "nvfp4_razer_w"), (r, b)
+                g = _special_gains(xf[r, 16 * b:16 * b + 16], int(s[r, b]), ts, fmt)
+                best = max(g)
+                pos_neg = [(g[i], g[i + 1]) for i in range(0, len(g), 2)]
+                assert any(gp == gn == best for gp, gn in pos_neg), (r, b, g)
+                ties += 1
+    if fmt in ("nvfp4", "mxfp4", "mxfp4_ceil"):
+        assert sse == ssen and ties == 0
+
+
+def test_the_kernels_second_pair_is_the_oracles():
+    """The weight mode's second special-value pair is one constant on each side (they
+    share no code): the CUDA source's value equals the oracle's default."""
+    import os
+    import re
+    import oracle
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = open(os.path.join(root, "activation_quantization_block_b200", "csrc", "fp4q_common.cuh")).read()
+    m = re.search(r"constexpr float kRazerWPair = ([0-9.]+)f;", src)
+    assert m and float(m.group(1)) == oracle.razer_w_pair() == 2.5
