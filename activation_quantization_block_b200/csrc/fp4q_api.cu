@@ -9,6 +9,7 @@
 
 #include "fp4q.h"
 #include "fp4q_internal.h"
+#include "fp4q_scale.h"
 
 using namespace fp4q;
 
@@ -206,6 +207,31 @@ fp4q_status_t fp4q_error(const void* x, int64_t ldx,
                                sse_part, &n_sse, st));
     if (s != FP4Q_SUCCESS) return s;
     return from_cuda(launch_sse_finalize(sse_part, n_sse, (double)n, mse, st));
+}
+
+fp4q_status_t fp4q_tensor_scale(const void* x, int64_t rows, int64_t cols, int64_t ldx, fp4q_format_t fmt,
+                                int rotate, float* tensor_scale, void* workspace, size_t workspace_bytes,
+                                fp4q_stream_t stream)
+{
+    fp4q_status_t s = check_shape(rows, cols, fmt, rotate);
+    if (s != FP4Q_SUCCESS) return s;
+    if (fmt == FP4Q_MXFP4 || tensor_scale == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    if (!aligned(tensor_scale, 4)) return FP4Q_ERROR_MISALIGNED;
+    const int64_t n = rows * cols;
+    if (n > 0) {
+        if ((s = check_matrix(x, cols, ldx)) != FP4Q_SUCCESS) return s;
+        if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < kWorkspaceBytes)
+            return FP4Q_ERROR_WORKSPACE;
+    }
+    if ((s = check_device()) != FP4Q_SUCCESS) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n == 0) return from_cuda(cudaMemsetAsync(tensor_scale, 0, sizeof(float), st));
+    float* amax_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsAmaxOffset);
+    const Geometry g = make_geometry(rows, cols, ldx);
+    int n_amax = 0;
+    s = from_cuda(launch_amax(static_cast<const uint16_t*>(x), g, rotate, amax_part, &n_amax, st));
+    if (s != FP4Q_SUCCESS) return s;
+    return from_cuda(launch_tensor_scale(amax_part, n_amax, fmt, tensor_scale, st));
 }
 
 fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)

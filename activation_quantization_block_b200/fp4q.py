@@ -34,7 +34,7 @@ ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch",
                "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm",
                "fp4q_outlier_capacity", "fp4q_separate_outliers", "fp4q_scatter_outliers",
-               "fp4q_selftest_timeout")
+               "fp4q_selftest_timeout", "fp4q_tensor_scale")
 
 
 class TensorDesc(ctypes.Structure):
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.fp4q_scatter_outliers.restype = i32
         L.fp4q_selftest_timeout.argtypes = [vp]
         L.fp4q_selftest_timeout.restype = i32
+        L.fp4q_tensor_scale.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, sz, vp]
+        L.fp4q_tensor_scale.restype = i32
         _lib = L
     return _lib
 
@@ -155,6 +157,12 @@ def fp4q_error(x, ldx, codes, scales, tensor_scale, rows, cols, fmt, rotate, mse
     return lib().fp4q_error(_ptr(x), ldx, _ptr(codes), _ptr(scales), _ptr(tensor_scale), rows, cols,
                             _fmt(fmt), int(rotate), _ptr(mse), _ptr(workspace), workspace_bytes,
                             _stream(stream))
+
+
+def fp4q_tensor_scale(x, rows, cols, ldx, fmt, rotate, tensor_scale, workspace, workspace_bytes,
+                      stream=None) -> int:
+    return lib().fp4q_tensor_scale(_ptr(x), rows, cols, ldx, _fmt(fmt), int(rotate), _ptr(tensor_scale),
+                                   _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def fp4q_quantize_noalloc(x, rows, cols, ldx, fmt, rotate, flags, codes, scales, tensor_scale, mse,
@@ -301,6 +309,19 @@ def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_sc
     st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize")
     return Quantized(codes, scales, ts, mse)
+
+
+def tensor_scale(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, out: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The tensor scale s_t of an NVFP4 format alone (float32 [1] on x's device): the value quantize
+    computes when no tensor_scale is given."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda:
+        raise TypeError("x must be a bf16 CUDA tensor")
+    rows, cols, ld = _rows_cols_ld(x)
+    ts = out if out is not None else torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else workspace_for(x.device, stream)
+    _check(fp4q_tensor_scale(x, rows, cols, ld, fmt, rotate, ts, ws, ws.numel(), stream), "fp4q_tensor_scale")
+    return ts
 
 
 def empty_like_quantized(x: torch.Tensor, fmt, want_mse: bool = True) -> Quantized:

@@ -95,7 +95,7 @@
 extern "C" {
 #endif
 
-#define FP4Q_ABI_VERSION 2
+#define FP4Q_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define FP4Q_API __attribute__((visibility("default")))
@@ -176,6 +176,28 @@ FP4Q_API fp4q_status_t fp4q_error(const void* x, int64_t ldx,
                          const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
                          int64_t rows, int64_t cols, fp4q_format_t fmt, int rotate,
                          double* mse, void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
+
+/* The tensor scale alone: *tensor_scale = s_t of x (bf16 [rows][ldx]) for an
+ * NVFP4 format, exactly the value fp4q_quantize computes and writes without
+ * FP4Q_FLAG_TENSOR_SCALE_GIVEN (the absmax of the rotated values when
+ * rotate = 1).
+ *
+ * Purpose: one tensor split by rows over several devices.  The map from the
+ * absmax to s_t is monotone (a correctly rounded division by a positive
+ * constant), so the largest s_t over the parts equals the s_t of the whole
+ * tensor.  Each part calls this, the parts exchange the maximum, and each
+ * part then calls fp4q_quantize with the flag; the codes and scales equal
+ * those of the whole tensor quantized on one device.
+ *  fmt            FP4Q_NVFP4, FP4Q_NVFP4_RAZER or FP4Q_NVFP4_RAZER_W; MXFP4
+ *                 has no tensor scale (FP4Q_ERROR_INVALID_VALUE).
+ *  tensor_scale   device output, 1 float, 4-byte aligned.  0 when rows or
+ *                 cols is 0.
+ *  workspace      as fp4q_quantize.
+ * Validation as fp4q_quantize.  Enqueues two kernels: the absmax pass and a
+ * one-CTA reduction of its per-CTA maxima. */
+FP4Q_API fp4q_status_t fp4q_tensor_scale(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                         fp4q_format_t fmt, int rotate, float* tensor_scale,
+                                         void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
 
 /* One tensor of a batch: as the arguments of fp4q_quantize (device pointers;
  * mse may be NULL, tensor_scale may be NULL for MXFP4). */

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_status_strings_workspace():
-    assert fp4q.fp4q_abi_version() == 2
+    assert fp4q.fp4q_abi_version() == 3
     for code in range(7):
         assert fp4q.fp4q_status_string(code)
     assert fp4q.fp4q_status_string(99) == "unknown status"
@@ -257,6 +257,30 @@ def test_scatter_outliers_rejects_bad_arguments(kw, expect):
     args = dict(out_cols=A, out_vals=A, out_count=A, rows=4, cols=64, cap=3, y=A, ldy=64, stream=0)
     args.update(kw)
     assert fp4q.fp4q_scatter_outliers(**args) == ST[expect]
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(fmt=2), "FP4Q_ERROR_INVALID_VALUE"),                   # MXFP4 has no tensor scale
+    (dict(fmt=4), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rotate=2), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(rows=-1), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(tensor_scale=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(tensor_scale=A + 2), "FP4Q_ERROR_MISALIGNED"),
+    (dict(cols=40, ldx=40), "FP4Q_ERROR_SHAPE"),
+    (dict(rotate=1, cols=48, ldx=48), "FP4Q_ERROR_SHAPE"),
+    (dict(ldx=32), "FP4Q_ERROR_SHAPE"),
+    (dict(x=None), "FP4Q_ERROR_INVALID_VALUE"),
+    (dict(x=A + 8), "FP4Q_ERROR_MISALIGNED"),
+    (dict(ldx=68), "FP4Q_ERROR_MISALIGNED"),
+    (dict(workspace=None), "FP4Q_ERROR_WORKSPACE"),
+    (dict(workspace=A + 8), "FP4Q_ERROR_WORKSPACE"),
+    (dict(workspace_bytes=WS - 1), "FP4Q_ERROR_WORKSPACE"),
+])
+def test_tensor_scale_rejects_bad_arguments(kw, expect):
+    args = dict(x=A, rows=4, cols=64, ldx=64, fmt=1, rotate=0, tensor_scale=A, workspace=A, workspace_bytes=WS,
+                stream=0)
+    args.update(kw)
+    assert fp4q.fp4q_tensor_scale(**args) == ST[expect]
 
 
 def test_build_entry_expects_the_header_abi_version():
