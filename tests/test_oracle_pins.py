@@ -215,6 +215,27 @@ def test_tensor_scale_maps_amax_to_6x448(orc):
         assert orc.tensor_scale_from_amax(2688.0 * 2.0 ** k) == 2.0 ** k
 
 
+def test_tensor_amax_is_the_largest_magnitude(orc):
+    x = (np.random.default_rng(21).standard_normal((300, 256)) * 0.02).astype(np.float32)
+    x[123, 45] = -0.75
+    xb = orc.f32_to_bf16(x)
+    assert orc.tensor_amax(xb, False) == np.abs(bf.bits_to_f32(xb)).max() == 0.75
+
+
+@pytest.mark.parametrize("fmt,c", [("nvfp4", 2688), ("nvfp4_razer_w", 180)])
+def test_tensor_scale_is_the_rounded_quotient_and_monotone(orc, fmt, c):
+    """s_t = RN(A / c): checked against the exact quotient rounded once, and monotone in A
+    (what lets parts of a row-split tensor exchange their s_t instead of their absmax)."""
+    rng = np.random.default_rng(22)
+    a = np.sort(np.concatenate([rng.uniform(0, 50, 400), 10.0 ** rng.uniform(-30, 30, 400)]).astype(np.float32))
+    a = np.concatenate([a, np.nextafter(a, np.float32(np.inf))])
+    a.sort()
+    st = [orc.tensor_scale_from_amax(float(v), fmt) for v in a]
+    for v, s_ in zip(a, st):
+        assert np.float32(s_) == bf.rn_f32(Fraction(float(v)) / c)
+    assert all(x <= y for x, y in zip(st, st[1:]))
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer"])
 def test_max_block_gets_scale_448(orc, fmt):
     rng = np.random.default_rng(17)
