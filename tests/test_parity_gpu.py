@@ -513,3 +513,26 @@ def test_rotated_nvfp4_full_size_sampled(orc, dev, fmt):
     e = fp4q.error(x, q, fmt, rotate=True)
     torch.cuda.synchronize()
     assert rel(q.mse.item(), e.item()) <= 1e-4
+
+
+def test_rejected_calls_leave_no_cuda_error_pending(dev):
+    """Calls rejected by validation return before any CUDA call, so nothing is left pending:
+    a valid call right after them (whose launches check cudaGetLastError) succeeds and matches
+    a clean run."""
+    x = synthetic.llm_weight(64, 256, seed=50, device="cpu").to(dev)
+    want = fp4q.quantize(x, "nvfp4_razer")
+    q = fp4q.empty_like_quantized(x, "nvfp4_razer")
+    ws = torch.empty(fp4q.fp4q_workspace_size(64, 256, 1, 0), dtype=torch.uint8, device=dev)
+    args = dict(x=x, rows=64, cols=256, ldx=256, fmt=1, rotate=0, flags=0, codes=q.codes, scales=q.scales,
+                tensor_scale=q.tensor_scale, mse=q.mse, workspace=ws, workspace_bytes=ws.numel())
+    for kw in (dict(fmt=7), dict(cols=40, ldx=40), dict(ldx=260), dict(codes=None), dict(workspace_bytes=16),
+               dict(rows=-1), dict(flags=8)):
+        assert fp4q.fp4q_quantize(**{**args, **kw}) != 0, kw
+    y = torch.empty_like(x)
+    assert fp4q.fp4q_dequantize(q.codes, q.scales, q.tensor_scale, 64, 256, 9, 0, y, 256) != 0
+    assert fp4q.fp4q_tensor_scale(x, 64, 256, 256, 2, 0, q.tensor_scale, ws, ws.numel()) != 0
+    assert fp4q.fp4q_quantize(**args) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(q.codes, want.codes) and torch.equal(q.scales, want.scales)
+    assert q.tensor_scale.item() == want.tensor_scale.item()
+    assert rel(q.mse.item(), want.mse.item()) <= 1e-12
