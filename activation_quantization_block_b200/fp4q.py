@@ -283,30 +283,55 @@ def _rows_cols_ld(x: torch.Tensor):
     return x.shape[0], x.shape[1], x.stride(0) if x.shape[0] > 1 else x.shape[1]
 
 
+def _device(*tensors) -> torch.device:
+    """The one CUDA device every given tensor (None skipped) lives on.  The C ABI takes device
+    pointers only and cannot tell a host address from a device one, so a host tensor, or a
+    tensor of another device, is rejected here before its address reaches a kernel."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise TypeError("fp4q takes CUDA tensors only")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on two devices: {dev} and {t.device}")
+    if dev is None:
+        raise TypeError("no tensor given")
+    return dev
+
+
+def _bf16(*tensors):
+    for t in tensors:
+        if t is not None and t.dtype != torch.bfloat16:
+            raise TypeError("expected bf16 tensors")
+
+
 def quantize(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, tensor_scale: torch.Tensor | None = None,
              want_mse: bool = True, out: Quantized | None = None, workspace: torch.Tensor | None = None,
              stream=None, mx_ceil: bool = False) -> Quantized:
     """Quantize a bf16 CUDA matrix; returns codes, scales, tensor scale and (optionally) the MSE.
 
     mx_ceil (MXFP4): block exponent without clipping (FP4Q_FLAG_MX_CEIL_SCALE)."""
-    if x.dtype != torch.bfloat16 or not x.is_cuda:
-        raise TypeError("x must be a bf16 CUDA tensor")
+    dev = _device(x, tensor_scale, workspace, *(out or ()))
+    _bf16(x)
     rows, cols, ld = _rows_cols_ld(x)
     f = _fmt(fmt)
     B = block_size(f)
-    dev = x.device
-    if out is None:
-        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
-        scales = torch.empty(rows, cols // B, dtype=torch.uint8, device=dev)
-        ts = torch.zeros(1, dtype=torch.float32, device=dev) if tensor_scale is None else tensor_scale
-        mse = torch.empty(1, dtype=torch.float64, device=dev) if want_mse else None
-    else:
-        codes, scales, ts, mse = out
-        if tensor_scale is not None:
-            ts = tensor_scale
-    ws = workspace if workspace is not None else workspace_for(dev, stream)
-    flags = (FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
-    st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
+    with torch.cuda.device(dev):
+        if out is None:
+            codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+            scales = torch.empty(rows, cols // B, dtype=torch.uint8, device=dev)
+            ts = torch.zeros(1, dtype=torch.float32, device=dev) if tensor_scale is None else tensor_scale
+            mse = torch.empty(1, dtype=torch.float64, device=dev) if want_mse else None
+        else:
+            codes, scales, ts, mse = out
+            if tensor_scale is not None:
+                ts = tensor_scale
+        ws = workspace if workspace is not None else workspace_for(dev, stream)
+        flags = (FLAG_TENSOR_SCALE_GIVEN if tensor_scale is not None else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
+        st = fp4q_quantize(x, rows, cols, ld, f, rotate, flags, codes, scales, ts, mse, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize")
     return Quantized(codes, scales, ts, mse)
 
@@ -315,12 +340,14 @@ def tensor_scale(x: torch.Tensor, fmt="nvfp4_razer", rotate: bool = False, out: 
                  workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """The tensor scale s_t of an NVFP4 format alone (float32 [1] on x's device): the value quantize
     computes when no tensor_scale is given."""
-    if x.dtype != torch.bfloat16 or not x.is_cuda:
-        raise TypeError("x must be a bf16 CUDA tensor")
+    dev = _device(x, out, workspace)
+    _bf16(x)
     rows, cols, ld = _rows_cols_ld(x)
-    ts = out if out is not None else torch.empty(1, dtype=torch.float32, device=x.device)
-    ws = workspace if workspace is not None else workspace_for(x.device, stream)
-    _check(fp4q_tensor_scale(x, rows, cols, ld, fmt, rotate, ts, ws, ws.numel(), stream), "fp4q_tensor_scale")
+    with torch.cuda.device(dev):
+        ts = out if out is not None else torch.empty(1, dtype=torch.float32, device=dev)
+        ws = workspace if workspace is not None else workspace_for(dev, stream)
+        st = fp4q_tensor_scale(x, rows, cols, ld, fmt, rotate, ts, ws, ws.numel(), stream)
+    _check(st, "fp4q_tensor_scale")
     return ts
 
 
@@ -341,14 +368,16 @@ def quantize_batch(xs, fmt="nvfp4_razer", rotate: bool = False, outs=None, scale
     With scale_given, each out's tensor_scale holds the input scale."""
     if not xs:
         return []
-    dev = xs[0].device
-    if outs is None:
-        outs = [empty_like_quantized(x, fmt, want_mse) for x in xs]
-    descs = _descs([tensor_desc(x, q) for x, q in zip(xs, outs)])
-    need = fp4q_batch_workspace_size(len(xs), descs, fmt, rotate)
-    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
-    flags = (FLAG_TENSOR_SCALE_GIVEN if scale_given else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
-    st = fp4q_quantize_batch(len(xs), descs, fmt, rotate, flags, ws, ws.numel(), stream)
+    dev = _device(*xs, workspace, *(t for q in (outs or ()) for t in q))
+    _bf16(*xs)
+    with torch.cuda.device(dev):
+        if outs is None:
+            outs = [empty_like_quantized(x, fmt, want_mse) for x in xs]
+        descs = _descs([tensor_desc(x, q) for x, q in zip(xs, outs)])
+        need = fp4q_batch_workspace_size(len(xs), descs, fmt, rotate)
+        ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+        flags = (FLAG_TENSOR_SCALE_GIVEN if scale_given else 0) | (FLAG_MX_CEIL_SCALE if mx_ceil else 0)
+        st = fp4q_quantize_batch(len(xs), descs, fmt, rotate, flags, ws, ws.numel(), stream)
     _check(st, "fp4q_quantize_batch")
     return outs
 
@@ -356,10 +385,13 @@ def quantize_batch(xs, fmt="nvfp4_razer", rotate: bool = False, outs=None, scale
 def dequantize(q: Quantized, fmt="nvfp4_razer", rotate: bool = False, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """bf16 reconstruction of a quantized matrix."""
+    dev = _device(*q, out)
+    _bf16(out)
     rows, cols = q.codes.shape[0], q.codes.shape[1] * 2
-    y = out if out is not None else torch.empty(rows, cols, dtype=torch.bfloat16, device=q.codes.device)
-    ldy = y.stride(0) if rows > 1 else cols
-    st = fp4q_dequantize(q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, y, ldy, stream)
+    with torch.cuda.device(dev):
+        y = out if out is not None else torch.empty(rows, cols, dtype=torch.bfloat16, device=dev)
+        ldy = y.stride(0) if rows > 1 else cols
+        st = fp4q_dequantize(q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, y, ldy, stream)
     _check(st, "fp4q_dequantize")
     return y
 
@@ -367,11 +399,14 @@ def dequantize(q: Quantized, fmt="nvfp4_razer", rotate: bool = False, out: torch
 def error(x: torch.Tensor, q: Quantized, fmt="nvfp4_razer", rotate: bool = False,
           workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """MSE (fp64 [1] on the device) of the reconstruction against x."""
+    dev = _device(x, *q, workspace)
+    _bf16(x)
     rows, cols, ld = _rows_cols_ld(x)
-    mse = torch.empty(1, dtype=torch.float64, device=x.device)
-    ws = workspace if workspace is not None else workspace_for(x.device, stream)
-    st = fp4q_error(x, ld, q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, mse, ws,
-                    ws.numel(), stream)
+    with torch.cuda.device(dev):
+        mse = torch.empty(1, dtype=torch.float64, device=dev)
+        ws = workspace if workspace is not None else workspace_for(dev, stream)
+        st = fp4q_error(x, ld, q.codes, q.scales, q.tensor_scale, rows, cols, _fmt(fmt), rotate, mse, ws,
+                        ws.numel(), stream)
     _check(st, "fp4q_error")
     return mse
 
@@ -385,26 +420,33 @@ class MmaOperand(NamedTuple):
 
 def mma_operand(q: Quantized, fmt, stream=None) -> MmaOperand:
     """Tensor-core operand form of a quantized NVFP4-family matrix."""
+    dev = _device(*q)
     rows, cols = q.codes.shape[0], q.codes.shape[1] * 2
     npl = fp4q_mma_planes(fmt)
     if npl == 0:
         raise Fp4qError(1, "no operand form for this format")
-    planes = torch.empty(rows, npl * cols // 2, dtype=torch.uint8, device=q.codes.device)
-    sf = torch.empty(max(1, fp4q_mma_sf_bytes(rows, cols)), dtype=torch.uint8, device=q.codes.device)
-    _check(fp4q_mma_pack(q.codes, q.scales, rows, cols, fmt, planes, sf, stream), "fp4q_mma_pack")
+    with torch.cuda.device(dev):
+        planes = torch.empty(rows, npl * cols // 2, dtype=torch.uint8, device=dev)
+        sf = torch.empty(max(1, fp4q_mma_sf_bytes(rows, cols)), dtype=torch.uint8, device=dev)
+        st = fp4q_mma_pack(q.codes, q.scales, rows, cols, fmt, planes, sf, stream)
+    _check(st, "fp4q_mma_pack")
     return MmaOperand(planes, sf, q.tensor_scale, npl)
 
 
 def gemm(a: MmaOperand, w: MmaOperand, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """bf16 y = A^ W^T of two operands in tensor-core form (A: M x K, W: N x K)."""
+    dev = _device(a.planes, a.sf, a.tensor_scale, w.planes, w.sf, w.tensor_scale, out)
+    _bf16(out)
     M, N = a.planes.shape[0], w.planes.shape[0]
     K = a.planes.shape[1] * 2 // a.nplanes
     if w.planes.shape[1] * 2 // w.nplanes != K:
         raise ValueError("inner dimensions differ")
-    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=a.planes.device)
-    ldy = y.stride(0) if M > 1 else N
-    _check(fp4q_gemm(a.planes, a.sf, a.nplanes, a.tensor_scale, w.planes, w.sf, w.nplanes, w.tensor_scale, M, N, K,
-                     y, ldy, stream), "fp4q_gemm")
+    with torch.cuda.device(dev):
+        y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ldy = y.stride(0) if M > 1 else N
+        st = fp4q_gemm(a.planes, a.sf, a.nplanes, a.tensor_scale, w.planes, w.sf, w.nplanes, w.tensor_scale, M, N,
+                       K, y, ldy, stream)
+    _check(st, "fp4q_gemm")
     return y
 
 
@@ -417,22 +459,28 @@ class Outliers(NamedTuple):
 
 def separate_outliers(x: torch.Tensor, k: float = 4.0, max_frac: float = 0.02, stream=None) -> Outliers:
     """Sparse outlier separation of a bf16 CUDA matrix (rows are the groups)."""
+    dev = _device(x)
+    _bf16(x)
     rows, cols, ld = _rows_cols_ld(x)
     cap = fp4q_outlier_capacity(cols, max_frac)
-    dev = x.device
-    o = Outliers(torch.empty(rows, cols, dtype=torch.bfloat16, device=dev),
-                 torch.zeros(rows, max(cap, 1), dtype=torch.int16, device=dev),
-                 torch.zeros(rows, max(cap, 1), dtype=torch.float16, device=dev),
-                 torch.zeros(rows, dtype=torch.int32, device=dev))
-    _check(fp4q_separate_outliers(x, rows, cols, ld, k, max_frac, o.bulk, cols, o.cols, o.vals, o.count, stream),
-           "fp4q_separate_outliers")
+    with torch.cuda.device(dev):
+        o = Outliers(torch.empty(rows, cols, dtype=torch.bfloat16, device=dev),
+                     torch.zeros(rows, max(cap, 1), dtype=torch.int16, device=dev),
+                     torch.zeros(rows, max(cap, 1), dtype=torch.float16, device=dev),
+                     torch.zeros(rows, dtype=torch.int32, device=dev))
+        st = fp4q_separate_outliers(x, rows, cols, ld, k, max_frac, o.bulk, cols, o.cols, o.vals, o.count, stream)
+    _check(st, "fp4q_separate_outliers")
     return o
 
 
 def scatter_outliers(o: Outliers, y: torch.Tensor, max_frac: float = 0.02, stream=None) -> torch.Tensor:
     """Put the outliers of o back into the bf16 reconstruction y (in place)."""
+    dev = _device(*o, y)
+    _bf16(y)
     rows, cols = y.shape
     cap = fp4q_outlier_capacity(cols, max_frac)
     ldy = y.stride(0) if rows > 1 else cols
-    _check(fp4q_scatter_outliers(o.cols, o.vals, o.count, rows, cols, cap, y, ldy, stream), "fp4q_scatter_outliers")
+    with torch.cuda.device(dev):
+        st = fp4q_scatter_outliers(o.cols, o.vals, o.count, rows, cols, cap, y, ldy, stream)
+    _check(st, "fp4q_scatter_outliers")
     return y

@@ -289,3 +289,47 @@ def test_build_entry_expects_the_header_abi_version():
     entry = open(os.path.join(ROOT, "__graft_entry__.py")).read()
     assert f"fp4q_abi_version() == {ver}" in entry
     assert fp4q.fp4q_abi_version() == int(ver)
+
+
+# ---- the torch-level wrappers reject host tensors before any address reaches the library
+
+def _cpu_quantized(rows=4, cols=64):
+    import torch
+    return fp4q.Quantized(torch.zeros(rows, cols // 2, dtype=torch.uint8), torch.zeros(rows, cols // 16, dtype=torch.uint8),
+                          torch.zeros(1), torch.zeros(1, dtype=torch.float64))
+
+
+@pytest.mark.parametrize("call", [
+    lambda x, q: fp4q.quantize(x),
+    lambda x, q: fp4q.tensor_scale(x),
+    lambda x, q: fp4q.quantize_batch([x]),
+    lambda x, q: fp4q.dequantize(q),
+    lambda x, q: fp4q.error(x, q),
+    lambda x, q: fp4q.mma_operand(q, "nvfp4"),
+    lambda x, q: fp4q.separate_outliers(x),
+    lambda x, q: fp4q.scatter_outliers(fp4q.Outliers(x, q.codes, q.codes, q.codes), x),
+])
+def test_wrappers_reject_host_tensors(call):
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="CUDA tensors only"):
+        call(x, _cpu_quantized())
+
+
+def test_gemm_rejects_host_operands():
+    import torch
+    op = fp4q.MmaOperand(torch.zeros(128, 128, dtype=torch.uint8), torch.zeros(512, dtype=torch.uint8),
+                         torch.ones(1), 1)
+    with pytest.raises(TypeError, match="CUDA tensors only"):
+        fp4q.gemm(op, op)
+
+
+def test_device_of_mixed_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        fp4q._device(None, None)
+    with pytest.raises(TypeError):
+        fp4q._device(torch.zeros(1, device="meta"))
+    with pytest.raises(TypeError, match="bf16"):
+        fp4q._bf16(torch.zeros(1))
+    fp4q._bf16(None, torch.zeros(1, dtype=torch.bfloat16))
