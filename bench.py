@@ -231,6 +231,22 @@ def job_throughput(elements_per_rank: int, world: int, steps: int, ms: float) ->
     return elements_per_rank * world * steps / (ms / 1e3)
 
 
+def sha256_of(tensors) -> str:
+    """SHA-256 over the bytes of the given tensors in order (copied to the host); a failure is
+    reported in the string instead of ending the run."""
+    import hashlib
+
+    import torch
+    try:
+        h = hashlib.sha256()
+        for t in tensors:
+            flat = t.detach().contiguous().reshape(-1)
+            h.update(flat.view(torch.uint8).cpu().numpy().tobytes())
+        return h.hexdigest()
+    except Exception as e:  # the digest is a label, not a measurement
+        return f"unavailable: {type(e).__name__}: {e}"
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -298,6 +314,8 @@ def main():
             tensors.append((name, x, q))
     torch.cuda.synchronize()
     elements = sum(x.numel() for _, x, _ in tensors)
+    layer0 = len(layer_shapes())
+    inputs_sha = sha256_of([x for _, x, _ in tensors[:layer0]])
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     ws = torch.zeros(fp4q.fp4q_workspace_size(0, 0, FMT, 0), dtype=torch.uint8, device=dev)
@@ -379,6 +397,7 @@ def main():
 
     # ---- check a result, outside the timed region ---------------------------------
     mses = torch.cat([q.mse for _, _, q in tensors]).cpu()
+    outputs_sha = sha256_of([t for _, _, q in tensors[:layer0] for t in (q.codes, q.scales)])
     assert torch.isfinite(mses).all() and (mses > 0).all()
 
     # ---- end to end from pinned host memory -------------------------------------------
@@ -397,7 +416,9 @@ def main():
                    "api": "fp4q_quantize_batch, one call per step" if args.mode == "batch" else
                           "fp4q_quantize, one call per tensor",
                    "parallelism": f"dp{world} (independent weight sets, no collective)" if world > 1 else "1 GPU",
-                   "l2": f"no flush: each step reads {elements * 2 / 1e9:.2f} GB of inputs (> 126 MB L2)"},
+                   "l2": f"no flush: each step reads {elements * 2 / 1e9:.2f} GB of inputs (> 126 MB L2)",
+                   "inputs_sha256": f"layer 0 of rank 0, 7 bf16 tensors in order: {inputs_sha}"},
+        "outputs_sha256": f"layer 0 of rank 0, codes then scales of each tensor: {outputs_sha}",
         "achieved_gbs": BYTES_PER_ELEMENT * elements * world / (ms_per_step / 1e3) / 1e9,
         "pct_of_nominal_8tbs": 100 * BYTES_PER_ELEMENT * elements / (ms_per_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
         "roofline": roofline,

@@ -85,3 +85,17 @@ def test_clock_sampler_reads_a_running_nvidia_smi(monkeypatch, tmp_path):
     time.sleep(0.5)
     got = s.stop()
     assert got["samples"] >= 2 and got["sm_mhz"] == 1965.0 and got["reasons"] == ["sw_power_cap"]
+
+
+def test_sha256_of_tensors_is_the_digest_of_their_bytes():
+    import hashlib
+
+    import numpy as np
+    import torch
+    a = torch.arange(12, dtype=torch.float32).to(torch.bfloat16).reshape(3, 4)
+    b = torch.arange(6, dtype=torch.uint8)
+    want = hashlib.sha256(a.view(torch.int16).numpy().view(np.uint8).tobytes() + b.numpy().tobytes()).hexdigest()
+    assert bench.sha256_of([a, b]) == want
+    wide = torch.zeros(4, 8, dtype=torch.bfloat16)
+    assert bench.sha256_of([wide[:, :4]]) == bench.sha256_of([torch.zeros(4, 4, dtype=torch.bfloat16)])
+    assert bench.sha256_of([object()]).startswith("unavailable:")
