@@ -1,7 +1,7 @@
 """fp4q oracle: the plain CPU restatement of block-scaled 4-bit quantization.
 
 TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
-the CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
+the CPU-baseline leg and reference arm of ``bench.py`` may import this package.  The CUDA library
 and its Python binding never import, link or call it, and it imports nothing
 from them.
 

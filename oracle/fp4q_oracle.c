@@ -4,8 +4,8 @@
  * remapping, MXFP4, each optionally after a 32-point Walsh-Hadamard rotation).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
- * this file; only the test suite, the smoke check and the CPU-baseline leg of
- * the benchmark use it.  It shares no code, header, table or constant with the
+ * this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline and reference arm use it.  It shares no code, header, table or constant with the
  * CUDA library: every number below is restated here from the pages' text.
  *
  * Sources (title, section):
