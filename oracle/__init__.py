@@ -8,7 +8,7 @@ from them.
 The arithmetic lives in ``fp4q_oracle.c`` (scalar loops, IEEE binary32 /
 binary64, no fast-math); this module is a numpy/ctypes wrapper around it.  The
 header comment of the C file lists the page passages it follows and the
-readings it takes where the pages are silent.  Functions whose result is not
+readings it takes where the cited papers are silent.  Functions whose result is not
 pinned by an independent check are marked "parity unpinned" in their
 docstring; at present every function is pinned by ``tests/test_oracle_pins.py``.
 """

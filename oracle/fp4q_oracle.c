@@ -6,7 +6,7 @@
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
  * this file; only the test suite, the smoke check and the benchmark's CPU
  * baseline and reference arm use it.  It shares no code, header, table or constant with the
- * CUDA library: every number below is restated here from the pages' text.
+ * CUDA library: every number below is restated here from the cited papers' text.
  *
  * Sources (title, section):
  *  [RaZeR]  "RaZeR: Pushing the Limits of NVFP4 Quantization with Redundant
@@ -20,7 +20,7 @@
  *           "S-step" scale from the block maximum, rotations absorbed into the
  *           neighbouring weights).
  *
- * Readings where the pages are silent (each one restated where it is used):
+ * Readings where the papers are silent (each one restated where it is used):
  *  R1 element rounding: nearest E2M1 value, ties to the even code, |v| > 6
  *     saturates to 6, a zero result is always +0 (code 0b0000).
  *  R2 NVFP4 is two-level: a per-tensor fp32 scale s_t = RN(A / (6*448)) with A

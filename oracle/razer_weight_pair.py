@@ -4,8 +4,8 @@
 Remapping", technical summary sect. 2.2: with the two bits an E3M3 block scale
 frees, weights choose per block among four special values -- two pairs fixed
 offline, each a multiple of 0.5; the pair +-5 is the best single pair.  The
-pages do not name the second pair.  This script finds it the way the pages
-describe: over every multiple of 0.5 that is not already an E2M1 value (nor 5)
+paper does not name the second pair.  This script finds it the way the paper
+describes: over every multiple of 0.5 that is not already an E2M1 value (nor 5)
 up to 8, it quantizes a set of seeded synthetic LLM weight matrices in the
 weight mode with {+-5, +-s2} and keeps the s2 with the lowest total squared
 error.  It uses only the oracle.

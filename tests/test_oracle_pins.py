@@ -1,6 +1,6 @@
-"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+"""Pins for the CPU oracle: checks against what the papers and the mathematics fix.
 
-None of these compares the oracle with itself.  Each pin comes from the pages'
+None of these compares the oracle with itself.  Each pin comes from the papers'
 printed values (``tests/golden``), an exhaustive enumeration, exact rational
 arithmetic, a library cast (``ml_dtypes``, ``scipy``), a closed form or an
 invariant -- chosen so that a dropped term, a wrong sign, a wrong tie rule, a
@@ -23,7 +23,7 @@ pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
 # ---------------------------------------------------------------- E2M1 elements
 
-def test_e2m1_value_set_is_the_pages_set(orc):
+def test_e2m1_value_set_is_the_papers_set(orc):
     page = sorted(float(r[0]) for r in bf.read_golden("e2m1_value_set.txt"))
     mine = sorted(orc.e2m1_value(c) for c in range(16))
     assert mine == page
@@ -350,7 +350,7 @@ def test_idempotent_on_representable_inputs(orc, fmt):
 
 # ---------------------------------------------------------------- RaZeR invariants and worked case
 
-def test_razer_special_values_are_the_pages_pair(orc):
+def test_razer_special_values_are_the_papers_pair(orc):
     pair = {int(r[0]): float(r[1]) for r in bf.read_golden("razer_special_values.txt")}
     ts = 1.0
     for sel, val in pair.items():
