@@ -333,3 +333,48 @@ def test_device_of_mixed_tensors():
     with pytest.raises(TypeError, match="bf16"):
         fp4q._bf16(torch.zeros(1))
     fp4q._bf16(None, torch.zeros(1, dtype=torch.bfloat16))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <stdint.h>
+#include "fp4q.h"
+
+int main(void)
+{
+    /* a plain C caller: version, status strings and host-side validation (no device needed) */
+    if (fp4q_abi_version() != FP4Q_ABI_VERSION) return 1;
+    if (fp4q_status_string(FP4Q_ERROR_SHAPE)[0] == 0) return 2;
+    uintptr_t a = (uintptr_t)1 << 20;                      /* fake 16-byte-aligned addresses */
+    size_t ws = fp4q_workspace_size(4, 64, FP4Q_NVFP4_RAZER, 0);
+    fp4q_status_t s = fp4q_quantize((const void*)a, 4, 40, 40, FP4Q_NVFP4_RAZER, 0, 0, (uint8_t*)a, (uint8_t*)a,
+                                    (float*)a, NULL, (void*)a, ws, NULL);
+    if (s != FP4Q_ERROR_SHAPE) return 3;
+    s = fp4q_tensor_scale((const void*)a, 4, 64, 64, FP4Q_MXFP4, 0, (float*)a, (void*)a, ws, NULL);
+    if (s != FP4Q_ERROR_INVALID_VALUE) return 4;
+    s = fp4q_gemm((const uint8_t*)a, (const uint8_t*)a, 3, (const float*)a, (const uint8_t*)a, (const uint8_t*)a, 1,
+                  (const float*)a, 8, 8, 256, (void*)a, 8, NULL);
+    if (s != FP4Q_ERROR_INVALID_VALUE) return 5;
+    if (fp4q_mma_planes(FP4Q_NVFP4_RAZER) != 2 || fp4q_mma_planes(FP4Q_NVFP4) != 1) return 6;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_a_plain_c_program_links_and_calls_the_abi(tmp_path):
+    """The boundary is a C ABI: a C11 program compiles against include/fp4q.h alone, links
+    libfp4q.so and gets the documented statuses from host-side validation."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = fp4q.lib()._name
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    lib, f"-Wl,-rpath,{os.path.dirname(lib)}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
