@@ -461,6 +461,36 @@ def test_e3m3_encode_equals_exhaustive_argmin(orc):
         assert orc.e3m3_encode(np.float32(t)) == bf.e3m3_nearest(min(float(np.float32(t)), 30.0)), t
 
 
+def test_scale_widths_follow_the_paper(orc):
+    """E3M3 codes fit the 6 bits the paper gives the weight scale, and the weight mode's
+    selector lives exactly in the 8 - 6 = 2 bits that frees (tests/golden/scale_bits.txt)."""
+    bits = {r[0]: int(r[1]) for r in bf.read_golden("scale_bits.txt")}
+    assert bits == {"e4m3": 8, "e3m3": 6}
+    free = bits["e4m3"] - bits["e3m3"]
+    codes = [orc.e3m3_encode(np.float32(t)) for t in np.geomspace(1e-6, 1e6, 400)]
+    assert max(codes) == (1 << bits["e3m3"]) - 1 and min(codes) >= 0
+    assert all(orc.e4m3_encode(np.float32(t)) < (1 << (bits["e4m3"] - 1)) for t in np.geomspace(1e-6, 1e6, 400))
+    rng = np.random.default_rng(31)
+    x = orc.f32_to_bf16((rng.standard_normal((64, 256)) * 0.02).astype(np.float32))
+    _, scales, _, _ = orc.quantize(x, "nvfp4_razer_w", want_sse=False)
+    sel = scales >> bits["e3m3"]
+    assert sel.max() < (1 << free) and len(np.unique(sel)) == 1 << free
+
+
+def test_mxfp4_block_length_follows_the_paper(orc):
+    """One shared exponent per 32 elements (tests/golden/block_sizes.txt): a row of two blocks
+    whose magnitudes differ by 2^10 gets two scale bytes 10 apart, and every element of a block
+    decodes with its own block's exponent."""
+    B = {r[0]: int(r[1]) for r in bf.read_golden("block_sizes.txt")}["mxfp4"]
+    assert orc.block_size("mxfp4") == B == 32
+    v = np.concatenate([np.full(B, 1.0), np.full(B, 1024.0)]).astype(np.float32)[None, :]
+    x = orc.f32_to_bf16(v)
+    codes, scales, _, sse = orc.quantize(x, "mxfp4", False)
+    assert scales.shape == (1, 2) and int(scales[0, 1]) - int(scales[0, 0]) == 10 and sse == 0.0
+    _, y16 = orc.dequantize(codes, scales, 0.0, "mxfp4", False)
+    assert np.array_equal(y16, x)
+
+
 def test_weight_mode_tensor_scale_maps_amax_to_6x30(orc):
     for k in range(-20, 20):
         assert orc.tensor_scale_from_amax(180.0 * 2.0 ** k, "nvfp4_razer_w") == np.float32(2.0 ** k)
