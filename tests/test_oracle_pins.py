@@ -752,6 +752,28 @@ def test_f32_to_f16_saturating_matches_numpy(orc):
         assert orc.f16_value(got) == float(ref)
 
 
+def test_outlier_rule_follows_the_paper(orc):
+    """The defaults and storage of the separation are the page's (tests/golden/outlier_rule.txt):
+    k = 4, at most 2 % of a row, fp16 values, the row mean in the bulk."""
+    rule = {r[0]: r[1] for r in bf.read_golden("outlier_rule.txt")}
+    k, frac = float(rule["k"]), float(rule["max_frac"])
+    assert rule["value_format"] == "fp16" and rule["bulk_fill"] == "group_mean"
+    for cols in (8, 49, 50, 100, 1024, 4096, 14336):
+        assert orc.outlier_capacity(cols) == orc.outlier_capacity(cols, frac) == int(np.floor(frac * cols + 1e-9))
+    # one row: 250 zeros and a 0.5 spike; mean 0.5/251 and sigma about 0.0315, so the spike
+    # is past 4 sigma and is the only outlier; its value comes back as the fp16 bits of 0.5
+    row = np.zeros((1, 256), np.float32)
+    row[0, 100] = 0.5
+    x = orc.f32_to_bf16(row)
+    bulk, oc, ov, cnt, mu, thr = orc.separate_outliers(x)
+    mean = 0.5 / 256
+    sigma = np.sqrt(((row[0].astype(np.float64) - mean) ** 2).mean())
+    assert cnt[0] == 1 and oc[0, 0] == 100 and abs(mu[0] - mean) < 1e-15
+    assert abs(thr[0] - k * sigma) <= 1e-12 * k * sigma
+    assert ov[0, 0] == np.float16(0.5).view(np.uint16)
+    assert bulk[0, 100] == orc.f64_to_bf16(mean) and (np.delete(bulk[0], 100) == 0).all()
+
+
 def test_outliers_closed_form_rows(orc):
     """Rows of n - m zeros and m spikes of height h: mu = m h / n, sigma = h sqrt(m (n - m)) / n,
     and the spikes are outliers exactly when (n - m) / sqrt(m (n - m)) > k."""
