@@ -11,7 +11,8 @@ L2 (--no-flush keeps them).  Prints one JSON line: median and minimum time
 per call, elements/s and the call's algorithmic bytes per second
 (quantize: 2 B read + codes and scales written, plus 2 B for the absmax read
 when the tensor scale is computed; dequantize: codes and scales read + 2 B
-written; error: 2 B + codes and scales read).
+written; error: 2 B + codes and scales read; tensor_scale: 2 B read, the absmax
+pass alone).
 
 --op gemm times fp4q_gemm on the operand forms of a seeded activation-like A
 (M x K, --a-fmt) and LLM-weight W (N x K, --w-fmt) and reports TFLOP/s: useful
@@ -33,7 +34,8 @@ from . import fp4q, synthetic
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["quantize", "dequantize", "error", "gemm", "outliers"], default="quantize")
+    p.add_argument("--op", choices=["quantize", "dequantize", "error", "tensor_scale", "gemm", "outliers"],
+                   default="quantize")
     p.add_argument("--fmt", choices=list(fp4q.FORMATS), default="nvfp4_razer")
     p.add_argument("--rows", type=int, default=14336)
     p.add_argument("--cols", type=int, default=4096)
@@ -76,6 +78,12 @@ def main(argv=None):
         def call():
             return fp4q.fp4q_quantize(x, a.rows, a.cols, a.cols, a.fmt, int(a.rotate), flags, q.codes, q.scales,
                                       q.tensor_scale, None if a.no_mse else mse, ws, ws.numel())
+    elif a.op == "tensor_scale":
+        nbytes = 2 * n   # the absmax pass reads x once
+        ts = torch.empty(1, dtype=torch.float32, device=dev)
+
+        def call():
+            return fp4q.fp4q_tensor_scale(x, a.rows, a.cols, a.cols, a.fmt, int(a.rotate), ts, ws, ws.numel())
     elif a.op == "dequantize":
         nbytes = packed + 2 * n
 
