@@ -450,14 +450,18 @@ struct ScatterArgs {
 };
 
 // One thread per (row, slot): the slot's fp16 value, as bf16, to its column.
+// A column at or past the row stride is skipped, so that arrays not made by
+// the separation can never write outside y's [rows][ldy] extent.
 __global__ void __launch_bounds__(256) outlier_scatter_kernel(ScatterArgs a)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= a.rows * a.cap) return;
     const int64_t r = i / a.cap, s = i - r * a.cap;
     if (s >= a.out_count[r]) return;
+    const int64_t col = a.out_cols[i];
+    if (col >= a.ldy) return;
     const float v = __half2float(__ushort_as_half(a.out_vals[i]));
-    a.y[r * a.ldy + a.out_cols[i]] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    a.y[r * a.ldy + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 }  // namespace

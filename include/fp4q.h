@@ -361,8 +361,10 @@ FP4Q_API fp4q_status_t fp4q_separate_outliers(const void* x, int64_t rows, int64
                                               double max_frac, void* bulk, int64_t ldb, uint16_t* out_cols,
                                               uint16_t* out_vals, int32_t* out_count, fp4q_stream_t stream);
 
-/* y[r][out_cols[r][s]] = bf16(out_vals[r][s]) for s < out_count[r]: puts the
- * outliers back into a bf16 reconstruction y [rows][ldy]. */
+/* y[r][out_cols[r][s]] = bf16(out_vals[r][s]) for s < min(out_count[r], cap):
+ * puts the outliers back into a bf16 reconstruction y [rows][ldy].  The arrays
+ * are those fp4q_separate_outliers wrote (columns below cols); a column at or
+ * past ldy is skipped, so no write leaves y's [rows][ldy] extent. */
 FP4Q_API fp4q_status_t fp4q_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals,
                                              const int32_t* out_count, int64_t rows, int64_t cols, int64_t cap,
                                              void* y, int64_t ldy, fp4q_stream_t stream);
