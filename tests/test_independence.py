@@ -61,3 +61,14 @@ def test_nothing_committed_uses_the_working_folder():
         if rel.startswith("_work/") or rel.endswith(".md") or rel in (".gitignore", "tests/test_independence.py"):
             continue
         assert "_work/" not in _read(rel), rel
+
+
+def test_profile_summaries_name_committed_commands_only():
+    """Each ncu summary under profiles/ gives the command that made it, and that command runs
+    committed files (bench.py or the package's kernel_bench), never a working-folder script."""
+    for rel in _tracked("profiles"):
+        if not rel.endswith(".md"):
+            continue
+        text = _read(rel)
+        assert "_work" not in text, rel
+        assert "ncu " in text and ("python bench.py" in text or "activation_quantization_block_b200.kernel_bench" in text), rel
