@@ -230,6 +230,8 @@ def quantize(x: np.ndarray, fmt, rotate: bool = False, tensor_scale: float | Non
     rc = lib().orc_quantize(_ptr(x), rows, cols, x.strides[0] // 2, f, int(rotate),
                             int(tensor_scale is not None), _ptr(ts), _ptr(codes), _ptr(scales),
                             _ptr(sse) if want_sse else None, nthreads or default_threads())
+    if rc == -2:
+        raise FloatingPointError("oracle: an element reached the E2M1 encoder as NaN (non-finite input)")
     if rc != 0:
         raise ValueError(f"oracle rejected shape {x.shape} for format {fmt} rotate={rotate}")
     return codes, scales, np.float32(ts[0]), (float(sse[0]) if want_sse else None)

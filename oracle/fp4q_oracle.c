@@ -26,7 +26,10 @@
  *  R2 NVFP4 is two-level: a per-tensor fp32 scale s_t = RN(A / (6*448)) with A
  *     the tensor absmax, then per 16-block an E4M3 scale (round to nearest
  *     even, saturating at 448).  Elements are encoded as RN(y * r) with
- *     r = RN(1 / RN(dec(sb) * s_t)).
+ *     r = RN(1 / RN(dec(sb) * s_t)); where that reciprocal overflows to
+ *     infinity (den below about 2^-128, which only a tensor whose absmax is
+ *     below about 2^-107 can reach) they are encoded as RN(y / den) instead,
+ *     so every element still goes to its nearest code and a zero stays +0.
  *  R3 MXFP4 scale: e = floor(log2(block absmax)) - 2, clamped to [-127, 127],
  *     stored as the E8M0 byte e + 127.
  *  R4 RaZeR (activation mode): the pair {+5, -5}; the scale sign bit selects
@@ -145,6 +148,7 @@ int orc_e2m1_encode(float v)
 {
     double a = fabs((double)v);
     int m;
+    if (isnan(v)) return -1;           /* no E2M1 code is nearest to NaN */
     if (a <= 0.25) m = 0;
     else if (a < 0.75) m = 1;
     else if (a <= 1.25) m = 2;
@@ -464,10 +468,12 @@ static int razer_select(const float* v, int* q, int n, const double* sv, int ns)
 }
 
 /* Quantize the row y[0..cols) (already rotated when asked).  Writes codes and
- * scales for the row and returns nothing; s_t is used for NVFP4 formats. */
-static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
-                         uint8_t* row_codes, uint8_t* row_scales)
+ * scales for the row; s_t is used for NVFP4 formats.  Returns 0, or -1 when an
+ * element reached the E2M1 encoder as NaN (outside the finite-input contract). */
+static int quantize_row(const float* y, int64_t cols, int fmt, float s_t,
+                        uint8_t* row_codes, uint8_t* row_scales)
 {
+    int bad = 0;
     const int B = block_size(fmt);
     for (int64_t b0 = 0; b0 < cols; b0 += B) {
         float a = 0.0f;
@@ -498,8 +504,12 @@ static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
                 /* a zero (or underflowed) scale decodes every element to 0 */
                 for (int i = 0; i < B; ++i) q[i] = 0;
             } else {
+                /* R2: scale by the reciprocal; by division where it overflows */
                 float r = 1.0f / den;
-                for (int i = 0; i < B; ++i) { v[i] = y[b0 + i] * r; q[i] = orc_e2m1_encode(v[i]); }
+                for (int i = 0; i < B; ++i) {
+                    v[i] = isinf(r) ? y[b0 + i] / den : y[b0 + i] * r;
+                    q[i] = orc_e2m1_encode(v[i]);
+                }
                 if (fmt == ORC_NVFP4_RAZER) {
                     const double pair[2] = {5.0, -5.0};
                     sbyte |= razer_select(v, q, B, pair, 2) << 7;
@@ -509,9 +519,12 @@ static void quantize_row(const float* y, int64_t cols, int fmt, float s_t,
                 }
             }
         }
+        for (int i = 0; i < B; ++i)
+            if (q[i] < 0) { bad = 1; q[i] = 0; }
         row_scales[b0 / B] = (uint8_t)sbyte;
         for (int i = 0; i < B; ++i) set_code(row_codes, b0 + i, q[i]);
     }
+    return bad ? -1 : 0;
 }
 
 /* Reconstruct the row in the original domain (inverse rotation when asked). */
@@ -554,6 +567,7 @@ typedef struct {
     const uint16_t* x; int64_t r0, r1, cols, ldx; int fmt, rotate; float s_t;
     uint8_t* codes; uint8_t* scales; const uint8_t* ccodes; const uint8_t* cscales;
     float* y_f32; uint16_t* y_bf16; int64_t ldy; int want_sse; double sse;
+    int bad;   /* set when an element reached the E2M1 encoder as NaN */
 } row_job;
 
 static void* quant_worker(void* p)
@@ -567,7 +581,7 @@ static void* quant_worker(void* p)
         uint8_t* rc = j->codes + r * (j->cols / 2);
         uint8_t* rs = j->scales + r * (j->cols / B);
         load_row(j->x + r * j->ldx, j->cols, j->rotate, y);
-        quantize_row(y, j->cols, j->fmt, j->s_t, rc, rs);
+        if (quantize_row(y, j->cols, j->fmt, j->s_t, rc, rs) != 0) j->bad = 1;
         if (j->want_sse) {
             dequant_row(rc, rs, j->cols, j->fmt, j->rotate, j->s_t, xh);
             sse += row_sse(j->x + r * j->ldx, xh, j->cols);
@@ -578,7 +592,7 @@ static void* quant_worker(void* p)
     return NULL;
 }
 
-static double run_rows(void* (*fn)(void*), row_job proto, int64_t rows, int nthreads)
+static double run_rows(void* (*fn)(void*), row_job proto, int64_t rows, int nthreads, int* bad)
 {
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = (int)rows;
@@ -591,7 +605,11 @@ static double run_rows(void* (*fn)(void*), row_job proto, int64_t rows, int nthr
         pthread_create(&th[t], NULL, fn, &jobs[t]);
     }
     double sse = 0.0;
-    for (int t = 0; t < nthreads; ++t) { pthread_join(th[t], NULL); sse += jobs[t].sse; }
+    for (int t = 0; t < nthreads; ++t) {
+        pthread_join(th[t], NULL);
+        sse += jobs[t].sse;
+        if (bad && jobs[t].bad) *bad = 1;
+    }
     free(jobs); free(th);
     return sse;
 }
@@ -599,8 +617,9 @@ static double run_rows(void* (*fn)(void*), row_job proto, int64_t rows, int nthr
 /* Quantize a rows x cols bf16 matrix (row stride ldx elements).
  *  scale_given != 0: *tensor_scale is read (NVFP4 formats), else computed
  *  and written.  sse (nullable) receives the sum of squared errors against
- *  the fp32 reconstruction in the original domain.  Returns 0, or -1 on a
- *  shape the formats do not allow. */
+ *  the fp32 reconstruction in the original domain.  Returns 0, -1 on a
+ *  shape the formats do not allow, or -2 when an element reached the E2M1
+ *  encoder as NaN (non-finite input, outside the contract). */
 int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
                  int fmt, int rotate, int scale_given, float* tensor_scale,
                  uint8_t* codes, uint8_t* scales, double* sse, int nthreads)
@@ -619,9 +638,10 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx,
     row_job proto = {0};
     proto.x = x; proto.cols = cols; proto.ldx = ldx; proto.fmt = fmt; proto.rotate = rotate;
     proto.s_t = s_t; proto.codes = codes; proto.scales = scales; proto.want_sse = sse != NULL;
-    double s = run_rows(quant_worker, proto, rows, nthreads);
+    int bad = 0;
+    double s = run_rows(quant_worker, proto, rows, nthreads, &bad);
     if (sse) *sse = s;
-    return 0;
+    return bad ? -2 : 0;
 }
 
 static void* dequant_worker(void* p)
@@ -655,7 +675,7 @@ int orc_dequantize(const uint8_t* codes, const uint8_t* scales, float tensor_sca
     proto.cols = cols; proto.fmt = fmt; proto.rotate = rotate; proto.s_t = tensor_scale;
     proto.ccodes = codes; proto.cscales = scales; proto.y_f32 = y_f32; proto.y_bf16 = y_bf16;
     proto.ldy = ldy;
-    run_rows(dequant_worker, proto, rows, nthreads);
+    run_rows(dequant_worker, proto, rows, nthreads, NULL);
     return 0;
 }
 
@@ -686,7 +706,7 @@ int orc_error(const uint16_t* x, int64_t ldx, const uint8_t* codes, const uint8_
     row_job proto = {0};
     proto.x = x; proto.ldx = ldx; proto.cols = cols; proto.fmt = fmt; proto.rotate = rotate;
     proto.s_t = tensor_scale; proto.ccodes = codes; proto.cscales = scales;
-    *sse = run_rows(error_worker, proto, rows, nthreads);
+    *sse = run_rows(error_worker, proto, rows, nthreads, NULL);
     return 0;
 }
 

@@ -139,6 +139,29 @@ def rn_f32(fr: Fraction) -> np.float32:
     return np.float32(float(fr))
 
 
+def rn_f32_exact(fr: Fraction) -> np.float32:
+    """Round an exact rational to binary32, nearest even, subnormals included,
+    by integer arithmetic on its significand (no intermediate rounding)."""
+    if fr == 0:
+        return np.float32(0.0)
+    neg = fr < 0
+    a = -fr if neg else fr
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    if Fraction(2) ** e > a:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= a:
+        e += 1
+    qexp = max(e, -126) - 23                                       # the binary32 quantum at a
+    scaled = a / Fraction(2) ** qexp
+    n = scaled.numerator // scaled.denominator
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    val = Fraction(n) * Fraction(2) ** qexp
+    out = np.float32(np.inf) if val >= Fraction(2) ** 128 else np.float32(float(val))
+    return -out if neg else out
+
+
 def sylvester_hadamard(n: int = 32) -> np.ndarray:
     h = np.array([[1]], dtype=np.int64)
     while h.shape[0] < n:
@@ -203,8 +226,12 @@ def quantize_bruteforce(xbits: np.ndarray, fmt: str, rotate: bool, pair2: float 
                 scales[r, b] = sb
                 if sb == 0 or den == 0:
                     continue
-                rr = np.float32(np.float32(1) / den)
-                v = [np.float32(val * rr) for val in blk]
+                with np.errstate(over="ignore"):
+                    rr = np.float32(np.float32(1) / den)
+                if np.isinf(rr):   # the reciprocal overflows: scale by exact division, rounded once
+                    v = [rn_f32_exact(Fraction(float(val)) / Fraction(float(den))) for val in blk]
+                else:
+                    v = [np.float32(val * rr) for val in blk]
             q = [e2m1_nearest(float(vi)) for vi in v]
             if fmt == "nvfp4_razer":
                 idx, q = razer_pick(v, q, (5.0, -5.0))

@@ -279,6 +279,74 @@ def test_quantize_equals_bruteforce(orc, fmt, rotate):
         assert abs(sse - float(exact)) <= 1e-12 * max(1.0, float(exact))
 
 
+def _tiny_magnitude_inputs():
+    """bf16 tensors whose absmax lies between 2^-133 (the smallest bf16
+    subnormal) and 6 * 2^-128, zeros included.  Their block scales
+    den = RN(dec(sb) * s_t) fall below 2^-128, where RN(1 / den) overflows."""
+    rng = np.random.default_rng(23)
+    out = []
+    k = rng.integers(-127, 128, size=(4, 32)).astype(np.float64)   # subnormal multiples of 2^-133
+    k[rng.random(k.shape) < 0.25] = 0.0
+    out.append(k * 2.0 ** -133)
+    top = rng.uniform(-1.5, 1.5, size=(2, 64)) * 2.0 ** -126          # up to 6 * 2^-128
+    top[0, :5] = 0.0
+    top[1, 7] = 1.5 * 2.0 ** -126
+    out.append(top)
+    one = np.zeros((1, 32)); one[0, 3] = 2.0 ** -133; one[0, 20] = -2.0 ** -133
+    out.append(one)
+    return [a.astype(np.float32).astype(ml_dtypes.bfloat16).view(np.uint16) for a in out]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "nvfp4_razer_w"])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_overflowing_block_reciprocal_equals_bruteforce(orc, fmt, rotate):
+    """Where RN(1 / den) is infinite the elements are scaled by exact division
+    (rounded once), so each goes to its nearest code and zeros stay +0."""
+    for xb in _tiny_magnitude_inputs():
+        codes, scales, ts, sse = orc.quantize(xb, fmt, rotate)
+        assert 0 < ts < 2.0 ** -120
+        bcodes, bscales, bts = bf.quantize_bruteforce(xb, fmt, rotate, pair2=orc.razer_w_pair())
+        assert np.array_equal(codes, bcodes)
+        assert np.array_equal(scales, bscales)
+        assert ts == bts
+        nib = bf.unpack_codes(codes, xb.shape[1])
+        if not rotate:
+            assert np.all(nib[xb == 0] == 0)                 # zeros stay +0
+            nz = bf.bits_to_f32(xb) != 0
+            if nz.sum() > 8:                                  # not everything saturated to +-6
+                assert not np.all(np.isin(nib[nz], (7, 15)))
+        xhat = bf.dequantize_bruteforce(bcodes, bscales, bts, fmt, rotate, pair2=orc.razer_w_pair())
+        exact = bf.sse_exact(xb, xhat)
+        assert abs(sse - float(exact)) <= 1e-12 * max(float(exact), 2.0 ** -300)
+
+
+def test_overflowing_reciprocal_codes_are_nearest_to_the_exact_quotient(orc):
+    """Closed form, unrotated NVFP4: every code is the E2M1 value nearest to
+    RN(y / den), with den = RN(dec(sb) * s_t) from the scale byte the oracle wrote."""
+    for xb in _tiny_magnitude_inputs():
+        codes, scales, ts, _ = orc.quantize(xb, "nvfp4")
+        x = bf.bits_to_f32(xb)
+        nib = bf.unpack_codes(codes, xb.shape[1])
+        for r in range(x.shape[0]):
+            for j in range(x.shape[1]):
+                den = np.float32(np.float32(bf.E4M3_POS[int(scales[r, j // 16])]) * ts)
+                if den == 0:
+                    assert nib[r, j] == 0
+                    continue
+                assert np.isinf(np.float32(1.0) / den) or den >= 2.0 ** -128
+                v = bf.rn_f32_exact(Fraction(float(x[r, j])) / Fraction(float(den)))
+                assert nib[r, j] == bf.e2m1_nearest(float(v))
+
+
+def test_e2m1_encoder_refuses_nan(orc):
+    assert orc.e2m1_encode(float("nan")) == -1
+    xb = np.zeros((1, 16), np.float32)
+    xb[0, 3] = 1.0
+    xb[0, 5] = np.nan
+    with pytest.raises(FloatingPointError):
+        orc.quantize(xb.astype(ml_dtypes.bfloat16).view(np.uint16), "nvfp4")
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "nvfp4_razer", "mxfp4", "nvfp4_razer_w", "mxfp4_ceil"])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_dequantize_equals_bruteforce(orc, fmt, rotate):
