@@ -304,8 +304,8 @@ fp4q_status_t fp4q_scatter_outliers(const uint16_t* out_cols, const uint16_t* ou
         return FP4Q_ERROR_MISALIGNED;
     fp4q_status_t s = check_device();
     if (s != FP4Q_SUCCESS) return s;
-    return from_cuda(launch_scatter_outliers(out_cols, out_vals, out_count, rows, cap, static_cast<uint16_t*>(y),
-                                             ldy, reinterpret_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_scatter_outliers(out_cols, out_vals, out_count, rows, cols, cap,
+                                             static_cast<uint16_t*>(y), ldy, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int fp4q_mma_planes(fp4q_format_t fmt)

@@ -57,7 +57,7 @@ struct ChainArgs {
 };
 
 template <int FMT, bool ROT, bool SSE>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     chain_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap amap, ChainArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -229,15 +229,23 @@ struct View {
 size_t batch_workspace_bytes() { return (size_t)kRing * kMaxPartials * (sizeof(float) + sizeof(double)); }
 
 cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, int mx_ceil,
-                                  void* workspace, cudaStream_t st)
+                                  void* workspace, cudaStream_t st, bool single_layout)
 {
     if (n <= 0) return cudaSuccess;
     const bool computed = fmt != kMX && !scale_given;
     bool sse = false;
     for (int k = 0; k < n; ++k) sse = sse || ts[k].mse != nullptr;
     char* ws = static_cast<char*>(workspace);
-    auto amax_slot = [&](int64_t j) { return reinterpret_cast<float*>(ws + (j % kRing) * kMaxPartials * 4); };
+    // One tensor needs one slot of each kind (launch 0 writes the absmax
+    // partials that launch 1 reads; the launch that quantizes writes the error
+    // partials the next one reads), so it fits the single-call workspace.
+    single_layout = single_layout && n == 1;
+    auto amax_slot = [&](int64_t j) {
+        if (single_layout) return reinterpret_cast<float*>(ws + kWsAmaxOffset);
+        return reinterpret_cast<float*>(ws + (j % kRing) * kMaxPartials * 4);
+    };
     auto sse_slot = [&](int64_t j) {
+        if (single_layout) return reinterpret_cast<double*>(ws + kWsSseOffset);
         return reinterpret_cast<double*>(ws + (size_t)kRing * kMaxPartials * 4 + (j % kRing) * kMaxPartials * 8);
     };
     std::vector<View> views((size_t)n);

@@ -464,48 +464,6 @@ __device__ __forceinline__ void razer_from_v(const float* v, uint32_t& w0, uint3
     else razer_tent(v, w0, w1, sb);
 }
 
-// One 16-element NVFP4 / RaZeR block of values y (rotated ones, on the rotated
-// path) with absmax a: two code words and the scale byte and, when XH, the
-// fp32 reconstruction xh = RN(q den) (RaZeR winners: RN(special * den)).
-template <int FMT, bool XH>
-__device__ __forceinline__ void encode_nv16(const float* y, float a, const NvScale& sc, uint32_t& c0, uint32_t& c1,
-                                            uint32_t& sb_out, float* xh)
-{
-    constexpr bool RAZER = kRazer<FMT>;
-    uint32_t sb = nv_scale_code<FMT>(sc, a);
-    const float2 dr = nv_den_rcp(sc, sb);
-    const float den = dr.x, r = dr.y;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
-        v[i] = p.x;
-        v[i + 1] = p.y;
-    }
-    uint32_t w0 = canonical_zero(e2m1x8(v));
-    uint32_t w1 = canonical_zero(e2m1x8(v + 8));
-    if (RAZER) razer_from_v<FMT>(v, w0, w1, sb);
-    if (XH) {
-        float q[16];
-        decode16(w0, w1, q);
-        const float special = razer_special<FMT>(sb);
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            float q0 = q[i], q1 = q[i + 1];
-            if (RAZER) {
-                if ((((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu) == 8u) q0 = special;
-                if ((((i < 8 ? w0 : w1) >> (4 * ((i + 1) & 7))) & 0xFu) == 8u) q1 = special;
-            }
-            const float2 p = mul2_rn(make_float2(q0, q1), make_float2(den, den));
-            xh[i] = p.x;
-            xh[i + 1] = p.y;
-        }
-    }
-    c0 = w0;
-    c1 = w1;
-    sb_out = sb;
-}
-
 // ---------------------------------------------------------------------------
 // Unrotated NVFP4 / RaZeR blocks straight from the bf16 tile
 // ---------------------------------------------------------------------------
@@ -519,8 +477,9 @@ struct BlockOut {
 // at a0 and a1), given its unsigned scale byte and {den, rcp}: codes, scale
 // byte and the squared error in the original domain, each difference
 // y - RN(q den) taken in fp32 (zero when the element is reproduced) and
-// squared and summed in fp64.  Taken for the rare blocks the fast path below
-// does not cover.
+// squared and summed in fp64.  Elements are scaled by r = RN(1 / den), or
+// divided by den where r overflowed to infinity.  Taken for the rare blocks the
+// fast path below does not cover.
 template <int FMT>
 __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32_t sb, float den, float r)
 {
@@ -531,11 +490,16 @@ __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32
     w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
     float y[16], v[16];
     unpack16(w, y);
+    if (isinf(r)) {   // RN(1 / den) overflowed (den below about 2^-128): scale by division
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(y[i], den);
+    } else {
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
-        v[i] = p.x;
-        v[i + 1] = p.y;
+        for (int i = 0; i < 16; i += 2) {
+            const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+            v[i] = p.x;
+            v[i + 1] = p.y;
+        }
     }
     BlockOut o;
     o.w0 = canonical_zero(e2m1x8(v));
@@ -576,7 +540,11 @@ __device__ __noinline__ BlockOut nv_block_exact(uint32_t a0, uint32_t a1, uint32
 // nv_block_exact: max |v| > 6.5 (a saturated scale byte, or a subnormal one
 // far below the block absmax), a fast sum below 2^-30 (the block is reproduced
 // exactly or almost, and the exact sum keeps a zero error zero), or one that
-// is not finite (an infinite reciprocal).
+// is not finite (an infinite reciprocal: den below about 2^-128, where the
+// exact path divides).  A subnormal den with a finite reciprocal (den in
+// [2^-128, 2^-126), only in tensors whose absmax is below about 2^-105) stays
+// on the fast path: RN(q den) may round there by half a subnormal quantum,
+// which moves the block's error by about 2^-20 of itself.
 template <int FMT, bool SSE>
 __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_t a1, const NvScale& sc,
                                          uint32_t& c0, uint32_t& c1, uint32_t& sb_out, double& sse)
@@ -599,6 +567,13 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
         }
     }
     if (!SSE) {
+        if (isinf(dr.y)) {   // RN(1 / den) overflowed: the exact path divides
+            const BlockOut o = nv_block_exact<FMT>(a0, a1, sb, dr.x, dr.y);
+            c0 = o.w0;
+            c1 = o.w1;
+            sb_out = o.sb;
+            return;
+        }
         uint32_t w0 = canonical_zero(e2m1x8(v)), w1 = canonical_zero(e2m1x8(v + 8));
         if (RAZER) razer_from_v<FMT>(v, w0, w1, sb);
         c0 = w0;
@@ -686,14 +661,247 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
     }
 }
 
-// One 32-element MXFP4 block.  The exponent is floor(log2 a) - 2 (values in
-// [6, 8) 2^e saturate to 6) or, with ceil, the smallest e with a <= 6 * 2^e:
-// one more when a's significand exceeds 1.5 ("TORQ: Two-Level Orthogonal
-// Rotation for MXFP4 Quantization", sect. 2, S-step: the block maximum onto
-// the largest code), at most 125 so that 6 * 2^e stays finite in fp32.
-template <bool XH>
-__device__ __forceinline__ void encode_mx32(const float* y, float a, bool ceil, uint32_t* cw, uint32_t& sb_out,
-                                            float* xh)
+// ---------------------------------------------------------------------------
+// NVFP4 / RaZeR blocks, eight elements at a time
+// ---------------------------------------------------------------------------
+//
+// A block's elements are encoded in two runs of eight, each adding to running
+// sums, so that no per-element array outlives its run:
+//  - the codes (cvt.rn.satfinite.e2m1x2: nearest even, saturating);
+//  - with SSE, e = q - v for the regular grid value q of each scaled value v
+//    (exact, see e2m1x8_diff) and the sum of e^2;
+//  - RaZeR: for each element its gain of moving to sign(v) * 5 -- for |v| in
+//    (4.5, 5.5) the regular value is 4 or 6 and (|v| - q)^2 - (|v| - 5)^2 =
+//    1 - 2 ||v| - 5| = 2 |e| - 1, clamped at 0 elsewhere -- summed as U (all
+//    gains) and S (gains signed by v).  Every gain is a multiple of 2^-20 in
+//    [0, 1], so both sums are exact in fp32 whatever the order; gain(+5) =
+//    (U + S) / 2 and gain(-5) = (U - S) / 2.  A candidate marker per element,
+//    the E2M1 code of sign(v) * gain * 2^40, is +6 (0x7) for a candidate of
+//    +5, -6 (0xF) for one of -5 and +-0 otherwise;
+//  - the weight mode adds the pair 2.5 the same way (gain 1/4 - ||v| - 2.5|,
+//    multiples of 2^-22 up to 1/4; candidates of 2.5 and of 5 never overlap).
+// The 2|e| - 1 form of the gain of 5 holds while |v| <= 6.5; blocks beyond
+// that take the exact path (nv_block_exact_f32), which forms gains from v.
+
+struct NvRun {
+    uint32_t cw[2];          // code words, eight nibbles each
+    uint32_t k5[2], k2[2];   // candidate markers of 5 and (weight mode) of 2.5
+    float2 sq;               // sum of e^2, two lanes
+    float2 u5, s5, u2, s2;   // sums of the gains and of the signed gains, two lanes
+};
+
+// One run of eight scaled values v into run h (0 or 1) of the block.  GE: the
+// gains of 5 come from e (the fast path); otherwise from v.
+template <int FMT, bool SSE, bool GE>
+__device__ __forceinline__ void nv_run8(const float* v, int h, NvRun& st)
+{
+    constexpr bool RAZER = kRazer<FMT>;
+    float g[8];
+    if (SSE) {
+        float e[8];
+        st.cw[h] = e2m1x8_diff(v, e);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            st.sq = fma2_rn(make_float2(e[i], e[i + 1]), make_float2(e[i], e[i + 1]), st.sq);
+        if (RAZER && GE) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) g[i] = __saturatef(__fmaf_rn(2.0f, fabsf(e[i]), -1.0f));
+        }
+    } else {
+        st.cw[h] = e2m1x8(v);
+    }
+    if (RAZER && !(SSE && GE)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
+    }
+    if (RAZER) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const float2 gg = make_float2(g[i], g[i + 1]);
+            const float2 cs = make_float2(copysignf(g[i], v[i]), copysignf(g[i + 1], v[i + 1]));
+            st.u5 = add2_rn(st.u5, gg);
+            st.s5 = add2_rn(st.s5, cs);
+            const float2 m = mul2_rn(cs, make_float2(0x1p40f, 0x1p40f));
+            x[i] = m.x;
+            x[i + 1] = m.y;
+        }
+        st.k5[h] = e2m1x8(x);
+    }
+    if (FMT == kRW) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const float g0 = razer_gain_w2(v[i]), g1 = razer_gain_w2(v[i + 1]);
+            const float2 cs = make_float2(copysignf(g0, v[i]), copysignf(g1, v[i + 1]));
+            st.u2 = add2_rn(st.u2, make_float2(g0, g1));
+            st.s2 = add2_rn(st.s2, cs);
+            const float2 m = mul2_rn(cs, make_float2(0x1p40f, 0x1p40f));
+            x[i] = m.x;
+            x[i + 1] = m.y;
+        }
+        st.k2[h] = e2m1x8(x);
+    }
+}
+
+// Rewrite the winners flagged in k (nibbles 0xF after the sign flip below) to 0b1000.
+__device__ __forceinline__ uint32_t apply_winners(uint32_t w, uint32_t k)
+{
+    const uint32_t f = k & (k >> 3) & 0x11111111u;
+    return (w & ~(f * 15u)) | (f << 3);
+}
+
+// The block's RaZeR choice from its running sums: -5 only when its gain is
+// strictly larger than that of +5 (equal gains, or none, keep +5 with bit 7
+// clear); in the weight mode the pair 2.5 only when its better member gains
+// strictly more than the better of +-5, and in a pair the negative member
+// only when it gains strictly more (ties go to the lower selector; bits 6..7:
+// 0 +5, 1 -5, 2 +2.5, 3 -2.5).  Canonicalises -0 codes to +0, writes the
+// winners' codes as 0b1000 and the selector into sb, and returns the chosen
+// total gain (0 for NVFP4).
+template <int FMT>
+__device__ __forceinline__ float nv_finish(NvRun& st, uint32_t& sb)
+{
+    st.cw[0] = canonical_zero(st.cw[0]);
+    st.cw[1] = canonical_zero(st.cw[1]);
+    if (!kRazer<FMT>) return 0.0f;
+    const float U5 = st.u5.x + st.u5.y, S5 = st.s5.x + st.s5.y;
+    float G;
+    bool neg;
+    uint32_t k0 = st.k5[0], k1 = st.k5[1];
+    if (FMT == kRW) {
+        const float U2 = st.u2.x + st.u2.y, S2 = st.s2.x + st.s2.y;
+        const float t5 = U5 + fabsf(S5), t2 = U2 + fabsf(S2);
+        const bool p2 = t2 > t5;
+        neg = (p2 ? S2 : S5) < 0.0f;
+        if (p2) {
+            k0 = st.k2[0];
+            k1 = st.k2[1];
+        }
+        sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
+        G = 0.5f * fmaxf(t5, t2);
+    } else {
+        neg = S5 < 0.0f;
+        if (neg) sb |= 0x80u;
+        G = 0.5f * (U5 + fabsf(S5));
+    }
+    // markers of the chosen sign become 0xF: those of +5 (0x7) by flipping bit 3
+    const uint32_t flip = neg ? 0u : 0x88888888u;
+    st.cw[0] = apply_winners(st.cw[0], k0 ^ flip);
+    st.cw[1] = apply_winners(st.cw[1], k1 ^ flip);
+    return G;
+}
+
+// Exact squared error of eight values y against the reconstruction RN(q den)
+// of code word cw (RaZeR code 0b1000: the special value of scale byte sb),
+// each difference and its square summed in fp64, as the oracle does.
+template <int FMT>
+__device__ __forceinline__ double nv_sse8_exact(const float* y, uint32_t cw, uint32_t sb, float den)
+{
+    float q[8];
+    e2m1x8_to_f32(cw, q);
+    const float special = razer_special<FMT>(sb);
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float qi = (kRazer<FMT> && ((cw >> (4 * i)) & 0xFu) == 8u) ? special : q[i];
+        const double d = (double)y[i] - (double)__fmul_rn(qi, den);
+        s = fma(d, d, s);
+    }
+    return s;
+}
+
+// Scaled values of eight y: RN(y r), or RN(y / den) where r overflowed (DIV).
+template <bool DIV>
+__device__ __forceinline__ void nv_scale8(const float* y, float den, float r, float* v)
+{
+    if (DIV && isinf(r)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(y[i], den);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
+            v[i] = p.x;
+            v[i + 1] = p.y;
+        }
+    }
+}
+
+// One block of sixteen fp32 values y (rotated ones on the rotated path) with
+// absmax a, encoded from scratch in the exact way: gains from v, the error in
+// fp64 from the reconstruction, and division wherever RN(1 / den) overflowed
+// (DIV).  For the rare blocks the fast path does not cover (nv_block_redo).
+template <int FMT, bool SSE, bool DIV>
+__device__ __forceinline__ void nv_block_exact_f32(const float* y, uint32_t sb, float den, float r, uint32_t& c0,
+                                               uint32_t& c1, uint32_t& sb_out, double& sse)
+{
+    NvRun st = {};
+    float v[8];
+    nv_scale8<DIV>(y, den, r, v);
+    nv_run8<FMT, false, false>(v, 0, st);
+    nv_scale8<DIV>(y + 8, den, r, v);
+    nv_run8<FMT, false, false>(v, 1, st);
+    nv_finish<FMT>(st, sb);
+    c0 = st.cw[0];
+    c1 = st.cw[1];
+    sb_out = sb;
+    if (SSE) sse = nv_sse8_exact<FMT>(y, c0, sb, den) + nv_sse8_exact<FMT>(y + 8, c1, sb, den);
+}
+
+// The error of a block from its running sums, den^2 (sum e^2 - G), valid when
+// it is not too small (a block reproduced exactly or almost keeps the exact
+// sum, so that an exact reconstruction has error 0) and finite, and when
+// max |v| <= 6.5 for RaZeR (the 2|e| - 1 form of the gains).  den v differs
+// from y by at most 2^-23 |y| (two roundings), the only departure from the
+// exact error besides the fp32 rounding of the sums.
+template <int FMT>
+__device__ __forceinline__ bool nv_fast_error(const NvRun& st, float G, float a, float r, float& sv)
+{
+    sv = (st.sq.x + st.sq.y) - G;
+    return sv >= 0x1p-30f && sv <= 0x1p64f && (!kRazer<FMT> || __fmul_rn(a, r) <= 6.5f);
+}
+
+// One block of sixteen fp32 values y with absmax a (the rotated path): codes,
+// scale byte and, when SSE, the error in y's domain from the running sums.
+// Returns false (outputs unset) when the fast path does not hold -- an
+// overflowed reciprocal, or a fast error that does not hold -- and the caller
+// redoes the block (nv_block_redo).
+template <int FMT, bool SSE>
+__device__ __forceinline__ bool nv_block_f32(const float* y, float a, const NvScale& sc, uint32_t& c0,
+                                             uint32_t& c1, uint32_t& sb_out, double& sse)
+{
+    uint32_t sb = nv_scale_code<FMT>(sc, a);
+    const float2 dr = nv_den_rcp(sc, sb);
+    if (isinf(dr.y)) return false;
+    const uint32_t sb0 = sb;
+    NvRun st = {};
+    float v[8];
+    nv_scale8<false>(y, dr.x, dr.y, v);
+    nv_run8<FMT, SSE, true>(v, 0, st);
+    nv_scale8<false>(y + 8, dr.x, dr.y, v);
+    nv_run8<FMT, SSE, true>(v, 1, st);
+    const float G = nv_finish<FMT>(st, sb);
+    float sv = 0.0f;
+    if (SSE && !nv_fast_error<FMT>(st, G, a, dr.y, sv)) return false;
+    c0 = st.cw[0];
+    c1 = st.cw[1];
+    sb_out = sb;
+    if (SSE) sse = (double)sv * nv_den2(sc, sb0);
+    return true;
+}
+
+// One 32-element MXFP4 block of fp32 values y with absmax a.  The exponent is
+// floor(log2 a) - 2 (values in [6, 8) 2^e saturate to 6) or, with ceil, the
+// smallest e with a <= 6 * 2^e: one more when a's significand exceeds 1.5
+// ("TORQ: Two-Level Orthogonal Rotation for MXFP4 Quantization", sect. 2,
+// S-step: the block maximum onto the largest code), at most 125 so that
+// 6 * 2^e stays finite in fp32.  v = y 2^-e is exact, so e = q - v is exact
+// and the error (q - v)^2 2^2e is formed in the scaled domain; the fp32 sum
+// of e^2 is the only rounding.
+template <bool SSE>
+__device__ __forceinline__ void mx_block(const float* y, float a, bool ceil, uint32_t* cw, uint32_t& sb_out,
+                                         double& sse)
 {
     int e = -127;
     float r = 0.0f;
@@ -705,27 +913,27 @@ __device__ __forceinline__ void encode_mx32(const float* y, float a, bool ceil, 
         sb = (uint32_t)(e + 127);
         r = exp2i(-e);
     }
-    float v[32];
+    float2 sq = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        const float2 p = mul2_rn(make_float2(y[i], y[i + 1]), make_float2(r, r));
-        v[i] = p.x;
-        v[i + 1] = p.y;
-    }
+    for (int k = 0; k < 4; ++k) {
+        float v[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) cw[k] = canonical_zero(e2m1x8(v + 8 * k));
-    if (XH) {
-        const float s = exp2i(e);
-        float q[32];
-        decode16(cw[0], cw[1], q);
-        decode16(cw[2], cw[3], q + 16);
+        for (int i = 0; i < 8; i += 2) {
+            const float2 p = mul2_rn(make_float2(y[8 * k + i], y[8 * k + i + 1]), make_float2(r, r));
+            v[i] = p.x;
+            v[i + 1] = p.y;
+        }
+        if (SSE) {
+            float d[8];
+            cw[k] = canonical_zero(e2m1x8_diff(v, d));
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-            const float2 p = mul2_rn(make_float2(q[i], q[i + 1]), make_float2(s, s));
-            xh[i] = p.x;
-            xh[i + 1] = p.y;
+            for (int i = 0; i < 8; i += 2)
+                sq = fma2_rn(make_float2(d[i], d[i + 1]), make_float2(d[i], d[i + 1]), sq);
+        } else {
+            cw[k] = canonical_zero(e2m1x8(v));
         }
     }
+    if (SSE) sse = a > 0.0f ? ldexp((double)(sq.x + sq.y), 2 * e) : 0.0;
     sb_out = sb;
 }
 
@@ -918,9 +1126,40 @@ __device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint3
 // Per-tile work (shared by the single-tensor kernels and the batch scheduler)
 // ---------------------------------------------------------------------------
 
+// Block `half` of the unit (r, h) encoded again in the exact way from the tile
+// (rotated again when ROT): codes, scale byte and the error in fp64, with
+// division wherever RN(1 / den) overflowed.  Out of line and by value, so that
+// the fast path keeps its registers; only blocks that path does not cover
+// come here.
+template <int FMT, bool ROT>
+__device__ __noinline__ BlockOut nv_block_redo(uint32_t tile, uint32_t r, uint32_t h, uint32_t half, NvScale nsc)
+{
+    float y[32];
+    {
+        uint32_t w[16];
+        load_unit_words(tile, r, h, w);
+        unpack16(w, y);
+        unpack16(w + 8, y + 16);
+    }
+    if (ROT) wht32_inplace(y);
+    const float* yb = half ? y + 16 : y;
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(yb[i]));
+    const uint32_t sb = nv_scale_code<FMT>(nsc, a);
+    const float2 dr = nv_den_rcp(nsc, sb);
+    BlockOut o;
+    nv_block_exact_f32<FMT, true, true>(yb, sb, dr.x, dr.y, o.w0, o.w1, o.sb, o.sse);
+    return o;
+}
+
 // Q1-Q6 on the unit this thread owns in tile k (shared address `tile`):
 // rotate, block scales, encode, RaZeR select, pack and store codes and scales.
-// Returns the unit's squared error when SSE.
+// Returns the unit's squared error when SSE: in the original domain without
+// rotation; with rotation in the rotated domain, which the orthonormal
+// transform H / sqrt(32) maps onto the original one up to the fp32 rounding of
+// the rotated values (about 2^-24 of each value, far inside the rotated
+// paths' 1e-3 MSE tolerance).
 template <int FMT, bool ROT, bool SSE, bool FLAT>
 __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, int64_t k, uint8_t* codes,
                                                 uint8_t* scales, const NvScale& nsc, bool mx_ceil = false)
@@ -951,7 +1190,8 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                 if (SSE) acc += e;
             }
         } else {
-            float y[32], xh[32];
+            // rotated NVFP4 / RaZeR, and MXFP4: the error in the scaled (and rotated) domain
+            float y[32];
             {
                 uint32_t w[16];
                 load_unit_words(tile, r, h, w);
@@ -963,25 +1203,30 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
                 float am = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(y[i]));
-                encode_mx32<SSE>(y, am, mx_ceil, cw, sb0, xh);
+                double e = 0.0;
+                mx_block<SSE>(y, am, mx_ceil, cw, sb0, e);
+                if (SSE) acc += e;
             } else {
-                float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    a0 = fmaxf(a0, fabsf(y[i]));
-                    a1 = fmaxf(a1, fabsf(y[16 + i]));
+                for (int half = 0; half < 2; ++half) {
+                    float am = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(y[16 * half + i]));
+                    uint32_t c0 = 0, c1 = 0, sbh = 0;
+                    double e = 0.0;
+                    if (!nv_block_f32<FMT, SSE>(y + 16 * half, am, nsc, c0, c1, sbh, e)) {
+                        const BlockOut o = nv_block_redo<FMT, ROT>(tile, r, h, (uint32_t)half, nsc);
+                        c0 = o.w0;
+                        c1 = o.w1;
+                        sbh = o.sb;
+                        e = o.sse;
+                    }
+                    cw[2 * half] = c0;
+                    cw[2 * half + 1] = c1;
+                    if (half == 0) sb0 = sbh;
+                    else sb1 = sbh;
+                    if (SSE) acc += e;
                 }
-                encode_nv16<FMT, SSE>(y, a0, nsc, cw[0], cw[1], sb0, xh);
-                encode_nv16<FMT, SSE>(y + 16, a1, nsc, cw[2], cw[3], sb1, xh + 16);
-            }
-            if (SSE) {
-                // the original values again, from the tile still in shared memory
-                if (ROT) wht32_inplace(xh);
-                uint32_t w[16];
-                load_unit_words(tile, r, h, w);
-                unpack16(w, y);
-                unpack16(w + 8, y + 16);
-                acc += sse_of<32>(y, xh);
             }
         }
         int64_t co, so;

@@ -9,6 +9,7 @@
 namespace fp4q {
 
 constexpr int kThreads = 256;        // threads per CTA for every streaming kernel
+constexpr int kTileCtasPerSm = 3;        // resident CTAs per SM the tile kernels are compiled for
 constexpr int kMaxPartials = 4096;   // upper bound on CTAs of one pass (per-CTA partial slots)
 
 // Workspace layout: fp64 partial sums, then fp32 partial maxima.
@@ -79,7 +80,7 @@ cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t co
                                      uint16_t* bulk, int64_t ldb, uint16_t* out_cols, uint16_t* out_vals,
                                      int32_t* out_count, cudaStream_t st);
 cudaError_t launch_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals, const int32_t* out_count,
-                                    int64_t rows, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st);
+                                    int64_t rows, int64_t cols, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st);
 
 // Tile count of a bf16 matrix's view (see make_view): 16 KB tiles.
 int64_t view_tiles(const Geometry& g);
@@ -99,8 +100,9 @@ size_t batch_workspace_bytes();
 
 // Quantize n non-empty tensors as a chain of persistent kernels, one per tensor
 // (absmax pass of tensor j interleaved with the quantize pass of tensor j-1).
+// single_layout (n == 1): the partials use the single-call workspace layout
+// (kWorkspaceBytes) instead of the batch's rotating slots.
 cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rotate, int scale_given, int mx_ceil,
-                                  void* workspace,
-                                  cudaStream_t st);
+                                  void* workspace, cudaStream_t st, bool single_layout = false);
 
 }  // namespace fp4q

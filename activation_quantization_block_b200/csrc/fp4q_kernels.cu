@@ -96,7 +96,7 @@ struct QuantArgs {
 
 // Q1-Q6: rotate, block scale, encode, RaZeR select, pack, store, SSE partials.
 template <int FMT, bool ROT, bool SSE, bool FLAT>
-__global__ void __launch_bounds__(kThreads, 3) quantize_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a)
+__global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
@@ -161,7 +161,7 @@ struct ErrArgs {
 
 // Q8: squared error of a given encoding against x.
 template <int FMT, bool ROT, bool FLAT>
-__global__ void __launch_bounds__(kThreads, 3) error_kernel(const __grid_constant__ CUtensorMap xmap, ErrArgs a)
+__global__ void __launch_bounds__(kThreads, kTileCtasPerSm) error_kernel(const __grid_constant__ CUtensorMap xmap, ErrArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ double shd[32];

@@ -10,9 +10,11 @@
 // cudaMalloc / cudaFree can imply.  This entry point serves them: its scratch
 // is a file-scope device array that the CUDA module loader places on every
 // GPU that loads this library, so the call itself allocates nothing.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
 #include <mutex>
 
 #include "fp4q.h"
@@ -28,31 +30,78 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[FP4Q_NOALLOC_SC
 static_assert(FP4Q_NOALLOC_SCRATCH_BYTES >= fp4q::kWorkspaceBytes,
               "the static scratch must hold the quantize workspace");
 
-constexpr int kMaxDevices = 64;
+// Driver calls that name the current CUDA context: its handle, and its ID,
+// which is unique for the life of the process (a handle can be reused after a
+// context is destroyed, an ID cannot).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct Driver {
+    CtxGetCurrentFn get_current = nullptr;
+    CtxGetIdFn get_id = nullptr;
+};
+
+const Driver& driver()
+{
+    static Driver d;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            d.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            d.get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    return d;
+}
+
+// ID of the calling thread's current context; false when there is none yet or
+// the driver cannot say.
+bool current_context_id(unsigned long long* id)
+{
+    const Driver& d = driver();
+    CUcontext ctx = nullptr;
+    if (d.get_current == nullptr || d.get_id == nullptr) return false;
+    if (d.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return d.get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices];   // device address of g_noalloc_scratch, per device
+std::map<unsigned long long, void*> g_scratch_addr;   // device address of g_noalloc_scratch, per context
 
 // Host code cannot pass g_noalloc_scratch to a kernel: on the host that name is
-// a stand-in, not a device address.  Look the address up once per device, with
-// that device current.
+// a stand-in, not a device address, and the device address belongs to one CUDA
+// context.  So the address is looked up with cudaGetSymbolAddress in the
+// calling thread's current context, the first time a call runs in that
+// context, and cached under the context's ID: a later context (after
+// cudaDeviceReset, or one the caller created itself) gets its own lookup.
 fp4q_status_t scratch_address(void** out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
+    if (have_id) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_scratch_addr.find(id);
+        if (it != g_scratch_addr.end()) {
+            *out = it->second;
+            return FP4Q_SUCCESS;
+        }
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERROR_UNSUPPORTED_DEVICE;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return FP4Q_ERROR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
+    // the lookup made the device's primary context current if none was
+    if (have_id || current_context_id(&id)) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_scratch_addr[id] = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return FP4Q_SUCCESS;
 }
 

@@ -446,12 +446,13 @@ struct ScatterArgs {
     const uint16_t* out_vals;
     const int32_t* out_count;
     uint16_t* y;
-    int64_t rows, cap, ldy;
+    int64_t rows, cols, cap, ldy;
 };
 
 // One thread per (row, slot): the slot's fp16 value, as bf16, to its column.
-// A column at or past the row stride is skipped, so that arrays not made by
-// the separation can never write outside y's [rows][ldy] extent.
+// A column at or past cols is skipped, so that arrays not made by the
+// separation can never write into y's padding columns [cols, ldy) (which may
+// belong to another tensor) nor past the last row's cols elements.
 __global__ void __launch_bounds__(256) outlier_scatter_kernel(ScatterArgs a)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(256) outlier_scatter_kernel(ScatterArgs a)
     const int64_t r = i / a.cap, s = i - r * a.cap;
     if (s >= a.out_count[r]) return;
     const int64_t col = a.out_cols[i];
-    if (col >= a.ldy) return;
+    if (col >= a.cols) return;
     const float v = __half2float(__ushort_as_half(a.out_vals[i]));
     a.y[r * a.ldy + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
@@ -493,13 +494,13 @@ cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t co
 }
 
 cudaError_t launch_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals, const int32_t* out_count,
-                                    int64_t rows, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st)
+                                    int64_t rows, int64_t cols, int64_t cap, uint16_t* y, int64_t ldy, cudaStream_t st)
 {
     const int64_t n = rows * cap;
     if (n == 0) return cudaSuccess;
     const int64_t blocks = (n + 255) / 256;
     if (blocks >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-    ScatterArgs a{out_cols, out_vals, out_count, y, rows, cap, ldy};
+    ScatterArgs a{out_cols, out_vals, out_count, y, rows, cols, cap, ldy};
     outlier_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
     return cudaGetLastError();
 }

@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--layers", type=int, default=32, help="layers in the weight set (32 = the full 8B model)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads (2048^2 weight, activations, 70B MLP, dequantize sweep)")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--fmt", choices=["nvfp4_razer", "nvfp4", "nvfp4_razer_w"], default=FMT,
                    help="format of the run (all three read 4.5625 B/element with the computed tensor scale)")
@@ -193,18 +195,46 @@ def time_oracle(samples, nthreads):
     return n, time.perf_counter() - t0
 
 
-def cpu_baseline_leg():
-    """The oracle as it stands, on every host core, over one full layer (218 M elements)."""
+def cpu_baseline_leg(layer0=None):
+    """The oracle as it stands, on every host core, over one full layer (218 M elements).
+
+    ``layer0``: the GPU's own layer-0 inputs and results, copied to the host after the
+    timed region, as (x bf16 bits, codes, scales, tensor scale, mse) per tensor.  The
+    oracle then quantizes exactly those input bytes, and its results are compared
+    with the GPU's: codes, scales and tensor scales bit for bit, the MSE to its
+    relative difference.  Returns (cpu_baseline, parity or None)."""
+    import numpy as np
     import oracle
     from activation_quantization_block_b200 import synthetic
     nthreads = oracle.default_threads()
-    samples = []
-    for i, (name, r, c) in enumerate(layer_shapes()):
-        samples.append(synthetic.bf16_bits(synthetic.llm_weight(r, c, seed=synthetic.tensor_seed(2, 0, i))))
-    n, dt = time_oracle(samples, nthreads)
-    return {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+    if layer0 is None:
+        layer0 = [(synthetic.bf16_bits(synthetic.llm_weight(r, c, seed=synthetic.tensor_seed(2, 0, i))),)
+                  for i, (name, r, c) in enumerate(layer_shapes())]
+    n, results = 0, []
+    t0 = time.perf_counter()
+    for item in layer0:
+        results.append(oracle.quantize(item[0], FMT, False, want_sse=True, nthreads=nthreads))
+        n += item[0].size
+    dt = time.perf_counter() - t0
+    base = {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "sample": f"one full layer of the weight set (7 tensors, {n} elements), {dt:.2f} s wall, "
-                      f"computed tensor scale + MSE, {nthreads} threads"}
+                      f"computed tensor scale + MSE, {nthreads} threads"
+                      + (", on the GPU's own input bytes" if len(layer0[0]) > 1 else "")}
+    if len(layer0[0]) == 1:
+        return base, None
+    codes_ok, scales_ok, ts_ok, mse_rel = True, True, True, 0.0
+    for (xb, codes, scales, ts, mse), (rc, rs, rts, rsse) in zip(layer0, results):
+        codes_ok = codes_ok and bool(np.array_equal(codes, rc))
+        scales_ok = scales_ok and bool(np.array_equal(scales, rs))
+        ts_ok = ts_ok and bool(np.float32(ts) == np.float32(rts))
+        ref = rsse / xb.size
+        mse_rel = max(mse_rel, abs(mse - ref) / ref if ref > 0 else abs(mse))
+    parity = {"layer0_codes_scales_equal": codes_ok and scales_ok, "codes_equal": codes_ok,
+              "scales_equal": scales_ok, "tensor_scales_equal": ts_ok, "mse_max_rel": mse_rel,
+              "mse_tolerance": 1e-5, "tensors": len(layer0), "elements": n,
+              "how": "the oracle on the GPU's layer-0 input bytes (copied from the device after the timed "
+                     "region); codes, scales and tensor scales compared bit for bit, the MSE relatively"}
+    return base, parity
 
 
 # ---------------------------------------------------------------- multi-rank host logic
@@ -277,6 +307,142 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------- the other workloads
+
+CONFIG_REPEATS = 20
+FLUSH_BYTES = 256 << 20     # written before every timed call: more than the 126 MB L2
+
+
+def time_device(fn, flush, repeats=CONFIG_REPEATS, warmup=3):
+    """Median and minimum device time (us) of fn() over `repeats` calls, each preceded by a
+    write of a buffer larger than L2 (outside the timed pair of events).  The flush also
+    keeps the GPU busy while the host enqueues the call, so the events time the device."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    ts = []
+    for _ in range(repeats):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    us = sorted(1e3 * a.elapsed_time(b) for a, b in ts)
+    return statistics.median(us), us[0]
+
+
+def oracle_rates(xb, fmt, rotate, op="quantize", packed=None):
+    """The oracle's elements/s on host bf16 bits (quantize) or packed inputs (dequantize), on one
+    thread and on every core."""
+    import oracle
+    out = {}
+    for label, nt in (("oracle_1t", 1), ("oracle_nt", oracle.default_threads())):
+        t0 = time.perf_counter()
+        if op == "quantize":
+            oracle.quantize(xb, fmt, rotate, want_sse=True, nthreads=nt)
+            n = xb.size
+        else:
+            codes, scales, ts = packed
+            oracle.dequantize(codes, scales, ts, fmt, rotate, nthreads=nt)
+            n = codes.size * 2
+        out[label] = {"elements_per_s": n / (time.perf_counter() - t0), "threads": nt, "elements": n}
+    return out
+
+
+def measure_configs(dev, peak, with_oracle=True):
+    """Every other workload of the benchmark suite, each call timed alone (median of 20, L2
+    flushed before each): throughput, algorithmic GB/s and its fraction of the copy
+    bandwidth, the MSE, and the oracle's rates on the host cores (one thread on a row
+    slice, all cores on the stated slice).  The two small workloads also report the fixed
+    cost of a call (the same call on a 128 x 64 tensor) and its share of their time."""
+    import torch
+    from activation_quantization_block_b200 import fp4q, synthetic
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = []
+
+    def quant_entry(name, x, fmt, rotate, slice_rows, tiny_us=None):
+        rows, cols = x.shape
+        q = fp4q.empty_like_quantized(x, fmt)
+        ws = torch.zeros(fp4q.fp4q_workspace_size(rows, cols, fmt, rotate), dtype=torch.uint8, device=dev)
+
+        def call():
+            st = fp4q.fp4q_quantize(x, rows, cols, cols, fmt, rotate, 0, q.codes, q.scales, q.tensor_scale,
+                                    q.mse, ws, ws.numel())
+            if st != 0:
+                raise fp4q.Fp4qError(st, "fp4q_quantize")
+        med, best = time_device(call, flush)
+        n = x.numel()
+        B = fp4q.block_size(fmt)
+        nbytes = 2 * n + n // 2 + n // B + (2 * n if fmt != "mxfp4" else 0)
+        e = {"workload": name, "op": "quantize", "format": fmt, "rotate": rotate, "shape": [rows, cols],
+             "elements": n, "us_median": med, "us_min": best, "elements_per_s": n / (med / 1e6),
+             "alg_bytes": nbytes, "gbs": nbytes / (med / 1e6) / 1e9, "frac": nbytes / (med / 1e6) / 1e9 / peak,
+             "mse": float(q.mse.item())}
+        if tiny_us is not None:
+            e["call_overhead_us"] = tiny_us
+            e["call_overhead_share"] = min(1.0, tiny_us / med)
+        if with_oracle:
+            xb = synthetic.bf16_bits(x[:slice_rows])
+            e.update(oracle_rates(xb, fmt, bool(rotate)))
+            e["oracle_slice_rows"] = slice_rows
+        out.append(e)
+
+    def tiny_call_us(fmt, rotate):
+        x = synthetic.llm_weight(128, 64, seed=9, device=dev)
+        q = fp4q.empty_like_quantized(x, fmt)
+        ws = torch.zeros(fp4q.fp4q_workspace_size(128, 64, fmt, rotate), dtype=torch.uint8, device=dev)
+        return time_device(lambda: fp4q.fp4q_quantize(x, 128, 64, 64, fmt, rotate, 0, q.codes, q.scales,
+                                                      q.tensor_scale, q.mse, ws, ws.numel()), flush)[0]
+
+    # 2048 x 2048 LLM weight, NVFP4 and NVFP4_RAZER
+    x = synthetic.llm_weight(2048, 2048, seed=0, device=dev)
+    for fmt in ("nvfp4", "nvfp4_razer"):
+        quant_entry("2048x2048 llm weight N(0,0.02^2)+0.1% outliers x20, seed 0", x, fmt, 0, 2048,
+                    tiny_us=tiny_call_us(fmt, 0))
+    # 8192 x 4096 activations, MXFP4 with and without rotation
+    x = synthetic.activation_t3(8192, 4096, seed=1, device=dev)
+    for rot in (0, 1):
+        quant_entry("8192x4096 activations, column LogNormal(0,1) x Student-t(3), seed 1", x, "mxfp4", rot,
+                    512 if rot else 8192, tiny_us=tiny_call_us("mxfp4", rot))
+    del x
+    # 70B MLP block, NVFP4 / NVFP4_RAZER / MXFP4 + rotation
+    for i, (pname, r, c) in enumerate(synthetic.LLAMA3_70B_MLP):
+        x = synthetic.mlp_row_scaled(r, c, seed=synthetic.tensor_seed(3, 0, i), device=dev)
+        for fmt, rot in (("nvfp4", 0), ("nvfp4_razer", 0), ("mxfp4", 1)):
+            quant_entry(f"70B MLP {pname} {r}x{c}, row LogNormal(0,0.5) x N(0,0.015^2), seed 3", x, fmt, rot,
+                        256 if rot else 1024)
+        del x
+    torch.cuda.empty_cache()
+    # dequantize sweep 8192 x N
+    for N in (4096, 14336, 28672, 57344):
+        for fmt in ("nvfp4_razer", "mxfp4"):
+            codes, scales, ts = synthetic.random_packed(8192, N, fmt, seed=4, device=dev)
+            y = torch.empty(8192, N, dtype=torch.bfloat16, device=dev)
+
+            def call():
+                st = fp4q.fp4q_dequantize(codes, scales, ts, 8192, N, fmt, 0, y, N)
+                if st != 0:
+                    raise fp4q.Fp4qError(st, "fp4q_dequantize")
+            med, best = time_device(call, flush)
+            n = 8192 * N
+            nbytes = n // 2 + n // fp4q.block_size(fmt) + 2 * n
+            e = {"workload": f"dequantize sweep 8192x{N}, random codes and valid scales, seed 4", "op": "dequantize",
+                 "format": fmt, "rotate": 0, "shape": [8192, N], "elements": n, "us_median": med, "us_min": best,
+                 "elements_per_s": n / (med / 1e6), "alg_bytes": nbytes, "gbs": nbytes / (med / 1e6) / 1e9,
+                 "frac": nbytes / (med / 1e6) / 1e9 / peak}
+            if with_oracle and N == 4096:
+                e.update(oracle_rates(None, fmt, False, op="dequantize",
+                                      packed=(codes[:1024].cpu().numpy(), scales[:1024].cpu().numpy(), 1.0)))
+                e["oracle_slice_rows"] = 1024
+            out.append(e)
+            del codes, scales, y
+    del flush
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -399,6 +565,11 @@ def main():
     mses = torch.cat([q.mse for _, _, q in tensors]).cpu()
     outputs_sha = sha256_of([t for _, _, q in tensors[:layer0] for t in (q.codes, q.scales)])
     assert torch.isfinite(mses).all() and (mses > 0).all()
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    host_layer0 = None
+    if want_cpu:   # the GPU's own layer-0 bytes and results, for the oracle leg
+        host_layer0 = [(synthetic.bf16_bits(x), q.codes.cpu().numpy(), q.scales.cpu().numpy(),
+                        float(q.tensor_scale.item()), float(q.mse.item())) for _, x, q in tensors[:layer0]]
 
     # ---- end to end from pinned host memory -------------------------------------------
     e2e = None
@@ -426,8 +597,10 @@ def main():
         "gpu_launches": launches_per_call * len(calls) * args.steps,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_leg()
+    if want_cpu:
+        line["cpu_baseline"], line["parity"] = cpu_baseline_leg(host_layer0)
+    if rank == 0 and world == 1 and not args.no_configs:
+        line["configs"] = measure_configs(dev, peak, with_oracle=not args.no_cpu_baseline)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -268,9 +268,12 @@ FP4Q_API fp4q_status_t fp4q_selftest_timeout(fp4q_stream_t stream);
  * FP4Q_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
  * until the process exits.  The call allocates nothing and frees nothing.
  *
- *  - The first call on each device, with that device current, looks up the
- *    array's device address (cudaGetSymbolAddress) and caches it; make that
- *    first call before any stream capture.
+ *  - The array's device address belongs to one CUDA context.  The first call
+ *    in each context (the calling thread's current one; the device's primary
+ *    context for a runtime-API program) looks it up with cudaGetSymbolAddress
+ *    and caches it under that context's ID, so a call after cudaDeviceReset,
+ *    or under a context the caller made current itself, gets that context's
+ *    copy.  Make the first call in each context before any stream capture.
  *  - Every call on a device shares the one array, which keeps the previous
  *    call's contents.  Nothing in it needs clearing (each call writes every
  *    slot it reads), but calls that can overlap on the GPU -- on different
@@ -363,8 +366,9 @@ FP4Q_API fp4q_status_t fp4q_separate_outliers(const void* x, int64_t rows, int64
 
 /* y[r][out_cols[r][s]] = bf16(out_vals[r][s]) for s < min(out_count[r], cap):
  * puts the outliers back into a bf16 reconstruction y [rows][ldy].  The arrays
- * are those fp4q_separate_outliers wrote (columns below cols); a column at or
- * past ldy is skipped, so no write leaves y's [rows][ldy] extent. */
+ * are those fp4q_separate_outliers wrote (columns below cols); a slot whose
+ * column is at or past cols is skipped, so no write lands in y's padding
+ * columns [cols, ldy) or past element (rows-1)*ldy + cols - 1. */
 FP4Q_API fp4q_status_t fp4q_scatter_outliers(const uint16_t* out_cols, const uint16_t* out_vals,
                                              const int32_t* out_count, int64_t rows, int64_t cols, int64_t cap,
                                              void* y, int64_t ldy, fp4q_stream_t stream);

@@ -77,6 +77,31 @@ def test_scatter_puts_values_back(dev):
     assert np.array_equal(synthetic.bf16_bits(y), want.astype(ml_dtypes.bfloat16).view(np.uint16))
 
 
+def test_scatter_skips_columns_at_or_past_cols(dev):
+    """Hand-made slots whose columns lie in [cols, ldy) or beyond: nothing may land
+    in the padding columns of a strided y, nor past the last row's cols elements."""
+    rows, cols, ldy, guard = 5, 256, 264, 64
+    cap = fp4q.fp4q_outlier_capacity(cols, 0.02)            # 5
+    oc = np.zeros((rows, cap), np.uint16)
+    ov = np.full((rows, cap), 7.0, np.float16)
+    cnt = np.full(rows, cap, np.int32)
+    for r in range(rows):
+        oc[r] = [r, cols, cols + 3, ldy - 1, ldy + 40][:cap]   # one valid column, the rest out of range
+    o = fp4q.Outliers(None, torch.from_numpy(oc.view(np.int16)).to(dev), torch.from_numpy(ov).to(dev),
+                      torch.from_numpy(cnt).to(dev))
+    # y ends right after (rows-1)*ldy + cols elements; a guard region follows
+    n = (rows - 1) * ldy + cols
+    buf = torch.full((n + guard,), -3.0, dtype=torch.bfloat16, device=dev)
+    st = fp4q.fp4q_scatter_outliers(o.cols, o.vals, o.count, rows, cols, cap, buf, ldy)
+    assert st == 0, fp4q.fp4q_status_string(st)
+    torch.cuda.synchronize()
+    got = buf.float().cpu().numpy()
+    want = np.full(n + guard, -3.0, np.float32)
+    for r in range(rows):
+        want[r * ldy + r] = 7.0
+    assert np.array_equal(got, want)
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4_razer", "nvfp4_razer_w"])
 def test_separated_pipeline_lowers_the_error(orc, dev, fmt):
     """A 4096 x 4096 LLM weight (0.1 % outliers x20): the bulk's codes match the

@@ -17,6 +17,7 @@ import pytest
 import torch
 
 from activation_quantization_block_b200 import fp4q, synthetic
+from tests import bruteforce as bf
 
 pytestmark = pytest.mark.gpu
 
@@ -253,11 +254,31 @@ def test_zeros_and_zero_rows(orc, dev, fmt):
     check_exact(orc, y.to(dev), fmt)
 
 
+def _nibbles(codes: np.ndarray) -> np.ndarray:
+    out = np.zeros((codes.shape[0], codes.shape[1] * 2), dtype=np.int64)
+    out[:, 0::2] = codes & 0x0F
+    out[:, 1::2] = codes >> 4
+    return out
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_extreme_magnitudes(orc, dev, fmt):
     rng = np.random.default_rng(8)
     sub = rng.integers(1, 128, size=(4, 64)) * 2.0 ** -133 * rng.choice([-1, 1], size=(4, 64))
-    check_exact(orc, _bf(sub).to(dev), fmt)                       # bf16 subnormals only
+    sub[rng.random(sub.shape) < 0.2] = 0.0                          # zeros among them
+    near = rng.uniform(-1.5, 1.5, size=(4, 64)) * 2.0 ** -126       # absmax up to 6 * 2^-128
+    near[0, :7] = 0.0
+    for tiny in (sub, near):
+        # bf16 subnormals (and their neighbours): for NVFP4 formats every block's
+        # RN(1 / den) overflows, and elements are scaled by division instead
+        xt = _bf(tiny)
+        codes, scales, ts, _ = check_exact(orc, xt.to(dev), fmt)
+        assert np.all(_nibbles(codes)[bits(xt) == 0] == 0), "a zero must stay code +0"
+        bcodes, bscales, bts = bf.quantize_bruteforce(bits(xt), fmt, False)
+        assert np.array_equal(codes, bcodes) and np.array_equal(scales, bscales)
+        if fmt != "mxfp4":
+            assert ts == bts and 0 < ts < 2.0 ** -120
+        check_rotated(orc, xt.to(dev), fmt)
     big = rng.standard_normal((4, 64)) * 1e37
     big[1, 3] = 3.3895313892515355e38                              # largest bf16
     big[2, 7] = -3.3895313892515355e38
