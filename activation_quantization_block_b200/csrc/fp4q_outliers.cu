@@ -7,12 +7,14 @@
 // positions, and the bulk, with the group mean in their place, is quantized.
 // The group is a matrix row, handled by one warp (rows of up to 8192 elements)
 // or one CTA, the row copied once into shared memory:
-//   1. mu = sum / n and sigma = sqrt(sum (x - mu)^2 / n) in fp64 (fixed-order
-//      reductions), threshold T = k sigma;
+//   1. mu and sigma in one fp64 pass over the row (sums of x - c and of its
+//      square around c, the row's first element; fixed-order reductions),
+//      threshold T = k sigma;
 //   2. one pass writes the bulk row (the mean, rounded to bf16, at every
 //      outlier) and the outliers in column order, their slots from prefix
 //      counts; |x - mu| > T is decided in fp32 outside a guard band that covers
-//      the fp32 roundings, in fp64 inside it;
+//      the fp32 roundings, in fp64 inside it; a step in which no element of the
+//      warp (or CTA) comes near the threshold copies the row and counts nothing;
 //   3. only if that pass counted more than cap = floor(max_frac * n): T becomes
 //      the cap-th largest deviation, found by bisection on the deviations' fp64
 //      bit patterns (monotone for non-negative values), ties at T are taken
@@ -147,6 +149,37 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rn(double m)
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Mean and population deviation of a row of n8 16-byte chunks of bf16 in
+// shared memory, in one pass: the sums S1 = sum (x - c) and S2 = sum (x - c)^2
+// around c, the row's first element, give mu = c + S1 / n and
+// sigma^2 = S2 / n - (S1 / n)^2 (taken as 0 if rounding makes it negative).
+// Every difference, square and sum is fp64, eight partial sums per thread
+// combined in a fixed order and then by `reduce` (a fixed-order sum over the
+// warp or the CTA).  Shifting by an element of the row keeps the cancellation
+// in sigma^2 small: its relative rounding is about 2^-53 ((mu - c) / sigma)^2.
+template <typename Reduce>
+__device__ __forceinline__ void row_moments(uint32_t row, int64_t n8, int64_t first, int64_t stride, double c,
+                                            Reduce reduce, double& mu, double& sigma)
+{
+    double p1[8] = {0, 0, 0, 0, 0, 0, 0, 0}, p2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int64_t i = first; i < n8; i += stride) {
+        float v[8];
+        load8(row, 8 * i, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const double d = (double)v[q] - c;
+            p1[q] += d;
+            p2[q] = fma(d, d, p2[q]);
+        }
+    }
+    const double n = (double)(8 * n8);
+    const double s1 = reduce(((p1[0] + p1[1]) + (p1[2] + p1[3])) + ((p1[4] + p1[5]) + (p1[6] + p1[7])));
+    const double s2 = reduce(((p2[0] + p2[1]) + (p2[2] + p2[3])) + ((p2[4] + p2[5]) + (p2[6] + p2[7])));
+    const double m1 = s1 / n;
+    mu = c + m1;
+    sigma = sqrt(fmax(s2 / n - m1 * m1, 0.0));
+}
+
 __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a)
 {
     extern __shared__ uint4 srow_raw[];
@@ -160,28 +193,14 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
     copy_row(srow_raw, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n / 8, t, kOutThreads);
     __syncthreads();
 
-    // 1. mean and deviation (eight partial sums per thread, combined in a fixed order)
-    double p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
-        float v[8];
-        load8(row, j, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] += (double)v[i];
+    // 1. mean and deviation, one pass over the row in shared memory
+    double mu, thr;
+    {
+        float v0[8];
+        load8(row, 0, v0);
+        row_moments(row, n / 8, t, kOutThreads, (double)v0[0], [&](double v) { return cta_sum(v, shd); }, mu, thr);
+        thr *= a.k;
     }
-    const double mu = cta_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])), shd) / (double)n;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) p[i] = 0.0;
-    for (int64_t j = 8 * (int64_t)t; j < n; j += kOutTile) {
-        float v[8];
-        load8(row, j, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const double d = (double)v[i] - mu;
-            p[i] = fma(d, d, p[i]);
-        }
-    }
-    double thr = a.k * sqrt(cta_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])), shd) /
-                            (double)n);
 
     // 2. bulk row and outliers in column order, speculatively with k sigma (the
     // count stays within the cap in the usual case); above the cap, the cap-th
@@ -212,6 +231,17 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
             if (in) {
                 w = lds128(row + 2u * (uint32_t)j);
                 load8(row, j, v);
+            }
+            // the usual step: no element of the CTA's chunks near or above the
+            // threshold, so the bulk is the row unchanged and nothing is counted
+            float dm = 0.0f;
+            if (in && !none) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dm = fmaxf(dm, fabsf(v[i] - mu32));
+            }
+            if (__syncthreads_and(none || dm - t32 < -band)) {
+                if (in) *reinterpret_cast<uint4*>(brow + j) = w;
+                continue;
             }
             uint32_t gmask = 0, emask = 0;
             if (in && !none) {
@@ -320,30 +350,13 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
     copy_row(srow, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n8, lane, 32);
     __syncwarp();
 
-    // eight independent partial sums per lane (one per position in the 16-byte
-    // chunk), combined in a fixed order: the additions overlap instead of
-    // forming one chain of fp64 latencies
-    double p[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int64_t i = lane; i < n8; i += 32) {
-        float v[8];
-        load8(row, 8 * i, v);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) p[q] += (double)v[q];
+    double mu, thr;
+    {
+        float v0[8];
+        load8(row, 0, v0);
+        row_moments(row, n8, lane, 32, (double)v0[0], [](double v) { return warp_sum(v); }, mu, thr);
+        thr *= a.k;
     }
-    const double mu = warp_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]))) / (double)n;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) p[q] = 0.0;
-    for (int64_t i = lane; i < n8; i += 32) {
-        float v[8];
-        load8(row, 8 * i, v);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const double d = (double)v[q] - mu;
-            p[q] = fma(d, d, p[q]);
-        }
-    }
-    double thr =
-        a.k * sqrt(warp_sum(((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]))) / (double)n);
 
     auto count_where = [&](auto pred) {
         int c = 0;
@@ -376,6 +389,17 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
             if (in) {
                 wd = lds128(row + 16u * (uint32_t)i);
                 load8(row, 8 * i, v);
+            }
+            // the usual step: no element of the warp's chunks near or above the
+            // threshold, so the bulk is the row unchanged and nothing is counted
+            float dm = 0.0f;
+            if (in && !none) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dm = fmaxf(dm, fabsf(v[q] - mu32));
+            }
+            if (__all_sync(0xFFFFFFFFu, none || dm - t32 < -band)) {
+                if (in) *reinterpret_cast<uint4*>(brow + 8 * i) = wd;
+                continue;
             }
             uint32_t gmask = 0, emask = 0;
             if (in && !none) {

@@ -99,3 +99,35 @@ def test_sha256_of_tensors_is_the_digest_of_their_bytes():
     wide = torch.zeros(4, 8, dtype=torch.bfloat16)
     assert bench.sha256_of([wide[:, :4]]) == bench.sha256_of([torch.zeros(4, 4, dtype=torch.bfloat16)])
     assert bench.sha256_of([object()]).startswith("unavailable:")
+
+
+def test_cpu_baseline_leg_checks_the_gpu_results_against_the_oracle():
+    """The oracle leg quantizes the given input bytes and compares the given results with its
+    own: equal results report parity, and one changed code byte, scale byte, tensor scale or
+    an MSE off by more than 1e-5 is caught.  (Results here come from the oracle itself.)"""
+    import numpy as np
+    import oracle
+
+    import bench
+    from activation_quantization_block_b200 import synthetic
+    xs = [synthetic.bf16_bits(synthetic.llm_weight(r, c, seed=70 + i)) for i, (r, c) in enumerate([(32, 64), (8, 256)])]
+    layer0 = []
+    for xb in xs:
+        codes, scales, ts, sse = oracle.quantize(xb, bench.FMT, False)
+        layer0.append((xb, codes, scales, float(ts), sse / xb.size))
+    base, parity = bench.cpu_baseline_leg(layer0)
+    assert base["kind"] == "oracle" and base["value"] > 0 and "own input bytes" in base["sample"]
+    assert parity["layer0_codes_scales_equal"] and parity["tensor_scales_equal"] and parity["mse_max_rel"] < 1e-12
+    bad_codes = layer0[1][1].copy()
+    bad_codes[3, 5] ^= 0x10
+    _, p = bench.cpu_baseline_leg([layer0[0], (xs[1], bad_codes) + layer0[1][2:]])
+    assert not p["codes_equal"] and p["scales_equal"] and not p["layer0_codes_scales_equal"]
+    bad_scales = layer0[0][2].copy()
+    bad_scales[0, 0] ^= 1
+    _, p = bench.cpu_baseline_leg([(xs[0], layer0[0][1], bad_scales) + layer0[0][3:]])
+    assert not p["scales_equal"]
+    _, p = bench.cpu_baseline_leg([layer0[0][:3] + (np.nextafter(np.float32(layer0[0][3]), np.float32(1)),
+                                                     layer0[0][4])])
+    assert not p["tensor_scales_equal"]
+    _, p = bench.cpu_baseline_leg([layer0[0][:4] + (layer0[0][4] * (1 + 3e-5),)])
+    assert p["mse_max_rel"] > p["mse_tolerance"]
