@@ -1,9 +1,11 @@
 // C ABI of fp4q (declared in include/fp4q.h): argument validation, workspace
 // carving and kernel dispatch.  Validation happens on the host before any
 // launch; a rejected call enqueues nothing.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
 #include <mutex>
 #include <vector>
 
@@ -13,7 +15,44 @@
 
 using namespace fp4q;
 
+#ifndef FP4Q_DEBUG
+#define FP4Q_DEBUG 0
+#endif
+
+// The one set of device error words of the library (see device_error_words).
+__device__ unsigned int g_fp4q_error_words[kErrorWords];
+
 namespace {
+
+// Driver calls that name the calling thread's current CUDA context: its handle
+// and its ID, unique for the life of the process.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id)
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (get_current == nullptr || get_id == nullptr) return false;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+std::mutex g_err_mu;
+std::map<unsigned long long, unsigned int*> g_err_addr;   // device address of the words, per context ID
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
@@ -79,6 +118,30 @@ bool valid_flags(uint32_t flags, int fmt)
 }
 
 }  // namespace
+
+// The address belongs to one context: look it up with cudaGetSymbolAddress in
+// the calling thread's current context the first time, and cache it under the
+// context's ID (after cudaDeviceReset, or under another context, a new lookup).
+unsigned int* fp4q::device_error_words()
+{
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (have_id) {
+        std::lock_guard<std::mutex> lk(g_err_mu);
+        auto it = g_err_addr.find(id);
+        if (it != g_err_addr.end()) return it->second;
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fp4q_error_words) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (have_id || current_context_id(&id)) {
+        std::lock_guard<std::mutex> lk(g_err_mu);
+        g_err_addr[id] = static_cast<unsigned int*>(p);
+    }
+    return static_cast<unsigned int*>(p);
+}
 
 extern "C" {
 
@@ -239,16 +302,38 @@ fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear)
     if (bits == nullptr) return FP4Q_ERROR_INVALID_VALUE;
     fp4q_status_t s = check_device();
     if (s != FP4Q_SUCCESS) return s;
-    unsigned int v = 0, w = 0, u = 0, z = 0;
-    if (read_device_errors(&v, clear != 0) != cudaSuccess || read_batch_device_errors(&w, clear != 0) != cudaSuccess ||
-        read_gemm_device_errors(&u, clear != 0) != cudaSuccess ||
-        read_selftest_device_errors(&z, clear != 0) != cudaSuccess) {
+    unsigned int w[kErrorWords] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(w, g_fp4q_error_words, sizeof w) != cudaSuccess) {
         cudaGetLastError();
         return FP4Q_ERROR_CUDA;
     }
-    *bits = v | w | u | z;
+    if (clear) {
+        const unsigned int zero[kErrorWords] = {0, 0, 0, 0};
+        if (cudaMemcpyToSymbol(g_fp4q_error_words, zero, sizeof zero) != cudaSuccess) {
+            cudaGetLastError();
+            return FP4Q_ERROR_CUDA;
+        }
+    }
+    *bits = w[0];
     return FP4Q_SUCCESS;
 }
+
+fp4q_status_t fp4q_device_error_site(uint32_t* site, uint64_t* offset)
+{
+    if (site == nullptr || offset == nullptr) return FP4Q_ERROR_INVALID_VALUE;
+    fp4q_status_t s = check_device();
+    if (s != FP4Q_SUCCESS) return s;
+    unsigned int w[kErrorWords] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(w, g_fp4q_error_words, sizeof w) != cudaSuccess) {
+        cudaGetLastError();
+        return FP4Q_ERROR_CUDA;
+    }
+    *site = w[1];
+    *offset = (uint64_t)w[2] | ((uint64_t)w[3] << 32);
+    return FP4Q_SUCCESS;
+}
+
+int fp4q_debug_build(void) { return FP4Q_DEBUG ? 1 : 0; }
 
 fp4q_status_t fp4q_selftest_timeout(fp4q_stream_t stream)
 {

@@ -54,6 +54,7 @@ struct ChainArgs {
     int32_t n_sse_in;
     int32_t has_fin;
     int32_t mx_ceil;
+    unsigned* err;          // the library's device error words
 };
 
 template <int FMT, bool ROT, bool SSE>
@@ -81,15 +82,29 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     const int64_t my_q = b < nq ? (nq - 1 - b) / G + 1 : 0;
     const int64_t my_a = ab < na ? (na - 1 - ab) / G + 1 : 0;
     const int64_t mine = my_q + my_a;
-    auto item = [&](int64_t jj, bool& is_q, int64_t& tile) {
-        const int64_t k = jj * my_q / mine;   // quantize items before item jj
-        is_q = (jj + 1) * my_q / mine > k;
-        tile = is_q ? nq - 1 - (b + k * G) : ab + (jj - k) * G;
+    // Thread 0 walks the items in order: before item jj come k = floor(jj my_q /
+    // mine) quantize items, stepped without a division (rem = jj my_q - k mine,
+    // in [0, mine); my_q <= mine, so one step adds at most one).
+    // The cursor lives in shared memory: only thread 0 uses it, and kept in
+    // registers across the tile loop it would cost the encoder registers.
+    __shared__ int64_t cur_k, cur_rem;
+    if (t == 0) cur_k = cur_rem = 0;
+    auto next_item = [&](int64_t jj, bool& is_q, int64_t& tile) {
+        const int64_t k0 = cur_k;
+        int64_t k1 = k0, rem1 = cur_rem + my_q;
+        if (rem1 >= mine) {
+            rem1 -= mine;
+            ++k1;
+        }
+        is_q = k1 > k0;
+        tile = is_q ? nq - 1 - (b + k0 * G) : ab + (jj - k0) * G;
+        cur_k = k1;
+        cur_rem = rem1;
     };
-    auto issue = [&](int64_t jj) {
+    auto issue = [&](int64_t jj) {   // thread 0, for jj = 0, 1, 2, ... in order
         bool is_q;
         int64_t tile;
-        item(jj, is_q, tile);
+        next_item(jj, is_q, tile);
         const int s = (int)(jj % kStages);
         slot_q[s] = is_q ? 1 : 0;
         slot_tile[s] = tile;
@@ -113,7 +128,9 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     if (a.has_q && FMT != kMX) {
         if (a.computed) {
             float mx = 0.0f;
-            for (int i = t; i < a.n_amax_in; i += kThreads) mx = fmaxf(mx, a.amax_in[i]);
+            for (int i = t; i < a.n_amax_in; i += kThreads)
+                if (in_bounds(4 * (int64_t)i, 4, 4 * (int64_t)kMaxPartials, kSiteAmaxPartialLoad, a.err))
+                    mx = fmaxf(mx, a.amax_in[i]);
             mx = block_max(mx, shf);
             s_t = tensor_scale_of<FMT>(mx);
             if (b == 0 && t == 0) *a.tensor_scale = s_t;
@@ -124,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     // Finaliser: fixed-order sum of the previous kernel's error partials.
     if (a.has_fin && b == 0) {
         double s = 0.0;
-        for (int i = t; i < a.n_sse_in; i += kThreads) s += a.sse_in[i];
+        for (int i = t; i < a.n_sse_in; i += kThreads)
+            if (in_bounds(8 * (int64_t)i, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialLoad, a.err)) s += a.sse_in[i];
         shd[t] = s;
         __syncthreads();
         for (int o = kThreads / 2; o > 0; o >>= 1) {
@@ -145,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     float m = 0.0f;
     for (int64_t jj = 0; jj < mine; ++jj) {
         if (!pipe_acquire(p, jj)) {
-            pipe_fail(p, jj, jj + kStages < mine ? jj + kStages : mine);
+            pipe_fail(p, jj, jj + kStages < mine ? jj + kStages : mine, a.err);
             break;
         }
         const int s = (int)(jj % kStages);
@@ -154,16 +172,18 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
         const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
         if (is_q) {
             if (a.q_flat)
-                acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0);
+                acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0,
+                                                          a.err);
             else
-                acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0);
+                acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0,
+                                                           a.err);
         } else {
             m = fmaxf(m, amax_tile<ROT>(tp));
         }
         pipe_release(p, jj);
         if (t == 0 && jj + kStages < mine) {
             if (!pipe_stage_free(p, jj)) {
-                pipe_fail(p, jj + 1, jj + kStages);
+                pipe_fail(p, jj + 1, jj + kStages, a.err);
                 break;
             }
             issue(jj + kStages);
@@ -171,11 +191,11 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     }
     if (a.has_a) {
         m = block_max(m, shf);
-        if (t == 0) a.amax_out[b] = m;
+        if (t == 0 && in_bounds(4 * b, 4, 4 * (int64_t)kMaxPartials, kSiteAmaxPartialStore, a.err)) a.amax_out[b] = m;
     }
     if (a.has_q && SSE) {
         acc = block_sum(acc, shd);
-        if (t == 0) a.sse_out[b] = acc;
+        if (t == 0 && in_bounds(8 * b, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialStore, a.err)) a.sse_out[b] = acc;
     }
 }
 
@@ -253,11 +273,14 @@ cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rot
         const Geometry g = make_geometry(ts[k].rows, ts[k].cols, ts[k].ldx);
         if (!make_view(ts[k].x, g, &views[(size_t)k].map, &views[(size_t)k].tl)) return cudaErrorInvalidValue;
     }
+    unsigned* err = device_error_words();
+    if (err == nullptr) return cudaErrorInvalidSymbol;
     const int lag = computed ? 1 : 0;            // kernel j quantizes tensor j - lag
     std::vector<int> grids((size_t)n + 2, 0);    // CTAs (= partials written) of kernel j
     for (int64_t j = 0; j < n + lag + 1; ++j) {
         ChainArgs a = {};
         a.mx_ceil = mx_ceil;
+        a.err = err;
         const int64_t kq = j - lag;              // tensor quantized by kernel j
         const int64_t ka = computed ? j : -1;    // tensor whose absmax pass kernel j runs
         const int64_t kf = j - lag - 1;          // tensor whose MSE kernel j finalises
@@ -304,17 +327,6 @@ cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rot
         grids[(size_t)j] = grid;
     }
     return cudaSuccess;
-}
-
-cudaError_t read_batch_device_errors(unsigned int* bits, bool clear)
-{
-    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    if (clear) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-    }
-    return e;
 }
 
 }  // namespace fp4q

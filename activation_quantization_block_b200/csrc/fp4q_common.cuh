@@ -42,9 +42,6 @@ __device__ __forceinline__ float tensor_scale_of(float amax)
     return __fdiv_rn(amax, FMT == kRW ? 180.0f : 2688.0f);
 }
 
-// Device error word of a translation unit (bits: kErrPipelineTimeout); each
-// unit that launches kernels reads and clears its own copy for the C ABI.
-static __device__ unsigned int g_device_error;
 
 // ---------------------------------------------------------------------------
 // Tiles and units
@@ -380,42 +377,6 @@ __device__ __forceinline__ void razer_tent(const float* v, uint32_t& w0, uint32_
     razer_apply(cs, sp[0].x + sp[0].y, w0, w1, sb);
 }
 
-// Weight-mode remap of one block (candidates +5, -5, +2.5, -2.5 = selectors
-// 0..3) given c5[i] = sign(v_i) * gain of remapping element i to
-// sign(v_i) * 5 and c2[i] likewise for 2.5, U5, U2 the sums of the gains and
-// S5, S2 the sums of the signed gains.  For either pair the better member's
-// gain is (U + |S|) / 2; these sums are exact (gains of 5 are multiples of
-// 2^-20 up to 1, of 2.5 multiples of 2^-22 up to 1/4), so the comparisons
-// are.  The pair 2.5 is taken only when its gain is strictly larger, and in
-// a pair the negative member only when its gain is strictly larger: ties go
-// to the lower selector.  Winners are flagged as in razer_apply, the gains of
-// the pair not taken multiplied by 0 (a candidate for one pair never is for
-// the other).  Returns the chosen gain.
-__device__ __forceinline__ float razer_w_apply(const float* c5, const float* c2, float U5, float S5, float U2,
-                                               float S2, uint32_t& w0, uint32_t& w1, uint32_t& sb)
-{
-    const float t5 = U5 + fabsf(S5), t2 = U2 + fabsf(S2);
-    const bool p2 = t2 > t5;
-    const bool neg = (p2 ? S2 : S5) < 0.0f;
-    const float sk = neg ? -0x1p40f : 0x1p40f;
-    const float k5 = p2 ? 0.0f : sk, k2 = p2 ? sk : 0.0f;
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const float2 p = fma2_rn(make_float2(c2[i], c2[i + 1]), make_float2(k2, k2),
-                                 mul2_rn(make_float2(c5[i], c5[i + 1]), make_float2(k5, k5)));
-        x[i] = p.x;
-        x[i + 1] = p.y;
-    }
-    const uint32_t k0 = e2m1x8(x), k1 = e2m1x8(x + 8);
-    const uint32_t f0 = k0 & ~(k0 >> 3) & 0x11111111u;
-    const uint32_t f1 = k1 & ~(k1 >> 3) & 0x11111111u;
-    w0 = (w0 & ~(f0 * 15u)) | (f0 << 3);
-    w1 = (w1 & ~(f1 * 15u)) | (f1 << 3);
-    sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
-    return 0.5f * fmaxf(t5, t2);
-}
-
 // Gain of remapping |v| to 2.5: its regular value is 2 (|v| <= 2.5) or 3,
 // and (|v| - q)^2 - (|v| - 2.5)^2 = 1/4 - | |v| - 2.5 |, positive exactly on
 // (2.25, 2.75) and clamped to 0 elsewhere; |v| - 2.5 is exact there, so the
@@ -425,42 +386,80 @@ __device__ __forceinline__ float razer_gain_w2(float v)
     return __saturatef(0.25f - fabsf(fabsf(v) - kRazerWPair));
 }
 
-// Weight-mode selection from the scaled values alone (any magnitude).
-__device__ __forceinline__ void razer_w_tent(const float* v, uint32_t& w0, uint32_t& w1, uint32_t& sb)
+// Rewrite the winners flagged in k (nibbles 0xF) to 0b1000.
+__device__ __forceinline__ uint32_t apply_winners(uint32_t w, uint32_t k)
 {
-    float c5[16], c2[16];
-    float2 u5[8], s5[8], u2[8], s2[8];
+    const uint32_t f = k & (k >> 3) & 0x11111111u;
+    return (w & ~(f * 15u)) | (f << 3);
+}
+
+
+// Weight-mode selection in running form: for each run of eight elements the
+// gains of 5 (from e = q - v when GE, else from v) and of 2.5, their sums and
+// signed sums, and a candidate marker
+// per element: the E2M1 code of sign(v) * gain * 2^40, +6 (0x7) for a
+// candidate of the positive member, -6 (0xF) of the negative one, +-0
+// otherwise.  Gains of 5 are multiples of 2^-20 up to 1 and gains of 2.5
+// multiples of 2^-22 up to 1/4, so every sum is exact in any order and the
+// comparisons are exact.  For either pair the better member's gain is
+// (U + |S|) / 2; the pair 2.5 is taken only when its gain is strictly larger,
+// and in a pair the negative member only when its gain is strictly larger
+// (ties go to the lower selector; a block with no gain keeps selector 0).  The
+// winners are the chosen value's candidates, found by flipping bit 3 of the
+// markers when the positive member wins.  Returns the chosen gain.
+template <bool GE>
+__device__ __forceinline__ float razer_w_select(const float* v, const float* e, uint32_t& w0, uint32_t& w1,
+                                                uint32_t& sb)
+{
+    float2 u5 = make_float2(0.0f, 0.0f), s5 = u5, u2 = u5, s2 = u5;
+    uint32_t k5[2], k2[2];
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        const float a0 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i]) - 5.0f), 1.0f));
-        const float a1 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[i + 1]) - 5.0f), 1.0f));
-        const float b0 = razer_gain_w2(v[i]), b1 = razer_gain_w2(v[i + 1]);
-        c5[i] = copysignf(a0, v[i]);
-        c5[i + 1] = copysignf(a1, v[i + 1]);
-        c2[i] = copysignf(b0, v[i]);
-        c2[i + 1] = copysignf(b1, v[i + 1]);
-        u5[i / 2] = make_float2(a0, a1);
-        u2[i / 2] = make_float2(b0, b1);
-        s5[i / 2] = make_float2(c5[i], c5[i + 1]);
-        s2[i / 2] = make_float2(c2[i], c2[i + 1]);
-    }
+    for (int hh = 0; hh < 2; ++hh) {
+        float x5[8], x2[8];
 #pragma unroll
-    for (int k = 4; k > 0; k >>= 1)
-#pragma unroll
-        for (int i = 0; i < k; ++i) {
-            u5[i] = add2_rn(u5[i], u5[i + k]);
-            s5[i] = add2_rn(s5[i], s5[i + k]);
-            u2[i] = add2_rn(u2[i], u2[i + k]);
-            s2[i] = add2_rn(s2[i], s2[i + k]);
+        for (int i = 0; i < 8; i += 2) {
+            const int j = 8 * hh + i;
+            float g0, g1;
+            if (GE) {
+                g0 = __saturatef(__fmaf_rn(2.0f, fabsf(e[j]), -1.0f));
+                g1 = __saturatef(__fmaf_rn(2.0f, fabsf(e[j + 1]), -1.0f));
+            } else {
+                g0 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[j]) - 5.0f), 1.0f));
+                g1 = __saturatef(__fmaf_rn(-2.0f, fabsf(fabsf(v[j + 1]) - 5.0f), 1.0f));
+            }
+            const float h0 = razer_gain_w2(v[j]), h1 = razer_gain_w2(v[j + 1]);
+            const float2 c5 = make_float2(copysignf(g0, v[j]), copysignf(g1, v[j + 1]));
+            const float2 c2 = make_float2(copysignf(h0, v[j]), copysignf(h1, v[j + 1]));
+            u5 = add2_rn(u5, make_float2(g0, g1));
+            s5 = add2_rn(s5, c5);
+            u2 = add2_rn(u2, make_float2(h0, h1));
+            s2 = add2_rn(s2, c2);
+            const float2 m5 = mul2_rn(c5, make_float2(0x1p40f, 0x1p40f));
+            const float2 m2 = mul2_rn(c2, make_float2(0x1p40f, 0x1p40f));
+            x5[i] = m5.x;
+            x5[i + 1] = m5.y;
+            x2[i] = m2.x;
+            x2[i + 1] = m2.y;
         }
-    razer_w_apply(c5, c2, u5[0].x + u5[0].y, s5[0].x + s5[0].y, u2[0].x + u2[0].y, s2[0].x + s2[0].y, w0, w1, sb);
+        k5[hh] = e2m1x8(x5);
+        k2[hh] = e2m1x8(x2);
+    }
+    const float S5 = s5.x + s5.y, S2 = s2.x + s2.y;
+    const float t5 = (u5.x + u5.y) + fabsf(S5), t2 = (u2.x + u2.y) + fabsf(S2);
+    const bool p2 = t2 > t5;
+    const bool neg = (p2 ? S2 : S5) < 0.0f;
+    const uint32_t flip = neg ? 0u : 0x88888888u;
+    w0 = apply_winners(w0, (p2 ? k2[0] : k5[0]) ^ flip);
+    w1 = apply_winners(w1, (p2 ? k2[1] : k5[1]) ^ flip);
+    sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
+    return 0.5f * fmaxf(t5, t2);
 }
 
 // Selection from the scaled values for either RaZeR mode.
 template <int FMT>
 __device__ __forceinline__ void razer_from_v(const float* v, uint32_t& w0, uint32_t& w1, uint32_t& sb)
 {
-    if (FMT == kRW) razer_w_tent(v, w0, w1, sb);
+    if (FMT == kRW) razer_w_select<false>(v, nullptr, w0, w1, sb);
     else razer_tent(v, w0, w1, sb);
 }
 
@@ -595,33 +594,7 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
     w1 = canonical_zero(w1);
     const uint32_t sb0 = sb;
     if (FMT == kRW) {
-        float c5[16], c2[16];
-        float2 u5[8], s5[8], u2[8], s2[8];
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            const float g0 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i]), -1.0f));
-            const float g1 = __saturatef(__fmaf_rn(2.0f, fabsf(e[i + 1]), -1.0f));
-            const float h0 = razer_gain_w2(v[i]), h1 = razer_gain_w2(v[i + 1]);
-            c5[i] = copysignf(g0, v[i]);
-            c5[i + 1] = copysignf(g1, v[i + 1]);
-            c2[i] = copysignf(h0, v[i]);
-            c2[i + 1] = copysignf(h1, v[i + 1]);
-            u5[i / 2] = make_float2(g0, g1);
-            u2[i / 2] = make_float2(h0, h1);
-            s5[i / 2] = make_float2(c5[i], c5[i + 1]);
-            s2[i / 2] = make_float2(c2[i], c2[i + 1]);
-        }
-#pragma unroll
-        for (int k = 4; k > 0; k >>= 1)
-#pragma unroll
-            for (int i = 0; i < k; ++i) {
-                u5[i] = add2_rn(u5[i], u5[i + k]);
-                s5[i] = add2_rn(s5[i], s5[i + k]);
-                u2[i] = add2_rn(u2[i], u2[i + k]);
-                s2[i] = add2_rn(s2[i], s2[i + k]);
-            }
-        sv -= razer_w_apply(c5, c2, u5[0].x + u5[0].y, s5[0].x + s5[0].y, u2[0].x + u2[0].y, s2[0].x + s2[0].y, w0,
-                            w1, sb);
+        sv -= razer_w_select<true>(v, e, w0, w1, sb);
     } else if (RAZER) {
         float cs[16];
         float2 gp[8], sp[8];
@@ -742,13 +715,6 @@ __device__ __forceinline__ void nv_run8(const float* v, int h, NvRun& st)
         }
         st.k2[h] = e2m1x8(x);
     }
-}
-
-// Rewrite the winners flagged in k (nibbles 0xF after the sign flip below) to 0b1000.
-__device__ __forceinline__ uint32_t apply_winners(uint32_t w, uint32_t k)
-{
-    const uint32_t f = k & (k >> 3) & 0x11111111u;
-    return (w & ~(f * 15u)) | (f << 3);
 }
 
 // The block's RaZeR choice from its running sums: -5 only when its gain is
@@ -990,11 +956,22 @@ __device__ __forceinline__ void decode_unit(const uint32_t* cw, const uint32_t* 
 }
 
 // Read a unit's codes and scale bytes (dense layouts).
+// With FP4Q_DEBUG, code_bytes and scale_bytes bound the two reads (an
+// out-of-bounds read is recorded in err and reads zeros instead).
 template <int FMT>
 __device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                                             int64_t code_off, int64_t scale_off, bool full, bool a16, uint32_t* cw,
-                                            uint32_t* sb)
+                                            uint32_t* sb, int64_t code_bytes = 0, int64_t scale_bytes = 0,
+                                            unsigned* err = nullptr)
 {
+    constexpr int B = FMT == kMX ? 32 : 16;
+    if (!in_bounds(code_off, full ? 16 : 8, code_bytes, kSiteCodesLoad, err) ||
+        !in_bounds(scale_off, (FMT != kMX && full) ? 2 : 1, scale_bytes, kSiteScalesLoad, err)) {
+        cw[0] = cw[1] = cw[2] = cw[3] = 0;
+        sb[0] = sb[1] = 0;
+        return;
+    }
+    (void)B;
     const uint8_t* cp = codes + code_off;
     if (full && a16) {
         const uint4 c = ldg_nc_v4(cp);
@@ -1103,11 +1080,12 @@ __device__ __forceinline__ bool pipe_stage_free(const Pipe& p, int64_t j)
     return mbar_wait(p.empty + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
 }
 
-// After a timeout: record it; thread 0 waits (bounded) for the copies it issued
-// that may still be in flight, tiles [from, to) of the schedule.
-__device__ __forceinline__ void pipe_fail(const Pipe& p, int64_t from, int64_t to)
+// After a timeout: record it in the error words `err`; thread 0 waits
+// (bounded) for the copies it issued that may still be in flight, tiles
+// [from, to) of the schedule.
+__device__ __forceinline__ void pipe_fail(const Pipe& p, int64_t from, int64_t to, unsigned* err)
 {
-    if ((threadIdx.x & 31) == 0) atomicOr(&g_device_error, kErrPipelineTimeout);
+    if ((threadIdx.x & 31) == 0) atomicOr(err, kErrPipelineTimeout);
     if (threadIdx.x == 0)
         for (int64_t q = from; q < to; ++q) pipe_acquire(p, q);
 }
@@ -1162,7 +1140,7 @@ __device__ __noinline__ BlockOut nv_block_redo(uint32_t tile, uint32_t r, uint32
 // paths' 1e-3 MSE tolerance).
 template <int FMT, bool ROT, bool SSE, bool FLAT>
 __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, int64_t k, uint8_t* codes,
-                                                uint8_t* scales, const NvScale& nsc, bool mx_ceil = false)
+                                                uint8_t* scales, const NvScale& nsc, bool mx_ceil, unsigned* err)
 {
     const int t = threadIdx.x;
     const bool a16 = FLAT || (tl.cols % 32) == 0;
@@ -1231,14 +1209,18 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
         }
         int64_t co, so;
         unit_offsets<FLAT, FMT>(tl, u, co, so);
-        store_codes(codes + co, cw, u.full, a16);
-        if (FMT == kMX) {
-            scales[so] = (uint8_t)sb0;
-        } else if (u.full && a16) {
-            *reinterpret_cast<unsigned short*>(scales + so) = (unsigned short)(sb0 | (sb1 << 8));
-        } else {
-            scales[so] = (uint8_t)sb0;
-            if (u.full) scales[so + 1] = (uint8_t)sb1;
+        constexpr int B = FMT == kMX ? 32 : 16;
+        const int64_t n = tl.rows * tl.cols;   // the bounds of the debug build's checks
+        if (in_bounds(co, u.full ? 16 : 8, n / 2, kSiteCodesStore, err)) store_codes(codes + co, cw, u.full, a16);
+        if (in_bounds(so, (FMT != kMX && u.full) ? 2 : 1, n / B, kSiteScalesStore, err)) {
+            if (FMT == kMX) {
+                scales[so] = (uint8_t)sb0;
+            } else if (u.full && a16) {
+                *reinterpret_cast<unsigned short*>(scales + so) = (unsigned short)(sb0 | (sb1 << 8));
+            } else {
+                scales[so] = (uint8_t)sb0;
+                if (u.full) scales[so + 1] = (uint8_t)sb1;
+            }
         }
     }
     return acc;

@@ -51,6 +51,7 @@ struct PackArgs {
     uint8_t* sf;
     int64_t rows, cols;
     int64_t rows_pad, nb, nb_pad;   // rows padded to 128, blocks per row, blocks padded to 4
+    unsigned* err;                  // the library's device error words
 };
 
 // Bit 0 of every nibble of w that equals 0b1000.
@@ -71,10 +72,17 @@ __global__ void __launch_bounds__(256) mma_pack_kernel(PackArgs a)
     const int64_t r = i / a.nb_pad, kb = i - r * a.nb_pad;
     const int64_t atoms = a.nb_pad / 4;
     const int64_t off = ((r / 128) * atoms + kb / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4;
+    const int64_t sf_bytes = (a.rows_pad / 128) * (a.nb_pad / 4) * 512, n = a.rows * a.cols;
+    constexpr int P = kRazer<FMT> ? 2 : 1;
+    if (!in_bounds(off, 1, sf_bytes, kSiteSfStore, a.err)) return;
     if (r >= a.rows || kb >= a.nb) {
         a.sf[off] = 0;
         return;
     }
+    if (!in_bounds(r * a.nb + kb, 1, n / 16, kSiteScalesLoad, a.err) ||
+        !in_bounds(r * (a.cols / 2) + 8 * kb, 8, n / 2, kSiteCodesLoad, a.err) ||
+        !in_bounds(r * P * (a.cols / 2) + 8 * kb, P == 1 ? 8 : a.cols / 2 + 8, P * n / 2, kSitePlanesStore, a.err))
+        return;
     const uint32_t sb = a.scales[r * a.nb + kb];
     const uint2 c = *reinterpret_cast<const uint2*>(a.codes + r * (a.cols / 2) + 8 * kb);
     uint32_t mag;
@@ -121,6 +129,7 @@ cudaError_t launch_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t
     a.rows_pad = (rows + 127) / 128 * 128;
     a.nb = cols / 16;
     a.nb_pad = (a.nb + 3) / 4 * 4;
+    if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     const int64_t n = a.rows_pad * a.nb_pad;
     if (n == 0) return cudaSuccess;
     const int64_t blocks = (n + 255) / 256;
@@ -248,6 +257,7 @@ struct GemmArgs {
     uint16_t* y;
     int64_t M, N, K, ldy;
     int32_t a_planes, w_planes;
+    unsigned* err;          // the library's device error words
 };
 
 // Y[m][n] = s_a s_w sum over plane pairs and k of A_p[m][k] W_q[n][k].
@@ -335,7 +345,7 @@ __global__ void __launch_bounds__(tc::kGemmThreads, tc::kCtasPerSm)
             }
         }
         if (!ok) {
-            atomicOr(&g_device_error, kErrPipelineTimeout);
+            atomicOr(g.err, kErrPipelineTimeout);
             for (int64_t q = gi - kStagesG < 0 ? 0 : gi - kStagesG; q < gi; ++q)   // copies still in flight
                 mbar_wait(full((int)(q % kStagesG)), (uint32_t)((q / kStagesG) & 1));
         }
@@ -373,7 +383,7 @@ __global__ void __launch_bounds__(tc::kGemmThreads, tc::kCtasPerSm)
             if (ok) tc::commit_to(acc_full);   // arrives when the tile's MMAs have completed
         }
         if (!ok) {
-            atomicOr(&g_device_error, kErrPipelineTimeout);
+            atomicOr(g.err, kErrPipelineTimeout);
             tc::commit_to(drain);              // wait (bounded) for the MMAs issued so far
             mbar_wait(drain, 0u);
         }
@@ -384,7 +394,7 @@ __global__ void __launch_bounds__(tc::kGemmThreads, tc::kCtasPerSm)
         const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);
         for (int64_t j = 0; j < my_tiles; ++j) {
             if (!mbar_wait(acc_full, (uint32_t)(j & 1))) {
-                if (lane == 0) atomicOr(&g_device_error, kErrPipelineTimeout);
+                if (lane == 0) atomicOr(g.err, kErrPipelineTimeout);
                 break;
             }
             tc::fence_after_sync();
@@ -396,7 +406,8 @@ __global__ void __launch_bounds__(tc::kGemmThreads, tc::kCtasPerSm)
                 if (n0 + c >= g.N) break;   // uniform across the warp
                 float v[32];
                 tc::tmem_ld32(trow + (uint32_t)c, v);
-                if (m < g.M) {
+                if (m < g.M && in_bounds(2 * (m * g.ldy + n0 + c), 2 * (g.N - n0 - c < 32 ? g.N - n0 - c : 32),
+                                         2 * ((g.M - 1) * g.ldy + g.N), kSiteGemmStore, g.err)) {
                     uint16_t* yrow = g.y + m * g.ldy + n0 + c;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -461,6 +472,7 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
     g.ldy = ldy;
     g.a_planes = a_np;
     g.w_planes = w_np;
+    if ((g.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
     if (tiles >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const int64_t cap = (int64_t)kCtasPerSm * sm_count();           // persistent: two CTAs per SM
@@ -470,17 +482,6 @@ cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a
     if (e != cudaSuccess) return e;
     gemm_w4a4_kernel<<<(unsigned)grid, kGemmThreads, kGemmSmem, st>>>(amap, wmap, g);
     return cudaGetLastError();
-}
-
-cudaError_t read_gemm_device_errors(unsigned int* bits, bool clear)
-{
-    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    if (clear) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-    }
-    return e;
 }
 
 }  // namespace fp4q

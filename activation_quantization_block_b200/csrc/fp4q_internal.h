@@ -56,10 +56,13 @@ cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t*
 cudaError_t launch_sse_finalize(const double* partials, int n, double count, double* mse,
                                 cudaStream_t st);
 
-// Copy the device error word of the current device to *bits (synchronous);
-// clear it afterwards when asked.  One word per kernel translation unit.
-cudaError_t read_device_errors(unsigned int* bits, bool clear);
-cudaError_t read_batch_device_errors(unsigned int* bits, bool clear);
+// The library's device error words in the calling thread's current CUDA
+// context, one array that every kernel records into: [0] error bits
+// (FP4Q_DEVICE_ERROR_*), [1] the site of the first out-of-bounds access a
+// FP4Q_DEBUG build found, [2] and [3] its byte offset (low and high halves).
+// Null when the address cannot be had (the launchers then fail the call).
+constexpr int kErrorWords = 4;
+unsigned int* device_error_words();
 
 // Tensor-core operand form and the W4A4 product (fp4q_gemm.cu).
 int64_t mma_sf_bytes(int64_t rows, int64_t cols);
@@ -68,11 +71,9 @@ cudaError_t launch_mma_pack(const uint8_t* codes, const uint8_t* scales, int64_t
 cudaError_t launch_gemm_w4a4(const uint8_t* a_planes, const uint8_t* a_sf, int a_np, const float* a_scale,
                              const uint8_t* w_planes, const uint8_t* w_sf, int w_np, const float* w_scale, int64_t M,
                              int64_t N, int64_t K, uint16_t* y, int64_t ldy, cudaStream_t st);
-cudaError_t read_gemm_device_errors(unsigned int* bits, bool clear);
 
 // Failure-path self-test (fp4q_selftest.cu).
 cudaError_t launch_timeout_selftest(cudaStream_t st);
-cudaError_t read_selftest_device_errors(unsigned int* bits, bool clear);
 
 // Sparse outlier separation (fp4q_outliers.cu).
 int64_t outlier_capacity(int64_t cols, double max_frac);

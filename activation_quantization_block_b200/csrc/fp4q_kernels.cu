@@ -47,6 +47,7 @@ namespace fp4q {
 struct AmaxArgs {
     Tiles tl;
     float* partials;
+    unsigned* err;          // the library's device error words
 };
 
 // Q0: per-CTA maxima of |x| (of |H x| when rotating).
@@ -64,21 +65,22 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ 
     float m = 0.0f;
     for (int64_t j = 0; j < sc.mine; ++j) {
         if (!pipe_acquire(p, j)) {
-            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine, a.err);
             break;
         }
         m = fmaxf(m, amax_tile<ROT>(p.tiles + (uint32_t)(j % kStages) * kTileBytes));
         pipe_release(p, j);
         if (t == 0 && j + kStages < sc.mine) {
             if (!pipe_stage_free(p, j)) {
-                pipe_fail(p, j + 1, j + kStages);
+                pipe_fail(p, j + 1, j + kStages, a.err);
                 break;
             }
             pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
         }
     }
     m = block_max(m, shf);
-    if (t == 0) a.partials[blockIdx.x] = m;
+    if (t == 0 && in_bounds(4 * (int64_t)blockIdx.x, 4, 4 * (int64_t)kMaxPartials, kSiteAmaxPartialStore, a.err))
+        a.partials[blockIdx.x] = m;
 }
 
 struct QuantArgs {
@@ -92,6 +94,7 @@ struct QuantArgs {
     int reverse;
     int mx_ceil;
     double* sse_partials;
+    unsigned* err;          // the library's device error words
 };
 
 // Q1-Q6: rotate, block scale, encode, RaZeR select, pack, store, SSE partials.
@@ -118,7 +121,9 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(cons
             s_t = *a.tensor_scale;
         } else {
             float m = 0.0f;
-            for (int i = t; i < a.n_amax; i += kThreads) m = fmaxf(m, a.amax_partials[i]);
+            for (int i = t; i < a.n_amax; i += kThreads)
+                if (in_bounds(4 * (int64_t)i, 4, 4 * (int64_t)kMaxPartials, kSiteAmaxPartialLoad, a.err))
+                    m = fmaxf(m, a.amax_partials[i]);
             m = block_max(m, shf);
             s_t = tensor_scale_of<FMT>(m);
             if (blockIdx.x == 0 && t == 0) *a.tensor_scale = s_t;
@@ -131,15 +136,16 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(cons
     double acc = 0.0;
     for (int64_t j = 0; j < sc.mine; ++j) {
         if (!pipe_acquire(p, j)) {
-            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine, a.err);
             break;
         }
         const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
-        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc, a.mx_ceil != 0);
+        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc, a.mx_ceil != 0,
+                                                  a.err);
         pipe_release(p, j);
         if (t == 0 && j + kStages < sc.mine) {
             if (!pipe_stage_free(p, j)) {
-                pipe_fail(p, j + 1, j + kStages);
+                pipe_fail(p, j + 1, j + kStages, a.err);
                 break;
             }
             pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
@@ -147,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(cons
     }
     if (SSE) {
         acc = block_sum(acc, shd);
-        if (t == 0) a.sse_partials[blockIdx.x] = acc;
+        if (t == 0 && in_bounds(8 * (int64_t)blockIdx.x, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialStore, a.err))
+            a.sse_partials[blockIdx.x] = acc;
     }
 }
 
@@ -157,6 +164,7 @@ struct ErrArgs {
     const uint8_t* scales;
     const float* tensor_scale;
     double* sse_partials;
+    unsigned* err;          // the library's device error words
 };
 
 // Q8: squared error of a given encoding against x.
@@ -181,10 +189,11 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) error_kernel(const _
         if (u.valid) {
             int64_t co, so;
             unit_offsets<FLAT, FMT>(a.tl, u, co, so);
-            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
+            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb, a.tl.rows * a.tl.cols / 2,
+                             a.tl.rows * a.tl.cols / (FMT == kMX ? 32 : 16), a.err);
         }
         if (!pipe_acquire(p, j)) {
-            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine);
+            pipe_fail(p, j, j + kStages < sc.mine ? j + kStages : sc.mine, a.err);
             break;
         }
         if (u.valid) {
@@ -205,14 +214,15 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) error_kernel(const _
         pipe_release(p, j);
         if (t == 0 && j + kStages < sc.mine) {
             if (!pipe_stage_free(p, j)) {
-                pipe_fail(p, j + 1, j + kStages);
+                pipe_fail(p, j + 1, j + kStages, a.err);
                 break;
             }
             pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
         }
     }
     acc = block_sum(acc, shd);
-    if (t == 0) a.sse_partials[blockIdx.x] = acc;
+    if (t == 0 && in_bounds(8 * (int64_t)blockIdx.x, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialStore, a.err))
+        a.sse_partials[blockIdx.x] = acc;
 }
 
 struct DeqArgs {
@@ -220,6 +230,7 @@ struct DeqArgs {
     const uint8_t* codes;
     const uint8_t* scales;
     const float* tensor_scale;
+    unsigned* err;          // the library's device error words
 };
 
 // Q7: reconstruct bf16 tiles in shared memory (the swizzled layout of the
@@ -244,7 +255,8 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const __grid_const
         if (u.valid) {
             int64_t co, so;
             unit_offsets<FLAT, FMT>(a.tl, u, co, so);
-            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
+            load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb, a.tl.rows * a.tl.cols / 2,
+                             a.tl.rows * a.tl.cols / (FMT == kMX ? 32 : 16), a.err);
         }
     }
     for (int64_t j = 0; j < sc.mine; ++j) {
@@ -256,7 +268,8 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const __grid_const
             if (u.valid) {
                 int64_t co, so;
                 unit_offsets<FLAT, FMT>(a.tl, u, co, so);
-                load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb);
+                load_packed<FMT>(a.codes, a.scales, co, so, u.full, a16, cw, sb, a.tl.rows * a.tl.cols / 2,
+                             a.tl.rows * a.tl.cols / (FMT == kMX ? 32 : 16), a.err);
             }
         }
         uint32_t o[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
@@ -288,12 +301,13 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const __grid_const
 
 // Sum n fp64 partials in a fixed order and write sum / count.
 __global__ void __launch_bounds__(kThreads) sse_finalize_kernel(const double* partials, int n, double count,
-                                                                double* mse)
+                                                                double* mse, unsigned* err)
 {
     __shared__ double sh[kThreads];
     pdl_wait();
     double s = 0.0;
-    for (int i = threadIdx.x; i < n; i += kThreads) s += partials[i];
+    for (int i = threadIdx.x; i < n; i += kThreads)
+        if (in_bounds(8 * (int64_t)i, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialLoad, err)) s += partials[i];
     sh[threadIdx.x] = s;
     __syncthreads();
     for (int o = kThreads / 2; o > 0; o >>= 1) {
@@ -314,6 +328,7 @@ cudaError_t launch_amax(const uint16_t* x, const Geometry& g, int rotate, float*
     AmaxArgs a;
     if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
     a.partials = partials;
+    if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     auto go = [&](auto kernel) {
         const int grid = grid_for(kernel, kPipeSmemBytes, a.tl.count);
         if (grid_out) *grid_out = grid;
@@ -346,6 +361,7 @@ cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int r
     CUtensorMap map;
     QuantArgs a;
     if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     a.codes = codes;
     a.scales = scales;
     a.tensor_scale = tensor_scale;
@@ -389,6 +405,7 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
     CUtensorMap map;
     DeqArgs a;
     if (!make_view(y, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     a.codes = codes;
     a.scales = scales;
     a.tensor_scale = tensor_scale;
@@ -423,6 +440,7 @@ cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t*
     CUtensorMap map;
     ErrArgs a;
     if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     a.codes = codes;
     a.scales = scales;
     a.tensor_scale = tensor_scale;
@@ -442,20 +460,11 @@ cudaError_t launch_error(const uint16_t* x, const uint8_t* codes, const uint8_t*
 
 cudaError_t launch_sse_finalize(const double* partials, int n, double count, double* mse, cudaStream_t st)
 {
-    return launch(sse_finalize_kernel, 1, 0, true, st, partials, n, count, mse);
+    unsigned* err = device_error_words();
+    if (err == nullptr) return cudaErrorInvalidSymbol;
+    return launch(sse_finalize_kernel, 1, 0, true, st, partials, n, count, mse, err);
 }
 
 int64_t view_tiles(const Geometry& g) { return view_tile_count(g); }
-
-cudaError_t read_device_errors(unsigned int* bits, bool clear)
-{
-    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    if (clear) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-    }
-    return e;
-}
 
 }  // namespace fp4q

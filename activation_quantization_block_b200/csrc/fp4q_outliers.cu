@@ -43,6 +43,8 @@ struct OutlierArgs {
     int32_t* out_count;
     int64_t ldx, ldb, cols, cap;
     double k;
+    int64_t rows;
+    unsigned* err;          // the library's device error words
 };
 
 // Sum over the CTA in a fixed order, result in every thread.
@@ -190,6 +192,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
     const int t = threadIdx.x;
     const int64_t n = a.cols;
     const uint32_t row = smem_u32(srow_raw);
+    if (!in_bounds(2 * r * a.ldx, 2 * n, 2 * ((a.rows - 1) * a.ldx + n), kSiteOutlierRowLoad, a.err)) return;
     copy_row(srow_raw, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n / 8, t, kOutThreads);
     __syncthreads();
 
@@ -217,6 +220,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
     };
     const uint16_t mub = f64_to_bf16_rn(mu);
     uint16_t* brow = a.bulk + r * a.ldb;
+    const int64_t bulk_bytes = 2 * ((a.rows - 1) * a.ldb + n);   // the debug build's bound of the bulk
     // d > t in fp32 outside a band covering the fp32 roundings of mu, t and d
     // (2^-20 of |mu| + t), in fp64 inside it; slots past the capacity are not written
     auto compact = [&](double t, long long tie_need, bool none) -> long long {
@@ -240,7 +244,8 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
                 for (int i = 0; i < 8; ++i) dm = fmaxf(dm, fabsf(v[i] - mu32));
             }
             if (__syncthreads_and(none || dm - t32 < -band)) {
-                if (in) *reinterpret_cast<uint4*>(brow + j) = w;
+                if (in && in_bounds(2 * (r * a.ldb + j), 16, bulk_bytes, kSiteBulkStore, a.err))
+                    *reinterpret_cast<uint4*>(brow + j) = w;
                 continue;
             }
             uint32_t gmask = 0, emask = 0;
@@ -276,14 +281,16 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
                     if (omask & (1u << i)) {
                         const uint32_t sh = (i & 1) ? 16u : 0u;
                         u[i >> 1] = (u[i >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
-                        if (slot < a.cap) {
+                        if (slot < a.cap &&
+                            in_bounds(2 * (r * a.cap + slot), 2, 2 * a.rows * a.cap, kSiteSlotStore, a.err)) {
                             a.out_cols[r * a.cap + slot] = (uint16_t)(j + i);
                             a.out_vals[r * a.cap + slot] =
                                 __half_as_ushort(__float2half_rn(fminf(fmaxf(v[i], -65504.0f), 65504.0f)));
                         }
                         ++slot;
                     }
-                *reinterpret_cast<uint4*>(brow + j) = make_uint4(u[0], u[1], u[2], u[3]);
+                if (in_bounds(2 * (r * a.ldb + j), 16, bulk_bytes, kSiteBulkStore, a.err))
+                    *reinterpret_cast<uint4*>(brow + j) = make_uint4(u[0], u[1], u[2], u[3]);
             }
             done += tot;
         }
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kOutThreads) outlier_rows_kernel(OutlierArgs a
         thr = __longlong_as_double((long long)lo);
         total = compact(thr, a.cap - count_where([&](double d) { return d > thr; }), false);
     }
-    if (t == 0) a.out_count[r] = (int32_t)total;
+    if (t == 0 && in_bounds(4 * r, 4, 4 * a.rows, kSiteCountStore, a.err)) a.out_count[r] = (int32_t)total;
 }
 
 // The same, one warp per row (rows of at most 8192 elements): warp w of CTA b
@@ -347,6 +354,7 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
     const int64_t n = a.cols, n8 = n / 8;
     uint4* srow = srows_raw + (int64_t)w * n8;
     const uint32_t row = smem_u32(srow);
+    if (!in_bounds(2 * r * a.ldx, 2 * n, 2 * ((rows - 1) * a.ldx + n), kSiteOutlierRowLoad, a.err)) return;
     copy_row(srow, reinterpret_cast<const uint4*>(a.x + r * a.ldx), n8, lane, 32);
     __syncwarp();
 
@@ -372,6 +380,7 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
     };
     const uint16_t mub = f64_to_bf16_rn(mu);
     uint16_t* brow = a.bulk + r * a.ldb;
+    const int64_t bulk_bytes = 2 * ((a.rows - 1) * a.ldb + n);   // the debug build's bound of the bulk
     // One pass: bulk row and outlier slots for threshold t (and, when tie_need > 0,
     // the first tie_need elements with d == t).  d > t is decided in fp32 where
     // |d32 - t32| exceeds a band covering the fp32 roundings of mu, t and d (each
@@ -398,7 +407,8 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
                 for (int q = 0; q < 8; ++q) dm = fmaxf(dm, fabsf(v[q] - mu32));
             }
             if (__all_sync(0xFFFFFFFFu, none || dm - t32 < -band)) {
-                if (in) *reinterpret_cast<uint4*>(brow + 8 * i) = wd;
+                if (in && in_bounds(2 * (r * a.ldb + 8 * i), 16, bulk_bytes, kSiteBulkStore, a.err))
+                    *reinterpret_cast<uint4*>(brow + 8 * i) = wd;
                 continue;
             }
             uint32_t gmask = 0, emask = 0;
@@ -434,14 +444,16 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
                     if (omask & (1u << q)) {
                         const uint32_t sh = (q & 1) ? 16u : 0u;
                         u[q >> 1] = (u[q >> 1] & ~(0xFFFFu << sh)) | ((uint32_t)mub << sh);
-                        if (slot < a.cap) {
+                        if (slot < a.cap &&
+                            in_bounds(2 * (r * a.cap + slot), 2, 2 * a.rows * a.cap, kSiteSlotStore, a.err)) {
                             a.out_cols[r * a.cap + slot] = (uint16_t)(8 * i + q);
                             a.out_vals[r * a.cap + slot] =
                                 __half_as_ushort(__float2half_rn(fminf(fmaxf(v[q], -65504.0f), 65504.0f)));
                         }
                         ++slot;
                     }
-                *reinterpret_cast<uint4*>(brow + 8 * i) = make_uint4(u[0], u[1], u[2], u[3]);
+                if (in_bounds(2 * (r * a.ldb + 8 * i), 16, bulk_bytes, kSiteBulkStore, a.err))
+                    *reinterpret_cast<uint4*>(brow + 8 * i) = make_uint4(u[0], u[1], u[2], u[3]);
             }
             done += tot;
         }
@@ -462,7 +474,7 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) outlier_rows_warp_kernel(Out
         thr = __longlong_as_double((long long)lo);
         total = compact(thr, a.cap - count_where([&](double d) { return d > thr; }), false);
     }
-    if (lane == 0) a.out_count[r] = (int32_t)total;
+    if (lane == 0 && in_bounds(4 * r, 4, 4 * a.rows, kSiteCountStore, a.err)) a.out_count[r] = (int32_t)total;
 }
 
 struct ScatterArgs {
@@ -471,6 +483,7 @@ struct ScatterArgs {
     const int32_t* out_count;
     uint16_t* y;
     int64_t rows, cols, cap, ldy;
+    unsigned* err;          // the library's device error words
 };
 
 // One thread per (row, slot): the slot's fp16 value, as bf16, to its column.
@@ -485,6 +498,7 @@ __global__ void __launch_bounds__(256) outlier_scatter_kernel(ScatterArgs a)
     if (s >= a.out_count[r]) return;
     const int64_t col = a.out_cols[i];
     if (col >= a.cols) return;
+    if (!in_bounds(2 * (r * a.ldy + col), 2, 2 * ((a.rows - 1) * a.ldy + a.cols), kSiteScatterStore, a.err)) return;
     const float v = __half2float(__ushort_as_half(a.out_vals[i]));
     a.y[r * a.ldy + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
@@ -498,7 +512,8 @@ cudaError_t launch_separate_outliers(const uint16_t* x, int64_t rows, int64_t co
                                      int32_t* out_count, cudaStream_t st)
 {
     if (rows == 0) return cudaSuccess;
-    OutlierArgs a{x, bulk, out_cols, out_vals, out_count, ldx, ldb, cols, cap, k};
+    OutlierArgs a{x, bulk, out_cols, out_vals, out_count, ldx, ldb, cols, cap, k, rows, device_error_words()};
+    if (a.err == nullptr) return cudaErrorInvalidSymbol;
     if (cols <= 8192) {   // one warp per row, at most 48 KB of rows per CTA
         int64_t rpc = (48 * 1024) / (cols * 2);
         rpc = rpc < 1 ? 1 : (rpc > kRowsPerCta ? kRowsPerCta : rpc);
@@ -524,7 +539,8 @@ cudaError_t launch_scatter_outliers(const uint16_t* out_cols, const uint16_t* ou
     if (n == 0) return cudaSuccess;
     const int64_t blocks = (n + 255) / 256;
     if (blocks >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-    ScatterArgs a{out_cols, out_vals, out_count, y, rows, cols, cap, ldy};
+    ScatterArgs a{out_cols, out_vals, out_count, y, rows, cols, cap, ldy, device_error_words()};
+    if (a.err == nullptr) return cudaErrorInvalidSymbol;
     outlier_scatter_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
     return cudaGetLastError();
 }

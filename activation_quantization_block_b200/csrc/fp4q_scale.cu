@@ -25,12 +25,15 @@ namespace {
 
 // One CTA: s_t from the n per-CTA maxima the absmax pass wrote.
 template <int FMT>
-__global__ void __launch_bounds__(kThreads) tensor_scale_kernel(const float* partials, int n, float* tensor_scale)
+__global__ void __launch_bounds__(kThreads) tensor_scale_kernel(const float* partials, int n, float* tensor_scale,
+                                                                unsigned* err)
 {
     __shared__ float sh[32];
     pdl_wait();
     float m = 0.0f;
-    for (int i = threadIdx.x; i < n; i += kThreads) m = fmaxf(m, partials[i]);
+    for (int i = threadIdx.x; i < n; i += kThreads)
+        if (in_bounds(4 * (int64_t)i, 4, 4 * (int64_t)kMaxPartials, kSiteAmaxPartialLoad, err))
+            m = fmaxf(m, partials[i]);
     m = block_max(m, sh);
     if (threadIdx.x == 0) *tensor_scale = tensor_scale_of<FMT>(m);
 }
@@ -39,10 +42,12 @@ __global__ void __launch_bounds__(kThreads) tensor_scale_kernel(const float* par
 
 cudaError_t launch_tensor_scale(const float* partials, int n, int fmt, float* tensor_scale, cudaStream_t st)
 {
+    unsigned* err = device_error_words();
+    if (err == nullptr) return cudaErrorInvalidSymbol;
     switch (fmt) {
-        case kNV: return launch(tensor_scale_kernel<kNV>, 1, 0, true, st, partials, n, tensor_scale);
-        case kRZ: return launch(tensor_scale_kernel<kRZ>, 1, 0, true, st, partials, n, tensor_scale);
-        case kRW: return launch(tensor_scale_kernel<kRW>, 1, 0, true, st, partials, n, tensor_scale);
+        case kNV: return launch(tensor_scale_kernel<kNV>, 1, 0, true, st, partials, n, tensor_scale, err);
+        case kRZ: return launch(tensor_scale_kernel<kRZ>, 1, 0, true, st, partials, n, tensor_scale, err);
+        case kRW: return launch(tensor_scale_kernel<kRW>, 1, 0, true, st, partials, n, tensor_scale, err);
         default: return cudaErrorInvalidValue;
     }
 }

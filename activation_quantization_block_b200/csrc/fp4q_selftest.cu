@@ -17,7 +17,7 @@ namespace fp4q {
 
 namespace {
 
-__global__ void timeout_selftest_kernel()
+__global__ void timeout_selftest_kernel(unsigned* err)
 {
     __shared__ uint64_t bar;
     const uint32_t b = smem_u32(&bar);
@@ -25,7 +25,7 @@ __global__ void timeout_selftest_kernel()
         mbar_init(b, 1);
         mbar_init_fence();
         mbar_arm(b, 16u);                  // 16 bytes expected; no copy is issued
-        if (!mbar_wait(b, 0u)) atomicOr(&g_device_error, kErrPipelineTimeout);
+        if (!mbar_wait(b, 0u)) atomicOr(err, kErrPipelineTimeout);
     }
 }
 
@@ -33,19 +33,10 @@ __global__ void timeout_selftest_kernel()
 
 cudaError_t launch_timeout_selftest(cudaStream_t st)
 {
-    timeout_selftest_kernel<<<1, 32, 0, st>>>();
+    unsigned* err = device_error_words();
+    if (err == nullptr) return cudaErrorInvalidSymbol;
+    timeout_selftest_kernel<<<1, 32, 0, st>>>(err);
     return cudaGetLastError();
-}
-
-cudaError_t read_selftest_device_errors(unsigned int* bits, bool clear)
-{
-    cudaError_t e = cudaMemcpyFromSymbol(bits, g_device_error, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    if (clear) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-    }
-    return e;
 }
 
 }  // namespace fp4q

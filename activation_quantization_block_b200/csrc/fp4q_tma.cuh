@@ -32,6 +32,36 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Bits of the device error word.
 constexpr unsigned kErrPipelineTimeout = 1u;
+constexpr unsigned kErrOutOfBounds = 2u;
+
+#ifndef FP4Q_DEBUG
+#define FP4Q_DEBUG 0
+#endif
+
+// Bounds check of a global access of `len` bytes at byte offset `off` into a
+// buffer of `extent` bytes, done only in builds with FP4Q_DEBUG (otherwise
+// always true, and compiled away).  An access outside the buffer sets
+// kErrOutOfBounds in the error words `err`; the first such access also leaves
+// its site (a number naming the access) and its offset; the caller skips it.
+__device__ __forceinline__ bool in_bounds(int64_t off, int64_t len, int64_t extent, unsigned site, unsigned* err)
+{
+    if (!FP4Q_DEBUG) return true;
+    if (off >= 0 && len >= 0 && off <= extent - len) return true;
+    atomicOr(err, kErrOutOfBounds);
+    if (atomicCAS(err + 1, 0u, site) == 0u) {
+        atomicExch(err + 2, (unsigned)((uint64_t)off & 0xFFFFFFFFu));
+        atomicExch(err + 3, (unsigned)((uint64_t)off >> 32));
+    }
+    return false;
+}
+
+// Sites of the checked accesses (fp4q_device_error_site).
+enum : unsigned {
+    kSiteCodesStore = 1, kSiteScalesStore, kSiteAmaxPartialStore, kSiteSsePartialStore, kSiteAmaxPartialLoad,
+    kSiteSsePartialLoad, kSiteCodesLoad, kSiteScalesLoad, kSiteScalarStore, kSiteScalarLoad, kSiteOutlierRowLoad,
+    kSiteBulkStore, kSiteSlotStore, kSiteCountStore, kSiteScatterStore, kSitePlanesStore, kSiteSfStore,
+    kSiteGemmStore, kSiteCountLoad, kSiteSlotLoad
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {

@@ -11,6 +11,7 @@ missing library is an error.
 from __future__ import annotations
 
 import ctypes
+import os
 from typing import NamedTuple
 
 import torch
@@ -34,7 +35,7 @@ ABI_SYMBOLS = ("fp4q_abi_version", "fp4q_status_string", "fp4q_workspace_size",
                "fp4q_device_errors", "fp4q_batch_workspace_size", "fp4q_quantize_batch",
                "fp4q_mma_planes", "fp4q_mma_sf_bytes", "fp4q_mma_pack", "fp4q_gemm",
                "fp4q_outlier_capacity", "fp4q_separate_outliers", "fp4q_scatter_outliers",
-               "fp4q_selftest_timeout", "fp4q_tensor_scale")
+               "fp4q_selftest_timeout", "fp4q_tensor_scale", "fp4q_device_error_site", "fp4q_debug_build")
 
 
 class TensorDesc(ctypes.Structure):
@@ -53,15 +54,25 @@ class Fp4qError(RuntimeError):
 _lib = None
 
 
+# FP4Q_DEBUG_LIBRARY=1 in the environment loads the bounds-checking build
+# (libfp4q_debug.so) in place of libfp4q.so.
+DEBUG_ENV = "FP4Q_DEBUG_LIBRARY"
+
+
+def _want_debug() -> bool:
+    return os.environ.get(DEBUG_ENV, "") not in ("", "0")
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.DEBUG_LIB if _want_debug() else _build.LIB
 
 
 def lib() -> ctypes.CDLL:
-    """Load (building first if the sources are newer) the in-tree libfp4q.so."""
+    """Load (building first if the sources are newer) the in-tree libfp4q.so, or with
+    FP4Q_DEBUG_LIBRARY=1 the bounds-checking libfp4q_debug.so."""
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(_build.build())
+        L = ctypes.CDLL(_build.build_debug() if _want_debug() else _build.build())
         vp, i64, i32, u32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
         L.fp4q_abi_version.argtypes = []
         L.fp4q_abi_version.restype = i32
@@ -77,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.fp4q_error.restype = i32
         L.fp4q_quantize_noalloc.argtypes = [vp, i64, i64, i64, i32, i32, u32, vp, vp, vp, vp, vp]
         L.fp4q_quantize_noalloc.restype = i32
+        L.fp4q_device_error_site.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint64)]
+        L.fp4q_device_error_site.restype = i32
+        L.fp4q_debug_build.argtypes = []
+        L.fp4q_debug_build.restype = i32
         L.fp4q_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         L.fp4q_device_errors.restype = i32
         L.fp4q_batch_workspace_size.argtypes = [i32, ctypes.POINTER(TensorDesc), i32, i32]
@@ -177,6 +192,18 @@ def fp4q_device_errors(clear: bool = False) -> tuple[int, int]:
     v = ctypes.c_uint32(0)
     st = lib().fp4q_device_errors(ctypes.byref(v), int(clear))
     return st, v.value
+
+
+def fp4q_device_error_site() -> tuple[int, int, int]:
+    """(status, site, byte offset) of the first out-of-bounds access a debug build found."""
+    site, off = ctypes.c_uint32(0), ctypes.c_uint64(0)
+    st = lib().fp4q_device_error_site(ctypes.byref(site), ctypes.byref(off))
+    return st, site.value, off.value
+
+
+def fp4q_debug_build() -> int:
+    """1 when the loaded library is the bounds-checking build."""
+    return lib().fp4q_debug_build()
 
 
 def _descs(descs):

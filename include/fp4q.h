@@ -95,7 +95,7 @@
 extern "C" {
 #endif
 
-#define FP4Q_ABI_VERSION 3
+#define FP4Q_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define FP4Q_API __attribute__((visibility("default")))
@@ -236,16 +236,32 @@ FP4Q_API fp4q_status_t fp4q_quantize_batch(int count, const fp4q_tensor_desc_t* 
 
 /* Bits of the device error word (fp4q_device_errors). */
 #define FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT 0x1u
+#define FP4Q_DEVICE_ERROR_OUT_OF_BOUNDS 0x2u   /* only a library built with FP4Q_DEBUG sets it */
 
-/* Read the device error word of the current device into *bits.
- * Every wait of a kernel in this library on its own copy pipeline gives up
- * after 2 s.  A CTA that gives up sets FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT in a
- * per-device word, waits (bounded) for its copies in flight and returns, so
- * the outputs of that call are incomplete.  This call is synchronous: it waits
- * for the device, copies the word to the host and, when clear != 0, resets it.
- * Returns FP4Q_ERROR_INVALID_VALUE for a null bits, FP4Q_ERROR_CUDA if the copy
- * fails. */
+/* Read the device error word of the current CUDA context into *bits.  Every
+ * kernel of the library records into one word per context.
+ *  - Every wait of a kernel on its own copy pipeline gives up after 2 s.  A
+ *    CTA that gives up sets FP4Q_DEVICE_ERROR_PIPELINE_TIMEOUT, waits (bounded)
+ *    for its copies in flight and returns, so the outputs of that call are
+ *    incomplete.
+ *  - A library built with FP4Q_DEBUG checks every global-memory access its
+ *    kernels make by hand (TMA copies are bounded by their tensor maps) against
+ *    the extent its arguments give the buffer.  An access outside it is
+ *    skipped and sets FP4Q_DEVICE_ERROR_OUT_OF_BOUNDS; the first one's site
+ *    and offset are kept (fp4q_device_error_site).
+ * This call is synchronous: it waits for the device, copies the word to the
+ * host and, when clear != 0, resets the word and the kept site.  Returns
+ * FP4Q_ERROR_INVALID_VALUE for a null bits, FP4Q_ERROR_CUDA if the copy fails. */
 FP4Q_API fp4q_status_t fp4q_device_errors(uint32_t* bits, int clear);
+
+/* The first out-of-bounds access a FP4Q_DEBUG library found since the word was
+ * last cleared: *site names the access (a number fixed in the source, 0 when
+ * there was none) and *offset is its byte offset into the buffer.  Synchronous,
+ * like fp4q_device_errors; both pointers must be non-null. */
+FP4Q_API fp4q_status_t fp4q_device_error_site(uint32_t* site, uint64_t* offset);
+
+/* 1 when the loaded library was built with FP4Q_DEBUG, else 0. */
+FP4Q_API int fp4q_debug_build(void);
 
 /* Exercise the failure path above: one kernel arms a pipeline barrier that no
  * copy will complete and waits on it with the library's bounded wait.  After

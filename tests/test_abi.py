@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_status_strings_workspace():
-    assert fp4q.fp4q_abi_version() == 3
+    assert fp4q.fp4q_abi_version() == 4
     for code in range(7):
         assert fp4q.fp4q_status_string(code)
     assert fp4q.fp4q_status_string(99) == "unknown status"
@@ -378,3 +378,20 @@ def test_a_plain_c_program_links_and_calls_the_abi(tmp_path):
                     lib, f"-Wl,-rpath,{os.path.dirname(lib)}"], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_the_bounds_checking_twin_loads_and_says_so():
+    """libfp4q_debug.so (FP4Q_DEBUG=1) exports the same C ABI and reports the debug build; the
+    release library does not.  Loading needs no GPU."""
+    import ctypes
+
+    from activation_quantization_block_b200 import _build
+    dbg = ctypes.CDLL(_build.build_debug())
+    rel = ctypes.CDLL(_build.build())
+    for L in (dbg, rel):
+        L.fp4q_debug_build.restype = ctypes.c_int
+        L.fp4q_abi_version.restype = ctypes.c_int
+        assert L.fp4q_abi_version() == 4
+        for name in fp4q.ABI_SYMBOLS:
+            assert hasattr(L, name), name
+    assert dbg.fp4q_debug_build() == 1 and rel.fp4q_debug_build() == 0
