@@ -84,22 +84,38 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
     const int64_t mine = my_q + my_a;
     // Thread 0 walks the items in order: before item jj come k = floor(jj my_q /
     // mine) quantize items, stepped without a division (rem = jj my_q - k mine,
-    // in [0, mine); my_q <= mine, so one step adds at most one).
-    // The cursor lives in shared memory: only thread 0 uses it, and kept in
-    // registers across the tile loop it would cost the encoder registers.
-    __shared__ int64_t cur_k, cur_rem;
-    if (t == 0) cur_k = cur_rem = 0;
+    // in [0, mine); my_q <= mine, so one step adds at most one).  Only thread 0
+    // uses the cursor.  Kept in shared memory it costs the encoder no registers;
+    // kept in registers it saves thread 0 a shared-memory round trip per refill.
+    // The weight mode measured faster with registers, the other formats with
+    // shared memory.
+    constexpr bool kCursorInRegs = FMT == kRW;
+    __shared__ int64_t cur_k_sh, cur_rem_sh;
+    int cur_k_r = 0, cur_rem_r = 0;   // fits: a tensor in device memory has fewer than 2^24 tiles
+    if (!kCursorInRegs && t == 0) cur_k_sh = cur_rem_sh = 0;
     auto next_item = [&](int64_t jj, bool& is_q, int64_t& tile) {
-        const int64_t k0 = cur_k;
-        int64_t k1 = k0, rem1 = cur_rem + my_q;
-        if (rem1 >= mine) {
-            rem1 -= mine;
-            ++k1;
+        int64_t k0, k1;
+        if constexpr (kCursorInRegs) {
+            k0 = cur_k_r;
+            cur_rem_r += (int)my_q;
+            if (cur_rem_r >= (int)mine) {
+                cur_rem_r -= (int)mine;
+                ++cur_k_r;
+            }
+            k1 = cur_k_r;
+        } else {
+            k0 = cur_k_sh;
+            k1 = k0;
+            int64_t rem1 = cur_rem_sh + my_q;
+            if (rem1 >= mine) {
+                rem1 -= mine;
+                ++k1;
+            }
+            cur_k_sh = k1;
+            cur_rem_sh = rem1;
         }
         is_q = k1 > k0;
         tile = is_q ? nq - 1 - (b + k0 * G) : ab + (jj - k0) * G;
-        cur_k = k1;
-        cur_rem = rem1;
     };
     auto issue = [&](int64_t jj) {   // thread 0, for jj = 0, 1, 2, ... in order
         bool is_q;

@@ -394,28 +394,29 @@ __device__ __forceinline__ uint32_t apply_winners(uint32_t w, uint32_t k)
 }
 
 
-// Weight-mode selection in running form: for each run of eight elements the
-// gains of 5 (from e = q - v when GE, else from v) and of 2.5, their sums and
-// signed sums, and a candidate marker
-// per element: the E2M1 code of sign(v) * gain * 2^40, +6 (0x7) for a
-// candidate of the positive member, -6 (0xF) of the negative one, +-0
-// otherwise.  Gains of 5 are multiples of 2^-20 up to 1 and gains of 2.5
-// multiples of 2^-22 up to 1/4, so every sum is exact in any order and the
-// comparisons are exact.  For either pair the better member's gain is
-// (U + |S|) / 2; the pair 2.5 is taken only when its gain is strictly larger,
-// and in a pair the negative member only when its gain is strictly larger
-// (ties go to the lower selector; a block with no gain keeps selector 0).  The
-// winners are the chosen value's candidates, found by flipping bit 3 of the
-// markers when the positive member wins.  Returns the chosen gain.
+// Weight-mode selection in running form.  w0, w1 hold the block's regular
+// codes.  For each run of eight elements: the gains of 5 (from e = q - v when
+// GE, else from v) and of 2.5, their sums and signed sums, and one candidate
+// marker per element for both pairs (no element is a candidate of both): the
+// E2M1 code of sign(v) * gain * 2^40, +6 (0x7) for a candidate of a positive
+// member, -6 (0xF) of a negative one, +-0 otherwise.  Gains of 5 are multiples
+// of 2^-20 up to 1 and gains of 2.5 multiples of 2^-22 up to 1/4, so every sum
+// is exact in any order and the comparisons are exact.  For either pair the
+// better member's gain is (U + |S|) / 2; the pair 2.5 is taken only when its
+// gain is strictly larger, and in a pair the negative member only when its
+// gain is strictly larger (ties go to the lower selector; a block with no gain
+// keeps selector 0).  The winners are the chosen value's candidates: markers
+// of the chosen sign (bit 3 flipped when the positive member wins) whose
+// element belongs to the chosen pair.  Returns the chosen gain.
 template <bool GE>
 __device__ __forceinline__ float razer_w_select(const float* v, const float* e, uint32_t& w0, uint32_t& w1,
                                                 uint32_t& sb)
 {
     float2 u5 = make_float2(0.0f, 0.0f), s5 = u5, u2 = u5, s2 = u5;
-    uint32_t k5[2], k2[2];
+    uint32_t k[2];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-        float x5[8], x2[8];
+        float x[8];
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
             const int j = 8 * hh + i;
@@ -434,23 +435,25 @@ __device__ __forceinline__ float razer_w_select(const float* v, const float* e, 
             s5 = add2_rn(s5, c5);
             u2 = add2_rn(u2, make_float2(h0, h1));
             s2 = add2_rn(s2, c2);
-            const float2 m5 = mul2_rn(c5, make_float2(0x1p40f, 0x1p40f));
-            const float2 m2 = mul2_rn(c2, make_float2(0x1p40f, 0x1p40f));
-            x5[i] = m5.x;
-            x5[i + 1] = m5.y;
-            x2[i] = m2.x;
-            x2[i + 1] = m2.y;
+            // one marker for both pairs: no element is a candidate of both, so
+            // at most one of c5, c2 is nonzero and their sum is exact
+            const float2 m = mul2_rn(add2_rn(c5, c2), make_float2(0x1p40f, 0x1p40f));
+            x[i] = m.x;
+            x[i + 1] = m.y;
         }
-        k5[hh] = e2m1x8(x5);
-        k2[hh] = e2m1x8(x2);
+        k[hh] = e2m1x8(x);
     }
     const float S5 = s5.x + s5.y, S2 = s2.x + s2.y;
     const float t5 = (u5.x + u5.y) + fabsf(S5), t2 = (u2.x + u2.y) + fabsf(S2);
     const bool p2 = t2 > t5;
     const bool neg = (p2 ? S2 : S5) < 0.0f;
     const uint32_t flip = neg ? 0u : 0x88888888u;
-    w0 = apply_winners(w0, (p2 ? k2[0] : k5[0]) ^ flip);
-    w1 = apply_winners(w1, (p2 ? k2[1] : k5[1]) ^ flip);
+    // The pair a candidate belongs to is bit 1 of its regular code's
+    // magnitude: 4 and 6 (codes 6, 7) for 5, 2 and 3 (codes 4, 5) for 2.5.
+    const uint32_t pm = p2 ? 0x11111111u : 0u;
+    // Bit 0 of a marker survives only where its element belongs to the chosen pair.
+    w0 = apply_winners(w0, (k[0] ^ flip) & ((((w0 >> 1) ^ pm) & 0x11111111u) | 0xEEEEEEEEu));
+    w1 = apply_winners(w1, (k[1] ^ flip) & ((((w1 >> 1) ^ pm) & 0x11111111u) | 0xEEEEEEEEu));
     sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
     return 0.5f * fmaxf(t5, t2);
 }
@@ -652,13 +655,15 @@ __device__ __forceinline__ void nv_block(const uint32_t* w, uint32_t a0, uint32_
 //    the E2M1 code of sign(v) * gain * 2^40, is +6 (0x7) for a candidate of
 //    +5, -6 (0xF) for one of -5 and +-0 otherwise;
 //  - the weight mode adds the pair 2.5 the same way (gain 1/4 - ||v| - 2.5|,
-//    multiples of 2^-22 up to 1/4; candidates of 2.5 and of 5 never overlap).
+//    multiples of 2^-22 up to 1/4).  Candidates of 2.5 and of 5 never
+//    overlap, so one marker word serves both pairs; bit 1 of an element's
+//    regular code magnitude tells which pair it is a candidate of.
 // The 2|e| - 1 form of the gain of 5 holds while |v| <= 6.5; blocks beyond
 // that take the exact path (nv_block_exact_f32), which forms gains from v.
 
 struct NvRun {
     uint32_t cw[2];          // code words, eight nibbles each
-    uint32_t k5[2], k2[2];   // candidate markers of 5 and (weight mode) of 2.5
+    uint32_t k[2];           // candidate markers of 5 and (weight mode) of 2.5
     float2 sq;               // sum of e^2, two lanes
     float2 u5, s5, u2, s2;   // sums of the gains and of the signed gains, two lanes
 };
@@ -692,28 +697,21 @@ __device__ __forceinline__ void nv_run8(const float* v, int h, NvRun& st)
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
             const float2 gg = make_float2(g[i], g[i + 1]);
-            const float2 cs = make_float2(copysignf(g[i], v[i]), copysignf(g[i + 1], v[i + 1]));
+            float2 cs = make_float2(copysignf(g[i], v[i]), copysignf(g[i + 1], v[i + 1]));
             st.u5 = add2_rn(st.u5, gg);
             st.s5 = add2_rn(st.s5, cs);
+            if (FMT == kRW) {
+                const float g0 = razer_gain_w2(v[i]), g1 = razer_gain_w2(v[i + 1]);
+                const float2 c2 = make_float2(copysignf(g0, v[i]), copysignf(g1, v[i + 1]));
+                st.u2 = add2_rn(st.u2, make_float2(g0, g1));
+                st.s2 = add2_rn(st.s2, c2);
+                cs = add2_rn(cs, c2);   // one marker for both pairs: no element is a candidate of both
+            }
             const float2 m = mul2_rn(cs, make_float2(0x1p40f, 0x1p40f));
             x[i] = m.x;
             x[i + 1] = m.y;
         }
-        st.k5[h] = e2m1x8(x);
-    }
-    if (FMT == kRW) {
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            const float g0 = razer_gain_w2(v[i]), g1 = razer_gain_w2(v[i + 1]);
-            const float2 cs = make_float2(copysignf(g0, v[i]), copysignf(g1, v[i + 1]));
-            st.u2 = add2_rn(st.u2, make_float2(g0, g1));
-            st.s2 = add2_rn(st.s2, cs);
-            const float2 m = mul2_rn(cs, make_float2(0x1p40f, 0x1p40f));
-            x[i] = m.x;
-            x[i + 1] = m.y;
-        }
-        st.k2[h] = e2m1x8(x);
+        st.k[h] = e2m1x8(x);
     }
 }
 
@@ -734,16 +732,17 @@ __device__ __forceinline__ float nv_finish(NvRun& st, uint32_t& sb)
     const float U5 = st.u5.x + st.u5.y, S5 = st.s5.x + st.s5.y;
     float G;
     bool neg;
-    uint32_t k0 = st.k5[0], k1 = st.k5[1];
+    uint32_t k0 = st.k[0], k1 = st.k[1];
     if (FMT == kRW) {
         const float U2 = st.u2.x + st.u2.y, S2 = st.s2.x + st.s2.y;
         const float t5 = U5 + fabsf(S5), t2 = U2 + fabsf(S2);
         const bool p2 = t2 > t5;
         neg = (p2 ? S2 : S5) < 0.0f;
-        if (p2) {
-            k0 = st.k2[0];
-            k1 = st.k2[1];
-        }
+        // Keep the markers of the chosen pair: bit 1 of the regular code's
+        // magnitude is set for 4 and 6 (candidates of 5), clear for 2 and 3.
+        const uint32_t pm = p2 ? 0x11111111u : 0u;
+        k0 &= (((st.cw[0] >> 1) ^ pm) & 0x11111111u) | 0xEEEEEEEEu;
+        k1 &= (((st.cw[1] >> 1) ^ pm) & 0x11111111u) | 0xEEEEEEEEu;
         sb |= (p2 ? 0x80u : 0u) | (neg ? 0x40u : 0u);
         G = 0.5f * fmaxf(t5, t2);
     } else {
