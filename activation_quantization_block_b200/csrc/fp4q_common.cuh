@@ -898,7 +898,7 @@ __device__ __forceinline__ void mx_block(const float* y, float a, bool ceil, uin
             cw[k] = canonical_zero(e2m1x8(v));
         }
     }
-    if (SSE) sse = a > 0.0f ? ldexp((double)(sq.x + sq.y), 2 * e) : 0.0;
+    if (SSE) sse = a > 0.0f ? (double)(sq.x + sq.y) * exp2i_f64(2 * e) : 0.0;   // 2e in [-254, 254]: exact
     sb_out = sb;
 }
 
@@ -1115,10 +1115,13 @@ __device__ __noinline__ BlockOut nv_block_redo(uint32_t tile, uint32_t r, uint32
     {
         uint32_t w[16];
         load_unit_words(tile, r, h, w);
-        unpack16(w, y);
-        unpack16(w + 8, y + 16);
+        if (ROT) {
+            wht32_from_bf16(w, y);
+        } else {
+            unpack16(w, y);
+            unpack16(w + 8, y + 16);
+        }
     }
-    if (ROT) wht32_inplace(y);
     const float* yb = half ? y + 16 : y;
     float a = 0.0f;
 #pragma unroll
@@ -1172,23 +1175,22 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
             {
                 uint32_t w[16];
                 load_unit_words(tile, r, h, w);
-                unpack16(w, y);
-                unpack16(w + 8, y + 16);
+                if (ROT) {
+                    wht32_from_bf16(w, y);
+                } else {
+                    unpack16(w, y);
+                    unpack16(w + 8, y + 16);
+                }
             }
-            if (ROT) wht32_inplace(y);
             if (FMT == kMX) {
-                float am = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(y[i]));
+                const float am = absmax_n<32>(y, 0.0f);
                 double e = 0.0;
                 mx_block<SSE>(y, am, mx_ceil, cw, sb0, e);
                 if (SSE) acc += e;
             } else {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    float am = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(y[16 * half + i]));
+                    const float am = absmax_n<16>(y + 16 * half, 0.0f);
                     uint32_t c0 = 0, c1 = 0, sbh = 0;
                     double e = 0.0;
                     if (!nv_block_f32<FMT, SSE>(y + 16 * half, am, nsc, c0, c1, sbh, e)) {
@@ -1236,11 +1238,8 @@ __device__ __forceinline__ float amax_tile(uint32_t tile)
     float m = 0.0f;
     if (ROT) {
         float y[32];
-        unpack16(w, y);
-        unpack16(w + 8, y + 16);
-        wht32_inplace(y);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(y[i]));
+        wht32_from_bf16(w, y);
+        m = absmax_n<32>(y, 0.0f);
     } else {
         uint32_t mm = w[0];
 #pragma unroll

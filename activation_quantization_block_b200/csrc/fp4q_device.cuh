@@ -256,6 +256,26 @@ __device__ __forceinline__ float exp2i(int k)
     return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
+// 2^k for k in [-1022, 1023] as fp64, from its exponent field.
+__device__ __forceinline__ double exp2i_f64(int k)
+{
+    return __longlong_as_double((long long)(k + 1023) << 52);
+}
+
+// max(|y_0|, ..., |y_{n-1}|, m) with three-input maxima.
+template <int N>
+__device__ __forceinline__ float absmax_n(const float* y, float m)
+{
+    int i = 0;
+#pragma unroll
+    for (; i + 1 < N; i += 2) {
+        const float a = fabsf(y[i]), b = fabsf(y[i + 1]);
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m), "f"(a), "f"(b));
+    }
+    if (i < N) m = fmaxf(m, fabsf(y[i]));
+    return m;
+}
+
 // ---- 32-point Walsh-Hadamard, in registers ----------------------------------
 
 // y <- H32 y (Sylvester order: H_ij = (-1)^popcount(i & j)), fp32 butterflies,
@@ -264,14 +284,10 @@ __device__ __forceinline__ float exp2i(int k)
 // pairs (y[i], y[i+1]) with (y[i+h], y[i+h+1]) and run two butterflies per
 // packed add / sub.  Every lane rounds as the scalar operation would, so the
 // result is the same bit for bit.
-__device__ __forceinline__ void wht32_inplace(float* y)
+// Butterfly stages of stride 2..16 and the 1/sqrt(32) scale (the stride-1
+// stage done).
+__device__ __forceinline__ void wht32_rest(float* y)
 {
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        const float a = y[i], b = y[i + 1];
-        y[i] = a + b;
-        y[i + 1] = a - b;
-    }
 #pragma unroll
     for (int h = 2; h < 32; h <<= 1) {
 #pragma unroll
@@ -293,6 +309,35 @@ __device__ __forceinline__ void wht32_inplace(float* y)
         y[i] = p.x;
         y[i + 1] = p.y;
     }
+}
+
+__device__ __forceinline__ void wht32_inplace(float* y)
+{
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        const float a = y[i], b = y[i + 1];
+        y[i] = a + b;
+        y[i + 1] = a - b;
+    }
+    wht32_rest(y);
+}
+
+// The same transform of the 32 bf16 values of w (element 2k in the low half
+// of w[k]): the stride-1 stage adds and subtracts each word's two values
+// straight from bf16 (add/sub.rn.f32.bf16 convert the bf16 operand exactly
+// and round once, as the fp32 add of the unpacked values does), which saves
+// unpacking the low halves.
+__device__ __forceinline__ void wht32_from_bf16(const uint32_t* w, float* y)
+{
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float hi = __uint_as_float(w[k] & 0xFFFF0000u);
+        asm("{\n\t.reg .b16 lo, up;\n\tmov.b32 {lo, up}, %2;\n\t"
+            "add.rn.f32.bf16 %0, lo, %3;\n\tsub.rn.f32.bf16 %1, lo, %3;\n\t}"
+            : "=f"(y[2 * k]), "=f"(y[2 * k + 1])
+            : "r"(w[k]), "f"(hi));
+    }
+    wht32_rest(y);
 }
 
 // ---- loads / stores -------------------------------------------------------
