@@ -33,6 +33,26 @@ namespace fp4q {
 
 constexpr int kRing = 3;   // rotating partial-buffer slots
 
+// CTA shape of the chain per format.  Twelve warps and tiles of 192 rows, two
+// CTAs per SM, measured faster than eight warps and 128 rows, three per SM,
+// except in the weight mode, whose encoder spills more in the larger CTA.
+// Thread t owns unit (row t / 2, half t % 2), so threads = 2 x rows.
+template <int FMT>
+struct ChainShape {
+    static constexpr int kRows = FMT == kRW ? 128 : 192;
+    static constexpr int kThreads = 2 * kRows;
+    static constexpr int kWarps = kThreads / 32;
+    static constexpr int kCtasPerSm = FMT == kRW ? 3 : 2;
+    static constexpr int kTileBytes = kRows * 128;
+    static constexpr int kSmemBytes = pipe_smem_bytes(kTileBytes);
+};
+
+inline int chain_rows(int fmt) { return fmt == kRW ? ChainShape<kRW>::kRows : ChainShape<kRZ>::kRows; }
+static_assert(ChainShape<kNV>::kRows == ChainShape<kRZ>::kRows && ChainShape<kMX>::kRows == ChainShape<kRZ>::kRows,
+              "chain_rows assumes one shape for every format but the weight mode");
+static_assert(ChainShape<kRZ>::kThreads <= 512 && ChainShape<kRW>::kThreads <= 512, "finaliser tree covers 512");
+static_assert(ChainShape<kRZ>::kRows <= 256, "TMA box rows");
+
 struct ChainArgs {
     // quantize part
     Tiles qtl;
@@ -58,16 +78,20 @@ struct ChainArgs {
 };
 
 template <int FMT, bool ROT, bool SSE>
-__global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
+__global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kCtasPerSm)
     chain_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap amap, ChainArgs a)
 {
+    using Shape = ChainShape<FMT>;
+    constexpr int kThreads = Shape::kThreads;
+    constexpr int kTileBytes = Shape::kTileBytes;
+    constexpr int kRows = Shape::kRows;
     extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
     __shared__ double shd[kThreads];
     __shared__ NvTable nvt;
     __shared__ int64_t slot_tile[kStages];   // item of each pipeline slot, decoded once by thread 0
     __shared__ int32_t slot_q[kStages];
-    const Pipe p = pipe_setup(smem_raw);
+    const Pipe p = pipe_setup<kTileBytes, Shape::kWarps>(smem_raw);
     const int t = threadIdx.x;
 
     // Items of this kernel: nq quantize tiles (walked backwards) and na absmax
@@ -126,11 +150,11 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
         slot_tile[s] = tile;
         int x, y;
         if (is_q) {
-            if (a.q_flat) tile_origin<true>(a.qtl, tile, x, y);
-            else tile_origin<false>(a.qtl, tile, x, y);
+            if (a.q_flat) tile_origin<true, kRows>(a.qtl, tile, x, y);
+            else tile_origin<false, kRows>(a.qtl, tile, x, y);
         } else {
-            if (a.a_flat) tile_origin<true>(a.atl, tile, x, y);
-            else tile_origin<false>(a.atl, tile, x, y);
+            if (a.a_flat) tile_origin<true, kRows>(a.atl, tile, x, y);
+            else tile_origin<false, kRows>(a.atl, tile, x, y);
         }
         mbar_arm(p.full + 8 * s, kTileBytes);
         tma_load_tile(p.tiles + s * kTileBytes, is_q ? &qmap : &amap, x, y, p.full + 8 * s);
@@ -161,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
             if (in_bounds(8 * (int64_t)i, 8, 8 * (int64_t)kMaxPartials, kSiteSsePartialLoad, a.err)) s += a.sse_in[i];
         shd[t] = s;
         __syncthreads();
-        for (int o = kThreads / 2; o > 0; o >>= 1) {
-            if (t < o) shd[t] += shd[t + o];
+        for (int o = 256; o > 0; o >>= 1) {   // fixed-order tree over kThreads <= 512 partial sums
+            if (t < o && t + o < kThreads) shd[t] += shd[t + o];
             __syncthreads();
         }
         if (t == 0) *a.fin_mse = a.fin_count > 0.0 ? shd[0] / a.fin_count : 0.0;
@@ -188,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm)
         const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
         if (is_q) {
             if (a.q_flat)
-                acc += quantize_tile<FMT, ROT, SSE, true>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0,
-                                                          a.err);
+                acc += quantize_tile<FMT, ROT, SSE, true, kRows>(tp, a.qtl, tile, a.codes, a.scales, nsc,
+                                                                 a.mx_ceil != 0, a.err);
             else
-                acc += quantize_tile<FMT, ROT, SSE, false>(tp, a.qtl, tile, a.codes, a.scales, nsc, a.mx_ceil != 0,
-                                                           a.err);
+                acc += quantize_tile<FMT, ROT, SSE, false, kRows>(tp, a.qtl, tile, a.codes, a.scales, nsc,
+                                                                  a.mx_ceil != 0, a.err);
         } else {
             m = fmaxf(m, amax_tile<ROT>(tp));
         }
@@ -225,10 +249,11 @@ template <int FMT, bool ROT, bool SSE>
 cudaError_t chain_go(const CUtensorMap& qmap, const CUtensorMap& amap, const ChainArgs& a, int64_t tiles, bool pdl,
                      int* grid_out, cudaStream_t st)
 {
+    using Shape = ChainShape<FMT>;
     auto kernel = chain_kernel<FMT, ROT, SSE>;
-    const int grid = grid_for(kernel, kPipeSmemBytes, tiles);
+    const int grid = grid_for(kernel, Shape::kSmemBytes, tiles, Shape::kThreads);
     *grid_out = grid;
-    return launch(kernel, grid, kPipeSmemBytes, pdl, st, qmap, amap, a);
+    return launch_threads(kernel, grid, Shape::kThreads, Shape::kSmemBytes, pdl, st, qmap, amap, a);
 }
 
 cudaError_t chain_dispatch(int fmt, bool rotate, bool sse, const CUtensorMap& qmap, const CUtensorMap& amap,
@@ -287,7 +312,8 @@ cudaError_t launch_quantize_batch(const BatchTensor* ts, int n, int fmt, int rot
     std::vector<View> views((size_t)n);
     for (int k = 0; k < n; ++k) {
         const Geometry g = make_geometry(ts[k].rows, ts[k].cols, ts[k].ldx);
-        if (!make_view(ts[k].x, g, &views[(size_t)k].map, &views[(size_t)k].tl)) return cudaErrorInvalidValue;
+        if (!make_view(ts[k].x, g, &views[(size_t)k].map, &views[(size_t)k].tl, chain_rows(fmt)))
+            return cudaErrorInvalidValue;
     }
     unsigned* err = device_error_words();
     if (err == nullptr) return cudaErrorInvalidSymbol;

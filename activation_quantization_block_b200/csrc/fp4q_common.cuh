@@ -54,16 +54,16 @@ struct Tiles {
     int64_t units;       // flat view: N / 32
 };
 
-template <bool FLAT>
+template <bool FLAT, int ROWS = kTileRows>
 __device__ __forceinline__ void tile_origin(const Tiles& tl, int64_t k, int& x, int& y)
 {
     if (FLAT) {
         x = 0;
-        y = (int)(k * kTileRows);
+        y = (int)(k * ROWS);
     } else {
         const int64_t rt = k / tl.col_tiles;
         x = (int)((k - rt * tl.col_tiles) * kTileCols);
-        y = (int)(rt * kTileRows);
+        y = (int)(rt * ROWS);
     }
 }
 
@@ -74,19 +74,19 @@ struct Unit {
     bool valid, full;
 };
 
-template <bool FLAT>
+template <bool FLAT, int ROWS = kTileRows>
 __device__ __forceinline__ Unit unit_of(const Tiles& tl, int64_t k, int t)
 {
     Unit u;
     if (FLAT) {
-        u.flat = k * (2 * kTileRows) + t;
+        u.flat = k * (2 * ROWS) + t;
         u.valid = u.flat < tl.units;
         u.full = true;
         u.row = u.col = 0;
     } else {
         const int64_t rt = k / tl.col_tiles;
         const int64_t ct = k - rt * tl.col_tiles;
-        u.row = rt * kTileRows + (t >> 1);
+        u.row = rt * ROWS + (t >> 1);
         u.col = ct * kTileCols + 32 * (t & 1);
         u.valid = u.row < tl.rows && u.col < tl.cols;
         u.full = u.col + 32 <= tl.cols;
@@ -995,7 +995,10 @@ __device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, c
 
 // Shared memory of a pipelined CTA: kStages tiles (1024-byte aligned for the
 // 128-byte swizzle), then a "full" and an "empty" mbarrier per stage.
-constexpr int kPipeSmemBytes = kStages * kTileBytes + 1024 + 128;
+// Dynamic shared memory of a pipeline of tiles of `tile_bytes`: the stages
+// (1024-byte aligned), the alignment slack and the barriers.
+constexpr int pipe_smem_bytes(int tile_bytes) { return kStages * tile_bytes + 1024 + 128; }
+constexpr int kPipeSmemBytes = pipe_smem_bytes(kTileBytes);
 constexpr int kWarps = kThreads / 32;
 
 // Stage s is "full" when its copy has landed (one arrival by thread 0 with the
@@ -1008,18 +1011,19 @@ struct Pipe {
     uint32_t empty;   // shared address of the empty barriers
 };
 
+template <int TILE_BYTES = kTileBytes, int WARPS = kWarps>
 __device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
 {
     const uint32_t base = smem_u32(smem_raw);
     Pipe p;
     p.tiles = (base + 1023u) & ~1023u;
-    p.full = p.tiles + kStages * kTileBytes;
+    p.full = p.tiles + kStages * TILE_BYTES;
     p.empty = p.full + 8 * kStages;
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int s = 0; s < kStages; ++s) {
             mbar_init(p.full + 8 * s, 1);
-            mbar_init(p.empty + 8 * s, kWarps);
+            mbar_init(p.empty + 8 * s, WARPS);
         }
         mbar_init_fence();
     }
@@ -1140,7 +1144,7 @@ __device__ __noinline__ BlockOut nv_block_redo(uint32_t tile, uint32_t r, uint32
 // transform H / sqrt(32) maps onto the original one up to the fp32 rounding of
 // the rotated values (about 2^-24 of each value, far inside the rotated
 // paths' 1e-3 MSE tolerance).
-template <int FMT, bool ROT, bool SSE, bool FLAT>
+template <int FMT, bool ROT, bool SSE, bool FLAT, int ROWS = kTileRows>
 __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, int64_t k, uint8_t* codes,
                                                 uint8_t* scales, const NvScale& nsc, bool mx_ceil, unsigned* err)
 {
@@ -1148,7 +1152,7 @@ __device__ __forceinline__ double quantize_tile(uint32_t tile, const Tiles& tl, 
     const bool a16 = FLAT || (tl.cols % 32) == 0;
     const uint32_t r = (uint32_t)t >> 1, h = (uint32_t)t & 1u;
     double acc = 0.0;
-    const Unit u = unit_of<FLAT>(tl, k, t);
+    const Unit u = unit_of<FLAT, ROWS>(tl, k, t);
     uint32_t cw[4] = {0, 0, 0, 0}, sb0 = 0, sb1 = 0;
     if (u.valid) {
         if (FMT != kMX && !ROT) {
