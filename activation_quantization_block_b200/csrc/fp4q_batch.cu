@@ -33,23 +33,27 @@ namespace fp4q {
 
 constexpr int kRing = 3;   // rotating partial-buffer slots
 
-// CTA shape of the chain per format.  Twelve warps and tiles of 192 rows, two
-// CTAs per SM, measured faster than eight warps and 128 rows, three per SM,
-// except in the weight mode, whose encoder spills more in the larger CTA.
-// Thread t owns unit (row t / 2, half t % 2), so threads = 2 x rows.
+// CTA shape of the chain: ten warps and tiles of 160 rows (20 KB), two CTAs
+// per SM with up to 96 registers a thread, measured faster in every format
+// than eight warps and 128 rows at three CTAs per SM (80 registers, where the
+// RaZeR encoders spill) and than twelve warps and 192 rows at two per SM.
+// Thread t owns unit (row t / 2, half t % 2), so threads = 2 x rows.  The
+// shape is a parameter of the format so that one format can move alone.
 template <int FMT>
 struct ChainShape {
-    static constexpr int kRows = FMT == kRW ? 128 : 192;
+    static constexpr int kRows = 160;
     static constexpr int kThreads = 2 * kRows;
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int kCtasPerSm = FMT == kRW ? 3 : 2;
+    static constexpr int kCtasPerSm = 2;
     static constexpr int kTileBytes = kRows * 128;
     static constexpr int kSmemBytes = pipe_smem_bytes(kTileBytes);
 };
 
 inline int chain_rows(int fmt) { return fmt == kRW ? ChainShape<kRW>::kRows : ChainShape<kRZ>::kRows; }
 static_assert(ChainShape<kNV>::kRows == ChainShape<kRZ>::kRows && ChainShape<kMX>::kRows == ChainShape<kRZ>::kRows,
-              "chain_rows assumes one shape for every format but the weight mode");
+              "chain_rows gives the weight mode its own shape and one shape to the other formats");
+static_assert(ChainShape<kRZ>::kRows % 8 == 0 && ChainShape<kRW>::kRows % 8 == 0,
+              "a tile is whole 1024-byte swizzle atoms of 8 rows");
 static_assert(ChainShape<kRZ>::kThreads <= 512 && ChainShape<kRW>::kThreads <= 512, "finaliser tree covers 512");
 static_assert(ChainShape<kRZ>::kRows <= 256, "TMA box rows");
 
