@@ -45,8 +45,9 @@ struct ChainShape {
     static constexpr int kThreads = 2 * kRows;
     static constexpr int kWarps = kThreads / 32;
     static constexpr int kCtasPerSm = 2;
+    static constexpr int kStages = 4;
     static constexpr int kTileBytes = kRows * 128;
-    static constexpr int kSmemBytes = pipe_smem_bytes(kTileBytes);
+    static constexpr int kSmemBytes = pipe_smem_bytes(kTileBytes, kStages);
 };
 
 inline int chain_rows(int fmt) { return fmt == kRW ? ChainShape<kRW>::kRows : ChainShape<kRZ>::kRows; }
@@ -89,13 +90,14 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     constexpr int kThreads = Shape::kThreads;
     constexpr int kTileBytes = Shape::kTileBytes;
     constexpr int kRows = Shape::kRows;
+    constexpr int kStages = Shape::kStages;
     extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
     __shared__ double shd[kThreads];
     __shared__ NvTable nvt;
     __shared__ int64_t slot_tile[kStages];   // item of each pipeline slot, decoded once by thread 0
     __shared__ int32_t slot_q[kStages];
-    const Pipe p = pipe_setup<kTileBytes, Shape::kWarps>(smem_raw);
+    const Pipe p = pipe_setup<kTileBytes, Shape::kWarps, kStages>(smem_raw);
     const int t = threadIdx.x;
 
     // Items of this kernel: nq quantize tiles (walked backwards) and na absmax
@@ -113,36 +115,17 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     // Thread 0 walks the items in order: before item jj come k = floor(jj my_q /
     // mine) quantize items, stepped without a division (rem = jj my_q - k mine,
     // in [0, mine); my_q <= mine, so one step adds at most one).  Only thread 0
-    // uses the cursor.  Kept in shared memory it costs the encoder no registers;
-    // kept in registers it saves thread 0 a shared-memory round trip per refill.
-    // The weight mode measured faster with registers, the other formats with
-    // shared memory.
-    constexpr bool kCursorInRegs = FMT == kRW;
-    __shared__ int64_t cur_k_sh, cur_rem_sh;
-    int cur_k_r = 0, cur_rem_r = 0;   // fits: a tensor in device memory has fewer than 2^24 tiles
-    if (!kCursorInRegs && t == 0) cur_k_sh = cur_rem_sh = 0;
+    // uses the cursor; it stays in registers (a shared-memory cursor, which
+    // spares the encoder two registers, measured slower at 96 registers).
+    int cur_k = 0, cur_rem = 0;   // fits: a tensor in device memory has fewer than 2^24 tiles
     auto next_item = [&](int64_t jj, bool& is_q, int64_t& tile) {
-        int64_t k0, k1;
-        if constexpr (kCursorInRegs) {
-            k0 = cur_k_r;
-            cur_rem_r += (int)my_q;
-            if (cur_rem_r >= (int)mine) {
-                cur_rem_r -= (int)mine;
-                ++cur_k_r;
-            }
-            k1 = cur_k_r;
-        } else {
-            k0 = cur_k_sh;
-            k1 = k0;
-            int64_t rem1 = cur_rem_sh + my_q;
-            if (rem1 >= mine) {
-                rem1 -= mine;
-                ++k1;
-            }
-            cur_k_sh = k1;
-            cur_rem_sh = rem1;
+        const int64_t k0 = cur_k;
+        cur_rem += (int)my_q;
+        if (cur_rem >= (int)mine) {
+            cur_rem -= (int)mine;
+            ++cur_k;
         }
-        is_q = k1 > k0;
+        is_q = cur_k > k0;
         tile = is_q ? nq - 1 - (b + k0 * G) : ab + (jj - k0) * G;
     };
     auto issue = [&](int64_t jj) {   // thread 0, for jj = 0, 1, 2, ... in order
@@ -206,8 +189,8 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     double acc = 0.0;
     float m = 0.0f;
     for (int64_t jj = 0; jj < mine; ++jj) {
-        if (!pipe_acquire(p, jj)) {
-            pipe_fail(p, jj, jj + kStages < mine ? jj + kStages : mine, a.err);
+        if (!pipe_acquire<kStages>(p, jj)) {
+            pipe_fail<kStages>(p, jj, jj + kStages < mine ? jj + kStages : mine, a.err);
             break;
         }
         const int s = (int)(jj % kStages);
@@ -224,10 +207,10 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
         } else {
             m = fmaxf(m, amax_tile<ROT>(tp));
         }
-        pipe_release(p, jj);
+        pipe_release<kStages>(p, jj);
         if (t == 0 && jj + kStages < mine) {
-            if (!pipe_stage_free(p, jj)) {
-                pipe_fail(p, jj + 1, jj + kStages, a.err);
+            if (!pipe_stage_free<kStages>(p, jj)) {
+                pipe_fail<kStages>(p, jj + 1, jj + kStages, a.err);
                 break;
             }
             issue(jj + kStages);

@@ -997,7 +997,7 @@ __device__ __forceinline__ void load_packed(const uint8_t* __restrict__ codes, c
 // 128-byte swizzle), then a "full" and an "empty" mbarrier per stage.
 // Dynamic shared memory of a pipeline of tiles of `tile_bytes`: the stages
 // (1024-byte aligned), the alignment slack and the barriers.
-constexpr int pipe_smem_bytes(int tile_bytes) { return kStages * tile_bytes + 1024 + 128; }
+constexpr int pipe_smem_bytes(int tile_bytes, int stages = kStages) { return stages * tile_bytes + 1024 + 128; }
 constexpr int kPipeSmemBytes = pipe_smem_bytes(kTileBytes);
 constexpr int kWarps = kThreads / 32;
 
@@ -1011,17 +1011,17 @@ struct Pipe {
     uint32_t empty;   // shared address of the empty barriers
 };
 
-template <int TILE_BYTES = kTileBytes, int WARPS = kWarps>
+template <int TILE_BYTES = kTileBytes, int WARPS = kWarps, int STAGES = kStages>
 __device__ __forceinline__ Pipe pipe_setup(uint8_t* smem_raw)
 {
     const uint32_t base = smem_u32(smem_raw);
     Pipe p;
     p.tiles = (base + 1023u) & ~1023u;
-    p.full = p.tiles + kStages * TILE_BYTES;
-    p.empty = p.full + 8 * kStages;
+    p.full = p.tiles + STAGES * TILE_BYTES;
+    p.empty = p.full + 8 * STAGES;
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(p.full + 8 * s, 1);
             mbar_init(p.empty + 8 * s, WARPS);
         }
@@ -1064,33 +1064,37 @@ __device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map
 }
 
 // Every thread: wait (bounded) until the j-th tile has landed.
+template <int STAGES = kStages>
 __device__ __forceinline__ bool pipe_acquire(const Pipe& p, int64_t j)
 {
-    return mbar_wait(p.full + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+    return mbar_wait(p.full + 8 * (int)(j % STAGES), (uint32_t)((j / STAGES) & 1));
 }
 
 // Every warp, after its last read of the j-th tile: release the stage.
+template <int STAGES = kStages>
 __device__ __forceinline__ void pipe_release(const Pipe& p, int64_t j)
 {
     __syncwarp();
     if ((threadIdx.x & 31) == 0)
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(p.empty + 8 * (int)(j % kStages)) : "memory");
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(p.empty + 8 * (int)(j % STAGES)) : "memory");
 }
 
 // Thread 0: wait (bounded) until every warp has released the j-th tile's stage.
+template <int STAGES = kStages>
 __device__ __forceinline__ bool pipe_stage_free(const Pipe& p, int64_t j)
 {
-    return mbar_wait(p.empty + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1));
+    return mbar_wait(p.empty + 8 * (int)(j % STAGES), (uint32_t)((j / STAGES) & 1));
 }
 
 // After a timeout: record it in the error words `err`; thread 0 waits
 // (bounded) for the copies it issued that may still be in flight, tiles
 // [from, to) of the schedule.
+template <int STAGES = kStages>
 __device__ __forceinline__ void pipe_fail(const Pipe& p, int64_t from, int64_t to, unsigned* err)
 {
     if ((threadIdx.x & 31) == 0) atomicOr(err, kErrPipelineTimeout);
     if (threadIdx.x == 0)
-        for (int64_t q = from; q < to; ++q) pipe_acquire(p, q);
+        for (int64_t q = from; q < to; ++q) pipe_acquire<STAGES>(p, q);
 }
 
 __device__ __forceinline__ void load_unit_words(uint32_t tile, uint32_t r, uint32_t h, uint32_t* w)
