@@ -95,8 +95,6 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     __shared__ float shf[32];
     __shared__ double shd[kThreads];
     __shared__ NvTable nvt;
-    __shared__ int64_t slot_tile[kStages];   // item of each pipeline slot, decoded once by thread 0
-    __shared__ int32_t slot_q[kStages];
     const Pipe p = pipe_setup<kTileBytes, Shape::kWarps, kStages>(smem_raw);
     const int t = threadIdx.x;
 
@@ -112,11 +110,12 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     const int64_t my_q = b < nq ? (nq - 1 - b) / G + 1 : 0;
     const int64_t my_a = ab < na ? (na - 1 - ab) / G + 1 : 0;
     const int64_t mine = my_q + my_a;
-    // Thread 0 walks the items in order: before item jj come k = floor(jj my_q /
-    // mine) quantize items, stepped without a division (rem = jj my_q - k mine,
-    // in [0, mine); my_q <= mine, so one step adds at most one).  Only thread 0
-    // uses the cursor; it stays in registers (a shared-memory cursor, which
-    // spares the encoder two registers, measured slower at 96 registers).
+    // The items in order: before item jj come k = floor(jj my_q / mine)
+    // quantize items, stepped without a division (rem = jj my_q - k mine, in
+    // [0, mine); my_q <= mine, so one step adds at most one).  Thread 0 walks
+    // the list kStages items ahead for the refills, and every thread walks its
+    // own copy as it consumes the items, all in registers (item slots in shared
+    // memory, or a shared-memory cursor, measured slower at 96 registers).
     int cur_k = 0, cur_rem = 0;   // fits: a tensor in device memory has fewer than 2^24 tiles
     auto next_item = [&](int64_t jj, bool& is_q, int64_t& tile) {
         const int64_t k0 = cur_k;
@@ -133,8 +132,6 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
         int64_t tile;
         next_item(jj, is_q, tile);
         const int s = (int)(jj % kStages);
-        slot_q[s] = is_q ? 1 : 0;
-        slot_tile[s] = tile;
         int x, y;
         if (is_q) {
             if (a.q_flat) tile_origin<true, kRows>(a.qtl, tile, x, y);
@@ -181,21 +178,26 @@ __global__ void __launch_bounds__(ChainShape<FMT>::kThreads, ChainShape<FMT>::kC
     pdl_trigger();
     NvScale nsc{};
     if (a.has_q && FMT != kMX) nsc = nv_scale_setup<FMT>(s_t, &nvt);
-    // The first items, written by thread 0, are visible after this barrier; a
-    // refill's item is written before thread 0 arms its stage, and the
-    // consumers' acquire of the landed phase makes it visible.
+    // Every thread finishes the prologue before the tile loop.
     __syncthreads();
 
     double acc = 0.0;
     float m = 0.0f;
+    int ck = 0, crem = 0;   // this thread's copy of the item walk
     for (int64_t jj = 0; jj < mine; ++jj) {
         if (!pipe_acquire<kStages>(p, jj)) {
             pipe_fail<kStages>(p, jj, jj + kStages < mine ? jj + kStages : mine, a.err);
             break;
         }
         const int s = (int)(jj % kStages);
-        const bool is_q = slot_q[s] != 0;
-        const int64_t tile = slot_tile[s];
+        const int ck0 = ck;
+        crem += (int)my_q;
+        if (crem >= (int)mine) {
+            crem -= (int)mine;
+            ++ck;
+        }
+        const bool is_q = ck > ck0;
+        const int64_t tile = nq - 1 - (b + (int64_t)ck0 * G);   // used for quantize items only
         const uint32_t tp = p.tiles + (uint32_t)s * kTileBytes;
         if (is_q) {
             if (a.q_flat)
