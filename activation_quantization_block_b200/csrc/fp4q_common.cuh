@@ -1052,15 +1052,16 @@ __device__ __forceinline__ Schedule make_schedule(int64_t count, bool reverse)
 }
 
 // Thread 0: start the copy of the j-th tile of the schedule into its stage.
-template <bool FLAT>
+template <bool FLAT, int ROWS = kTileRows>
 __device__ __forceinline__ void pipe_issue(const Pipe& p, const CUtensorMap* map, const Tiles& tl, const Schedule& sc,
                                            int64_t j)
 {
+    constexpr int kBytes = ROWS * 128;
     const int s = (int)(j % kStages);
     int x, y;
-    tile_origin<FLAT>(tl, sc.tile(j), x, y);
-    mbar_arm(p.full + 8 * s, kTileBytes);
-    tma_load_tile(p.tiles + s * kTileBytes, map, x, y, p.full + 8 * s);
+    tile_origin<FLAT, ROWS>(tl, sc.tile(j), x, y);
+    mbar_arm(p.full + 8 * s, kBytes);
+    tma_load_tile(p.tiles + s * kBytes, map, x, y, p.full + 8 * s);
 }
 
 // Every thread: wait (bounded) until the j-th tile has landed.

@@ -97,20 +97,45 @@ struct QuantArgs {
     unsigned* err;          // the library's device error words
 };
 
+// CTA shape of the quantize pass per format.  NVFP4 and the RaZeR weight
+// mode measured faster with ten warps, tiles of 160 rows (20 KB) and two CTAs
+// per SM (up to 96 registers a thread); RaZeR and MXFP4 keep eight warps,
+// 128-row tiles and three CTAs per SM.  Thread t owns unit (row t / 2, half
+// t % 2), so threads = 2 x rows.
+template <int FMT>
+struct QuantShape {
+    static constexpr bool kWide = FMT == kNV || FMT == kRW;
+    static constexpr int kRows = kWide ? 160 : kTileRows;
+    static constexpr int kThreads = 2 * kRows;
+    static constexpr int kWarps = kThreads / 32;
+    static constexpr int kCtasPerSm = kWide ? 2 : kTileCtasPerSm;
+    static constexpr int kTileBytes = kRows * 128;
+    static constexpr int kSmemBytes = pipe_smem_bytes(kTileBytes);
+};
+static_assert(QuantShape<kRZ>::kThreads == kThreads && QuantShape<kMX>::kThreads == kThreads,
+              "RaZeR and MXFP4 keep the streaming kernels' shape");
+
+inline int quant_rows(int fmt) { return (fmt == kNV || fmt == kRW) ? QuantShape<kNV>::kRows : kTileRows; }
+
 // Q1-Q6: rotate, block scale, encode, RaZeR select, pack, store, SSE partials.
 template <int FMT, bool ROT, bool SSE, bool FLAT>
-__global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a)
+__global__ void __launch_bounds__(QuantShape<FMT>::kThreads, QuantShape<FMT>::kCtasPerSm)
+    quantize_kernel(const __grid_constant__ CUtensorMap xmap, QuantArgs a)
 {
+    using Shape = QuantShape<FMT>;
+    constexpr int kThreads = Shape::kThreads;
+    constexpr int kRows = Shape::kRows;
+    constexpr int kTileBytes = Shape::kTileBytes;
     extern __shared__ uint8_t smem_raw[];
     __shared__ float shf[32];
     __shared__ double shd[32];
-    const Pipe p = pipe_setup(smem_raw);
+    const Pipe p = pipe_setup<kTileBytes, Shape::kWarps>(smem_raw);
     const Schedule sc = make_schedule(a.tl.count, a.reverse != 0);
     const int t = threadIdx.x;
     // x was complete before the preceding kernel of this call started, so the
     // first tiles may be fetched before waiting for that kernel.
     if (t == 0)
-        for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT>(p, &xmap, a.tl, sc, j);
+        for (int64_t j = 0; j < sc.mine && j < kStages; ++j) pipe_issue<FLAT, kRows>(p, &xmap, a.tl, sc, j);
     pdl_wait();
 
     // Tensor scale (NVFP4 formats): s_t = RN(A / (6 * 448)), or RN(A / (6 * 30))
@@ -140,15 +165,15 @@ __global__ void __launch_bounds__(kThreads, kTileCtasPerSm) quantize_kernel(cons
             break;
         }
         const uint32_t tile = p.tiles + (uint32_t)(j % kStages) * kTileBytes;
-        acc += quantize_tile<FMT, ROT, SSE, FLAT>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc, a.mx_ceil != 0,
-                                                  a.err);
+        acc += quantize_tile<FMT, ROT, SSE, FLAT, kRows>(tile, a.tl, sc.tile(j), a.codes, a.scales, nsc,
+                                                         a.mx_ceil != 0, a.err);
         pipe_release(p, j);
         if (t == 0 && j + kStages < sc.mine) {
             if (!pipe_stage_free(p, j)) {
                 pipe_fail(p, j + 1, j + kStages, a.err);
                 break;
             }
-            pipe_issue<FLAT>(p, &xmap, a.tl, sc, j + kStages);
+            pipe_issue<FLAT, kRows>(p, &xmap, a.tl, sc, j + kStages);
         }
     }
     if (SSE) {
@@ -343,10 +368,11 @@ template <int FMT, bool ROT>
 static cudaError_t quantize_dispatch(const CUtensorMap& map, const QuantArgs& a, bool sse, bool pdl, int* grid_out,
                                      cudaStream_t st)
 {
+    using Shape = QuantShape<FMT>;
     auto go = [&](auto kernel) {
-        const int grid = grid_for(kernel, kPipeSmemBytes, a.tl.count);
+        const int grid = grid_for(kernel, Shape::kSmemBytes, a.tl.count, Shape::kThreads);
         if (grid_out) *grid_out = grid;
-        return launch(kernel, grid, kPipeSmemBytes, pdl, st, map, a);
+        return launch_threads(kernel, grid, Shape::kThreads, Shape::kSmemBytes, pdl, st, map, a);
     };
     const bool flat = is_flat(a.tl);
     if (sse) return flat ? go(quantize_kernel<FMT, ROT, true, true>) : go(quantize_kernel<FMT, ROT, true, false>);
@@ -360,7 +386,7 @@ cudaError_t launch_quantize(const uint16_t* x, const Geometry& g, int fmt, int r
 {
     CUtensorMap map;
     QuantArgs a;
-    if (!make_view(x, g, &map, &a.tl)) return cudaErrorInvalidValue;
+    if (!make_view(x, g, &map, &a.tl, quant_rows(fmt))) return cudaErrorInvalidValue;
     if ((a.err = device_error_words()) == nullptr) return cudaErrorInvalidSymbol;
     a.codes = codes;
     a.scales = scales;
